@@ -1,0 +1,237 @@
+/*
+ * pagedattn.h -- C ABI of the paged KV-cache decode library (libpagedattn.so).
+ *
+ * Decode attention over a KV cache cut into fixed-size physical blocks that
+ * are scattered through a pooled cache and reached through a per-sequence
+ * block table (logical block i -> physical block id).  Sources, by page
+ * title and section:
+ *   [csdn-QA] "VLLM中PagedAttention如何降低显存碎片？" (ask.csdn.net), sections 二-四
+ *   [tech]    "PagedAttention技术解析：优化Transformer显存管理", sections 2.1-4.2
+ *   [course]  "vLLM内存管理与PagedAttention精讲", chapter 2, sections 2.2-2.5
+ *
+ * Conventions for every call below
+ *   - Pointers named *_d are DEVICE pointers owned by the caller (for
+ *     example PyTorch tensors).  Tensors are dense, row-major, with the
+ *     shapes given.  Device pointers passed to the attention and cache
+ *     calls must be 16-byte aligned.  The library never allocates device
+ *     memory; split decode takes a caller-owned workspace.
+ *   - Every device call is asynchronous on `stream` (NULL = legacy default
+ *     stream) and returns a pa_status describing argument checks and the
+ *     launch only.  Faults found by the kernels' own bounds checks or
+ *     bounded waits are recorded in a device-side error word that
+ *     pa_device_error() reads.
+ *   - On any non-PA_OK status pa_last_error() returns a message (thread
+ *     local, valid until the next call on that thread).
+ *   - Cache layout: k_cache and v_cache are two tensors
+ *     [num_blocks, block_size, num_kv_heads, head_dim]: a block holds
+ *     block_size tokens, each with its key (value) for every kv head and
+ *     every dimension ([course] 2.3; [csdn-QA] 三, separate K and V pages).
+ *     Bytes per block, K plus V: block_size * num_kv_heads * head_dim * 2 *
+ *     element size ([course] 2.3).
+ *   - Supported: dtype f32 or bf16 (q, key/value rows, caches and outputs
+ *     share one dtype; arithmetic is fp32), head_dim in {64, 128, 256},
+ *     block_size in {8, 16, 32}, num_heads / num_kv_heads in {1, 2, 4, 8}.
+ *     Anything else returns PA_ERR_UNSUPPORTED.
+ *   - Validation: with PA_VALIDATE=1 in the environment (or
+ *     pa_set_option(PA_OPT_VALIDATE, 1)) the calls first copy the index
+ *     arrays to the host (synchronising `stream`) and return
+ *     PA_ERR_BAD_BLOCK_ID for a block id outside [0, num_blocks), a
+ *     context length above max_blocks_per_seq * block_size, a slot outside
+ *     the pool, or a repeated copy destination.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,     /* null pointer, negative size, misalignment, Hq % Hk != 0 */
+    PA_ERR_UNSUPPORTED = 2,     /* dtype / head_dim / block_size / group size not built */
+    PA_ERR_OUT_OF_BLOCKS = 3,   /* allocator: free pool exhausted, state unchanged */
+    PA_ERR_BAD_BLOCK_ID = 4,    /* validation: index outside the pool or table */
+    PA_ERR_CUDA = 5,            /* a CUDA runtime / driver call failed */
+    PA_ERR_DEVICE_CHECK = 6     /* pa_device_error(): a kernel's own check fired */
+} pa_status;
+
+typedef enum pa_dtype { PA_DTYPE_F32 = 0, PA_DTYPE_BF16 = 1 } pa_dtype;
+
+/* Bits of the device-side error word (pa_device_error). */
+enum {
+    PA_DEVERR_BLOCK_ID = 1u,     /* decode met a table entry outside [0, num_blocks) */
+    PA_DEVERR_CONTEXT_LEN = 2u,  /* context length beyond the table; clamped */
+    PA_DEVERR_WAIT_TIMEOUT = 4u, /* a bounded pipeline wait gave up */
+    PA_DEVERR_SLOT = 8u,         /* reshape_and_cache slot outside the pool; row skipped */
+    PA_DEVERR_COPY_ID = 16u,     /* copy_blocks pair outside the pool; pair skipped */
+    PA_DEVERR_WORKSPACE = 32u    /* split decode: more partitions than the workspace holds */
+};
+
+typedef enum pa_option {
+    PA_OPT_VALIDATE = 0,         /* 0/1: host-side index validation before launch */
+    PA_OPT_DECODE_SPLIT_CTAS = 1 /* pa_decode CTAs per (sequence, kv head): 0 = auto, 1, 2, 4, 8 */
+} pa_option;
+
+const char* pa_last_error(void);
+const char* pa_status_string(pa_status status);
+int         pa_version(void);
+pa_status   pa_set_option(pa_option option, int value);
+int         pa_get_option(pa_option option);
+
+/* Synchronise `stream`, return the device error word in *flags (0 = none)
+ * and clear it when `clear` is non-zero.  Returns PA_ERR_DEVICE_CHECK when
+ * the word is non-zero. */
+pa_status pa_device_error(pa_stream_t stream, uint32_t* flags, int clear);
+
+/*
+ * pa_reshape_and_cache -- write new tokens' keys and values into the cache.
+ * A generated token's K/V rows go into the slot its sequence's newest block
+ * assigns to it ([course] 2.4.2: a new block only when the current one is
+ * full; [csdn-QA] 四 flow: allocate a free page, update the mapping).
+ *   key_d, value_d   [num_tokens, num_kv_heads, head_dim], dtype
+ *   k_cache_d, v_cache_d  [num_blocks, block_size, num_kv_heads, head_dim]
+ *   slot_mapping_d   int64 [num_tokens]: slot = block * block_size + row;
+ *                    -1 skips the token.  Duplicate slots race (undefined).
+ * The copy is exact (no conversion).  A slot >= num_blocks * block_size is
+ * skipped and sets PA_DEVERR_SLOT.
+ */
+pa_status pa_reshape_and_cache(const void* key_d, const void* value_d,
+                               void* k_cache_d, void* v_cache_d,
+                               const int64_t* slot_mapping_d, int num_tokens,
+                               int num_kv_heads, int head_dim, int block_size,
+                               int num_blocks, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_decode -- one decode step of attention over the paged cache.
+ * For each sequence s and query head h (kv head h / (num_heads/num_kv_heads)):
+ *   out[s,h] = sum_t softmax_t(scale * <q[s,h], K_s[t]>) V_s[t],
+ * t over the sequence's context_lens[s] tokens, token t read from physical
+ * block block_tables[s, t / block_size] at row t % block_size ([course] 2.2
+ * mapping, 2.5 block-wise loop; [csdn-QA] 三 items 4, 9).  The kernel walks
+ * the blocks with an online (running max / running sum) softmax, which
+ * reaches the same result as the plain softmax.
+ *   out_d            [num_seqs, num_heads, head_dim], dtype (written)
+ *   q_d              [num_seqs, num_heads, head_dim], dtype
+ *   block_tables_d   int32 [num_seqs, max_blocks_per_seq]; only the first
+ *                    ceil(context_lens[s] / block_size) entries are read
+ *   context_lens_d   int32 [num_seqs]; 0 gives a zero output row
+ * No workspace: a (sequence, kv head) may be split over a cluster of CTAs
+ * that merge through distributed shared memory.
+ */
+pa_status pa_decode(void* out_d, const void* q_d,
+                    const void* k_cache_d, const void* v_cache_d,
+                    const int32_t* block_tables_d, int max_blocks_per_seq,
+                    const int32_t* context_lens_d, int num_seqs, int num_heads,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                    float scale, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_decode_split -- long-context decode in fixed token partitions merged by
+ * log-sum-exp ("PagedAttention V2 ... block-wise computation",
+ * [csdn-QA] 四, last paragraph; sequences up to 1M tokens, [tech] 1).
+ * Partition p of sequence s covers tokens [p*P, min((p+1)*P, L_s)) with
+ * P = partition_size (a multiple of block_size).  A first kernel writes per
+ * (sequence, head, partition) the running max, the sum of exponentials and
+ * the unnormalised output into `workspace_d`; a second kernel merges them:
+ *   out = sum_p exp(m_p - M) o_p / sum_p exp(m_p - M) l_p,  M = max_p m_p.
+ * Sequences with a single partition are written directly by the first kernel.
+ *   max_context_len  >= every context_lens[s]; sizes the workspace
+ *   workspace_d      caller-owned device memory of at least
+ *                    pa_decode_split_workspace_bytes(...) bytes, 16-byte aligned
+ * Other arguments as pa_decode.
+ */
+size_t pa_decode_split_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                       int max_context_len, int partition_size);
+
+pa_status pa_decode_split(void* out_d, const void* q_d,
+                          const void* k_cache_d, const void* v_cache_d,
+                          const int32_t* block_tables_d, int max_blocks_per_seq,
+                          const int32_t* context_lens_d, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                          float scale, pa_dtype dtype, int max_context_len,
+                          int partition_size, void* workspace_d, size_t workspace_bytes,
+                          pa_stream_t stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write of shared blocks: for each pair
+ * (src, dst) the whole key block and value block dst <- src ([course] 2.4.3:
+ * a write to a block whose reference count exceeds one first copies it).
+ *   block_mapping_d  int64 [num_pairs, 2] (src, dst), device memory.
+ * Destinations must be distinct and must not be sources (else undefined).
+ * An id outside the pool skips the pair and sets PA_DEVERR_COPY_ID.
+ */
+pa_status pa_copy_blocks(void* k_cache_d, void* v_cache_d,
+                         const int64_t* block_mapping_d, int num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                         pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * Host block allocator ([tech] 2.1 Block {ref_count, is_allocated} and the
+ * pool descriptor, 4.2 immediate reclamation at ref_count 0 and a free pool;
+ * [csdn-QA] 三 item 7 slab-style frames, item 8 shared prefix pages;
+ * [course] 2.4 on-demand growth, sharing, copy-on-write).
+ * Host memory only; not thread-safe; the caller owns the handle.
+ * The free pool is a stack: it starts as initial_free_order (element 0 is
+ * handed out first; NULL = 0, 1, ..., num_blocks-1) and a block whose
+ * count reaches 0 is pushed on top.  Failing calls change nothing.
+ */
+typedef struct pa_allocator pa_allocator;
+
+pa_allocator* pa_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_order);
+void      pa_alloc_destroy(pa_allocator* alloc);
+pa_status pa_alloc_allocate(pa_allocator* alloc, int32_t* block_out);  /* ref := 1 */
+pa_status pa_alloc_incref(pa_allocator* alloc, int32_t block);         /* block must be allocated */
+pa_status pa_alloc_decref(pa_allocator* alloc, int32_t block);         /* 0 -> back on the stack */
+int       pa_alloc_num_free(const pa_allocator* alloc);
+int       pa_alloc_num_blocks(const pa_allocator* alloc);
+int       pa_alloc_block_size(const pa_allocator* alloc);
+int       pa_alloc_ref_count(const pa_allocator* alloc, int32_t block);  /* -1 if out of range */
+/* Free stack from top to bottom into out[0..capacity); *count = its size. */
+pa_status pa_alloc_free_order(const pa_allocator* alloc, int32_t* out, int capacity, int* count);
+
+/*
+ * Sequence helpers on caller-owned host tables.  A sequence of `length`
+ * tokens holds exactly ceil(length / block_size) table entries.
+ *
+ * pa_seq_append_slot: make room for token `*length`: a fresh block when
+ * the last one is full; otherwise, if the last block is shared
+ * (ref_count > 1), copy-on-write -- a fresh block replaces it in the table,
+ * the old block's count drops, and (*cow_src, *cow_dst) report the pair to
+ * copy (both -1 when no copy is needed).  *slot = block * block_size + row;
+ * *length is incremented.  `capacity` is the table's size.
+ */
+pa_status pa_seq_append_slot(pa_allocator* alloc, int32_t* table, int capacity, int* length,
+                             int64_t* slot, int32_t* cow_src, int32_t* cow_dst);
+
+/* One token for each of `num_seqs` sequences, in ascending index (the last
+ * sharer of a partial block writes in place).  tables: [num_seqs, stride];
+ * lengths [num_seqs] updated; slots [num_seqs]; cow_pairs [num_seqs, 2]
+ * receives *num_cow (src, dst) pairs.  All-or-nothing on OUT_OF_BLOCKS. */
+pa_status pa_seq_append_slots(pa_allocator* alloc, int32_t* tables, int stride, int* lengths,
+                              int num_seqs, int64_t* slots, int32_t* cow_pairs, int* num_cow);
+
+/* `num_tokens` successive appends to one sequence (a prompt).  slots may be
+ * NULL; (*cow_src, *cow_dst) report the copy the first append needed, if
+ * any.  All-or-nothing on OUT_OF_BLOCKS. */
+pa_status pa_seq_extend(pa_allocator* alloc, int32_t* table, int capacity, int* length,
+                        int num_tokens, int64_t* slots, int32_t* cow_src, int32_t* cow_dst);
+
+/* The child shares every parent block; each block's count goes up by one. */
+pa_status pa_seq_fork(pa_allocator* alloc, const int32_t* parent_table, int num_table_blocks,
+                      int32_t* child_table);
+
+/* Drop the sequence's reference on each of its blocks. */
+pa_status pa_seq_free(pa_allocator* alloc, const int32_t* table, int num_table_blocks);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

@@ -1,0 +1,251 @@
+"""Paged KV-cache decode on B200: Python binding of libpagedattn.so.
+
+Every function here only marshals arguments (tensor pointers, sizes, the
+current CUDA stream) into the C ABI declared in ``include/pagedattn.h``; all
+work on the hot path runs in the library's CUDA kernels.  PyTorch supplies
+device memory and streams.  There is no CPU fallback: the calls raise when
+the library is missing or a tensor is not on a CUDA device.
+
+Functions carry the C names:
+
+* ``pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping)``
+* ``pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale)``
+* ``pa_decode_split(out, q, ..., max_context_len, partition_size, workspace)``
+* ``pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size)``
+* ``pa_copy_blocks(k_cache, v_cache, block_mapping)``
+* ``pa_device_error(clear=True)``, ``pa_set_option(name, value)``
+
+and ``BlockAllocator`` wraps the host allocator (``pa_alloc_*`` / ``pa_seq_*``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SPLIT_CTAS,
+                      PA_OPT_VALIDATE, PagedAttnError, check, lib)
+
+__all__ = [
+    "pa_reshape_and_cache", "pa_decode", "pa_decode_split", "pa_decode_split_workspace_bytes",
+    "pa_copy_blocks", "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
+    "PagedAttnError", "OutOfBlocks", "DEVERR_BITS",
+]
+
+_DTYPES = {torch.float32: PA_DTYPE_F32, torch.bfloat16: PA_DTYPE_BF16}
+_OPTIONS = {"validate": PA_OPT_VALIDATE, "decode_split_ctas": PA_OPT_DECODE_SPLIT_CTAS}
+
+
+class OutOfBlocks(PagedAttnError):
+    pass
+
+
+def _dtype(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise ValueError(f"dtype {t.dtype} not supported (float32, bfloat16)") from None
+
+
+def _dev(*tensors):
+    for t in tensors:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
+    """key/value [T, Hk, D]; caches [NB, bs, Hk, D]; slot_mapping int64 [T]."""
+    _dev(key, value, k_cache, v_cache, slot_mapping)
+    nb, bs, hk, d = k_cache.shape
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    check(lib().pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(slot_mapping), key.shape[0], hk, d, bs, nb,
+                                     _dtype(k_cache), _stream(stream)))
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, stream=None):
+    """out/q [S, Hq, D]; caches [NB, bs, Hk, D]; block_tables int32 [S, maxB];
+    context_lens int32 [S].  Writes ``out`` and returns it."""
+    _dev(out, q, k_cache, v_cache, block_tables, context_lens)
+    s, hq, d = q.shape
+    nb, bs, hk, _ = k_cache.shape
+    check(lib().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                          block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb,
+                          float(scale), _dtype(q), _stream(stream)))
+    return out
+
+
+def pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len,
+                                    partition_size) -> int:
+    return int(lib().pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                     max_context_len, partition_size))
+
+
+def pa_decode_split(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                    max_context_len, partition_size=512, workspace=None, stream=None):
+    """Split-K decode; ``workspace`` is a CUDA byte tensor of at least
+    ``pa_decode_split_workspace_bytes(...)`` bytes (allocated here if None)."""
+    _dev(out, q, k_cache, v_cache, block_tables, context_lens)
+    s, hq, d = q.shape
+    nb, bs, hk, _ = k_cache.shape
+    need = pa_decode_split_workspace_bytes(s, hq, d, max_context_len, partition_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _dev(workspace)
+    nbytes = workspace.numel() * workspace.element_size()
+    check(lib().pa_decode_split(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), s,
+                                hq, hk, d, bs, nb, float(scale), _dtype(q), int(max_context_len),
+                                int(partition_size), _ptr(workspace), nbytes, _stream(stream)))
+    return out
+
+
+def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
+    """block_mapping int64 [P, 2] of (src, dst) on the device."""
+    _dev(k_cache, v_cache, block_mapping)
+    nb, bs, hk, d = k_cache.shape
+    if block_mapping.dtype != torch.int64:
+        raise ValueError("block_mapping must be int64")
+    check(lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping),
+                               block_mapping.shape[0], hk, d, bs, nb, _dtype(k_cache),
+                               _stream(stream)))
+
+
+def pa_device_error(clear: bool = True, stream=None) -> int:
+    """Synchronise the stream and return the device error word (0 = clean)."""
+    flags = ctypes.c_uint32(0)
+    status = lib().pa_device_error(_stream(stream), ctypes.byref(flags), int(clear))
+    if status not in (0, 6):
+        check(status)
+    return int(flags.value)
+
+
+def pa_set_option(name: str, value: int) -> None:
+    check(lib().pa_set_option(_OPTIONS[name], int(value)))
+
+
+def pa_get_option(name: str) -> int:
+    return int(lib().pa_get_option(_OPTIONS[name]))
+
+
+# --------------------------------------------------------------------------
+# Host allocator
+# --------------------------------------------------------------------------
+
+def _i32(a: np.ndarray):
+    if a.dtype != np.int32 or not a.flags["C_CONTIGUOUS"]:
+        raise ValueError("host tables must be contiguous int32 arrays")
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+class BlockAllocator:
+    """Ref-counted block pool (``pa_alloc_*``) plus the sequence helpers
+    (``pa_seq_*``) on host int32 tables."""
+
+    def __init__(self, num_blocks: int, block_size: int, initial_free_order=None):
+        order = None
+        if initial_free_order is not None:
+            order = np.ascontiguousarray(initial_free_order, dtype=np.int32)
+            if order.shape != (num_blocks,):
+                raise ValueError("initial_free_order must hold num_blocks entries")
+        self._keep = order
+        h = lib().pa_alloc_create(num_blocks, block_size, _i32(order) if order is not None else None)
+        if not h:
+            raise PagedAttnError(1, lib().pa_last_error().decode())
+        self._h = ctypes.c_void_p(h)
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib().pa_alloc_destroy(h)
+            self._h = None
+
+    @staticmethod
+    def _check(status):
+        if status == 3:
+            raise OutOfBlocks(3, lib().pa_last_error().decode())
+        check(status)
+
+    def allocate(self) -> int:
+        out = ctypes.c_int32(0)
+        self._check(lib().pa_alloc_allocate(self._h, ctypes.byref(out)))
+        return out.value
+
+    def incref(self, block: int) -> None:
+        self._check(lib().pa_alloc_incref(self._h, int(block)))
+
+    def decref(self, block: int) -> None:
+        self._check(lib().pa_alloc_decref(self._h, int(block)))
+
+    def num_free(self) -> int:
+        return int(lib().pa_alloc_num_free(self._h))
+
+    def ref_count(self, block: int) -> int:
+        return int(lib().pa_alloc_ref_count(self._h, int(block)))
+
+    def ref_counts(self) -> list:
+        return [self.ref_count(b) for b in range(self.num_blocks)]
+
+    def free_order(self) -> list:
+        buf = np.zeros(self.num_blocks, dtype=np.int32)
+        n = ctypes.c_int(0)
+        self._check(lib().pa_alloc_free_order(self._h, _i32(buf), self.num_blocks, ctypes.byref(n)))
+        return buf[: n.value].tolist()
+
+    def append_slot(self, table: np.ndarray, length: int):
+        """table: int32 array (mutated).  Returns (slot, cow or None, new_length)."""
+        ln = ctypes.c_int(length)
+        slot = ctypes.c_int64(0)
+        src, dst = ctypes.c_int32(-1), ctypes.c_int32(-1)
+        self._check(lib().pa_seq_append_slot(self._h, _i32(table), table.shape[0], ctypes.byref(ln),
+                                             ctypes.byref(slot), ctypes.byref(src),
+                                             ctypes.byref(dst)))
+        return slot.value, ((src.value, dst.value) if src.value >= 0 else None), ln.value
+
+    def append_slots(self, tables: np.ndarray, lengths: np.ndarray):
+        """tables int32 [S, stride], lengths int32 [S] (both mutated).
+        Returns (slots int64 [S], cow_pairs int32 [n, 2])."""
+        s = tables.shape[0]
+        slots = np.zeros(s, dtype=np.int64)
+        pairs = np.zeros((max(s, 1), 2), dtype=np.int32)
+        n = ctypes.c_int(0)
+        self._check(lib().pa_seq_append_slots(
+            self._h, _i32(tables), tables.shape[1],
+            lengths.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), s,
+            slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _i32(pairs), ctypes.byref(n)))
+        return slots, pairs[: n.value].copy()
+
+    def extend(self, table: np.ndarray, length: int, num_tokens: int, want_slots: bool = True):
+        ln = ctypes.c_int(length)
+        slots = np.zeros(max(num_tokens, 1), dtype=np.int64) if want_slots else None
+        src, dst = ctypes.c_int32(-1), ctypes.c_int32(-1)
+        self._check(lib().pa_seq_extend(
+            self._h, _i32(table), table.shape[0], ctypes.byref(ln), num_tokens,
+            slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)) if want_slots else None,
+            ctypes.byref(src), ctypes.byref(dst)))
+        cow = (src.value, dst.value) if src.value >= 0 else None
+        return (slots[:num_tokens] if want_slots else None), cow, ln.value
+
+    def fork(self, parent_table: np.ndarray, num_table_blocks: int, child_table: np.ndarray):
+        self._check(lib().pa_seq_fork(self._h, _i32(parent_table), num_table_blocks,
+                                      _i32(child_table)))
+
+    def free(self, table: np.ndarray, num_table_blocks: int):
+        self._check(lib().pa_seq_free(self._h, _i32(table), num_table_blocks))

@@ -1,0 +1,418 @@
+// C ABI of libpagedattn.so: argument checks, optional host-side index
+// validation, tensor-map encoding and dispatch to the kernel instances.
+// The public contract of every call is documented in include/pagedattn.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_set>
+#include <vector>
+
+#include <cudaTypedefs.h>
+
+#include "launch.cuh"
+
+namespace pa {
+
+namespace {
+
+thread_local std::string g_last_error;
+int g_validate = -1;                 // -1: read PA_VALIDATE on first use
+int g_decode_ctas = 0;               // 0: automatic
+
+bool validate_enabled() {
+    if (g_validate < 0) {
+        const char* v = std::getenv("PA_VALIDATE");
+        g_validate = (v && v[0] && v[0] != '0') ? 1 : 0;
+    }
+    return g_validate == 1;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_size(pa_dtype dt) { return dt == PA_DTYPE_F32 ? 4 : 2; }
+
+pa_status check_geometry(pa_dtype dt, int head_dim, int block_size) {
+    if (dt != PA_DTYPE_F32 && dt != PA_DTYPE_BF16)
+        return fail(PA_ERR_UNSUPPORTED, "dtype %d not supported", (int)dt);
+    if (head_dim != 64 && head_dim != 128 && head_dim != 256)
+        return fail(PA_ERR_UNSUPPORTED, "head_dim %d not built (64, 128, 256)", head_dim);
+    if (block_size != 8 && block_size != 16 && block_size != 32)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d not built (8, 16, 32)", block_size);
+    return PA_OK;
+}
+
+template <typename T>
+bool copy_to_host(std::vector<T>& dst, const T* src, size_t n, cudaStream_t stream) {
+    dst.resize(n);
+    if (n == 0) return true;
+    if (cudaMemcpyAsync(dst.data(), src, n * sizeof(T), cudaMemcpyDeviceToHost, stream) !=
+        cudaSuccess)
+        return false;
+    return cudaStreamSynchronize(stream) == cudaSuccess;
+}
+
+pa_status validate_decode(const int32_t* tables, int max_blocks, const int32_t* lens, int num_seqs,
+                          int block_size, int num_blocks, cudaStream_t stream) {
+    std::vector<int32_t> t, l;
+    if (!copy_to_host(l, lens, (size_t)num_seqs, stream) ||
+        !copy_to_host(t, tables, (size_t)num_seqs * max_blocks, stream))
+        return fail(PA_ERR_CUDA, "validation copy failed");
+    for (int s = 0; s < num_seqs; ++s) {
+        if (l[s] < 0 || (int64_t)l[s] > (int64_t)max_blocks * block_size)
+            return fail(PA_ERR_BAD_BLOCK_ID, "context_lens[%d] = %d outside [0, %lld]", s, l[s],
+                        (long long)max_blocks * block_size);
+        const int n = (l[s] + block_size - 1) / block_size;
+        for (int j = 0; j < n; ++j) {
+            const int32_t b = t[(size_t)s * max_blocks + j];
+            if (b < 0 || b >= num_blocks)
+                return fail(PA_ERR_BAD_BLOCK_ID, "block_tables[%d, %d] = %d outside [0, %d)", s, j,
+                            b, num_blocks);
+        }
+    }
+    return PA_OK;
+}
+
+pa_status check_decode_args(void* out, const void* q, const void* kc, const void* vc,
+                            const int32_t* tables, int max_blocks, const int32_t* lens,
+                            int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                            int block_size, int num_blocks, pa_dtype dt, float scale) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "sizes must be positive (num_seqs >= 0)");
+    if (num_seqs > 65535) return fail(PA_ERR_UNSUPPORTED, "num_seqs above 65535");
+    if (num_heads % num_kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARG, "num_heads %d is not a multiple of num_kv_heads %d",
+                    num_heads, num_kv_heads);
+    if (num_kv_heads > 65535) return fail(PA_ERR_UNSUPPORTED, "num_kv_heads above 65535");
+    if ((int64_t)max_blocks * block_size > 0x7fffffff)
+        return fail(PA_ERR_UNSUPPORTED, "max_blocks_per_seq * block_size overflows int32");
+    if (pa_status s = check_geometry(dt, head_dim, block_size)) return s;
+    const int g = num_heads / num_kv_heads;
+    if (g != 1 && g != 2 && g != 4 && g != 8)
+        return fail(PA_ERR_UNSUPPORTED, "group size %d not built (1, 2, 4, 8)", g);
+    if (!(scale == scale)) return fail(PA_ERR_INVALID_ARG, "scale is NaN");
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !kc || !vc || !tables || !lens)
+        return fail(PA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(kc) || !aligned16(vc))
+        return fail(PA_ERR_INVALID_ARG, "q, out and caches must be 16-byte aligned");
+    return PA_OK;
+}
+
+int auto_decode_ctas(int num_seqs, int num_kv_heads, int max_blocks, int block_size) {
+    const int64_t max_tokens = (int64_t)max_blocks * block_size;
+    const int64_t work = (int64_t)num_seqs * num_kv_heads;
+    const int64_t target = 16LL * num_sms();
+    int c = 1;
+    while (c < 8 && max_tokens / c > 2048 && work * c < target) c *= 2;
+    return c;
+}
+
+pa_status dispatch_decode(const DecodeLaunch& l, pa_dtype dt, int head_dim) {
+    if (dt == PA_DTYPE_F32) {
+        if (head_dim == 64) return launch_decode_f32_d64(l);
+        if (head_dim == 128) return launch_decode_f32_d128(l);
+        return launch_decode_f32_d256(l);
+    }
+    if (head_dim == 64) return launch_decode_bf16_d64(l);
+    if (head_dim == 128) return launch_decode_bf16_d128(l);
+    return launch_decode_bf16_d256(l);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+pa_status fail(pa_status status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
+pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
+                           int num_kv_heads, int block_size, int num_blocks, int rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t es = (cuuint64_t)elem_size(dtype);
+    cuuint64_t dims[4] = {(cuuint64_t)head_dim, (cuuint64_t)num_kv_heads, (cuuint64_t)block_size,
+                          (cuuint64_t)num_blocks};
+    cuuint64_t strides[3] = {head_dim * es, (cuuint64_t)num_kv_heads * head_dim * es,
+                             (cuuint64_t)block_size * num_kv_heads * head_dim * es};
+    cuuint32_t box[4] = {(cuuint32_t)head_dim, 1, (cuuint32_t)rows, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(map,
+                     dtype == PA_DTYPE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PA_OK;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char* pa_last_error(void) { return g_last_error.c_str(); }
+
+const char* pa_status_string(pa_status s) {
+    switch (s) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARG: return "invalid argument";
+        case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case PA_ERR_OUT_OF_BLOCKS: return "out of blocks";
+        case PA_ERR_BAD_BLOCK_ID: return "bad block id";
+        case PA_ERR_CUDA: return "cuda error";
+        case PA_ERR_DEVICE_CHECK: return "device check failed";
+    }
+    return "unknown status";
+}
+
+int pa_version(void) { return 1; }
+
+pa_status pa_set_option(pa_option option, int value) {
+    switch (option) {
+        case PA_OPT_VALIDATE: g_validate = value ? 1 : 0; return PA_OK;
+        case PA_OPT_DECODE_SPLIT_CTAS:
+            if (value != 0 && value != 1 && value != 2 && value != 4 && value != 8)
+                return fail(PA_ERR_INVALID_ARG, "CTAs per (sequence, kv head) must be 0,1,2,4,8");
+            g_decode_ctas = value;
+            return PA_OK;
+    }
+    return fail(PA_ERR_INVALID_ARG, "unknown option %d", (int)option);
+}
+
+int pa_get_option(pa_option option) {
+    switch (option) {
+        case PA_OPT_VALIDATE: return validate_enabled() ? 1 : 0;
+        case PA_OPT_DECODE_SPLIT_CTAS: return g_decode_ctas;
+    }
+    return -1;
+}
+
+pa_status pa_device_error(pa_stream_t stream, uint32_t* flags, int clear) {
+    if (!flags) return fail(PA_ERR_INVALID_ARG, "null flags");
+    unsigned* word = device_error_word();
+    if (!word) return fail(PA_ERR_CUDA, "device error word unavailable");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned v = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return fail(PA_ERR_CUDA, "reading the device error word: %s",
+                    cudaGetErrorString(cudaGetLastError()));
+    *flags = v;
+    if (clear && v && cudaMemset(word, 0, sizeof(unsigned)) != cudaSuccess)
+        return fail(PA_ERR_CUDA, "clearing the device error word failed");
+    if (v) return fail(PA_ERR_DEVICE_CHECK, "device error word 0x%x", v);
+    return PA_OK;
+}
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, pa_dtype dtype,
+                               pa_stream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "sizes must be positive (num_tokens >= 0)");
+    if (pa_status s = check_geometry(dtype, head_dim, block_size)) return s;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+        return fail(PA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_INVALID_ARG, "rows and caches must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t num_slots = (int64_t)num_blocks * block_size;
+    if (validate_enabled()) {
+        std::vector<int64_t> sl;
+        if (!copy_to_host(sl, slot_mapping, (size_t)num_tokens, st))
+            return fail(PA_ERR_CUDA, "validation copy failed");
+        std::unordered_set<int64_t> seen;
+        for (int t = 0; t < num_tokens; ++t) {
+            if (sl[t] < -1 || sl[t] >= num_slots)
+                return fail(PA_ERR_BAD_BLOCK_ID, "slot_mapping[%d] = %lld outside [-1, %lld)", t,
+                            (long long)sl[t], (long long)num_slots);
+            if (sl[t] >= 0 && !seen.insert(sl[t]).second)
+                return fail(PA_ERR_BAD_BLOCK_ID, "slot %lld written twice", (long long)sl[t]);
+        }
+    }
+    const int64_t row_bytes = (int64_t)num_kv_heads * head_dim * elem_size(dtype);
+    return launch_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, num_tokens,
+                                    row_bytes, num_slots, st);
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int max_blocks_per_seq,
+                    const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                    int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+                    pa_stream_t stream) {
+    if (pa_status s = check_decode_args(out, q, k_cache, v_cache, block_tables,
+                                        max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                                        num_kv_heads, head_dim, block_size, num_blocks, dtype,
+                                        scale))
+        return s;
+    if (num_seqs == 0) return PA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (validate_enabled())
+        if (pa_status s = validate_decode(block_tables, max_blocks_per_seq, context_lens,
+                                          num_seqs, block_size, num_blocks, st))
+            return s;
+    DecodeLaunch l = {};
+    l.args.out = out;
+    l.args.q = q;
+    l.args.block_tables = block_tables;
+    l.args.context_lens = context_lens;
+    l.args.err = device_error_word();
+    if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    l.args.scale_log2 = scale * 1.4426950408889634f;
+    l.args.max_blocks = max_blocks_per_seq;
+    l.args.max_tokens = max_blocks_per_seq * block_size;
+    l.args.num_heads = num_heads;
+    l.args.num_kv_heads = num_kv_heads;
+    l.args.num_blocks = num_blocks;
+    l.k_cache = k_cache;
+    l.v_cache = v_cache;
+    l.num_seqs = num_seqs;
+    l.num_kv_heads = num_kv_heads;
+    l.block_size = block_size;
+    l.group = num_heads / num_kv_heads;
+    l.ctas = g_decode_ctas ? g_decode_ctas
+                           : auto_decode_ctas(num_seqs, num_kv_heads, max_blocks_per_seq,
+                                              block_size);
+    l.split = false;
+    l.stream = st;
+    return dispatch_decode(l, dtype, head_dim);
+}
+
+size_t pa_decode_split_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                       int max_context_len, int partition_size) {
+    if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+        partition_size <= 0)
+        return 0;
+    const size_t parts = max_context_len == 0
+                             ? 1
+                             : (size_t)((max_context_len + (int64_t)partition_size - 1) /
+                                        partition_size);
+    const size_t rows = (size_t)num_seqs * num_heads * parts;
+    return 2 * align256(rows * sizeof(float)) + rows * head_dim * sizeof(float);
+}
+
+pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, int max_blocks_per_seq,
+                          const int32_t* context_lens, int num_seqs, int num_heads,
+                          int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                          float scale, pa_dtype dtype, int max_context_len, int partition_size,
+                          void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+    if (pa_status s = check_decode_args(out, q, k_cache, v_cache, block_tables,
+                                        max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                                        num_kv_heads, head_dim, block_size, num_blocks, dtype,
+                                        scale))
+        return s;
+    if (partition_size <= 0 || partition_size % block_size != 0)
+        return fail(PA_ERR_INVALID_ARG, "partition_size %d must be a positive multiple of %d",
+                    partition_size, block_size);
+    if (max_context_len < 0) return fail(PA_ERR_INVALID_ARG, "negative max_context_len");
+    if (num_seqs == 0) return PA_OK;
+    const size_t need = pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                        max_context_len, partition_size);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+        return fail(PA_ERR_INVALID_ARG, "workspace needs %zu bytes, 16-byte aligned", need);
+    const int64_t parts64 =
+        max_context_len == 0 ? 1 : ((int64_t)max_context_len + partition_size - 1) / partition_size;
+    if (parts64 > 0x7fffffff) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
+    if ((int64_t)num_seqs * num_heads > 0x7fffffff)
+        return fail(PA_ERR_UNSUPPORTED, "num_seqs * num_heads overflows int32");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (validate_enabled())
+        if (pa_status s = validate_decode(block_tables, max_blocks_per_seq, context_lens,
+                                          num_seqs, block_size, num_blocks, st))
+            return s;
+    const size_t rows = (size_t)num_seqs * num_heads * (size_t)parts64;
+    DecodeLaunch l = {};
+    char* ws = static_cast<char*>(workspace);
+    l.args.out = out;
+    l.args.q = q;
+    l.args.block_tables = block_tables;
+    l.args.context_lens = context_lens;
+    l.args.ws_m = reinterpret_cast<float*>(ws);
+    l.args.ws_l = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
+    l.args.ws_o = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
+    l.args.err = device_error_word();
+    if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    l.args.scale_log2 = scale * 1.4426950408889634f;
+    l.args.max_blocks = max_blocks_per_seq;
+    l.args.max_tokens = max_blocks_per_seq * block_size;
+    l.args.num_heads = num_heads;
+    l.args.num_kv_heads = num_kv_heads;
+    l.args.num_blocks = num_blocks;
+    l.args.part_tokens = partition_size;
+    l.args.max_parts = (int)parts64;
+    l.k_cache = k_cache;
+    l.v_cache = v_cache;
+    l.num_seqs = num_seqs;
+    l.num_kv_heads = num_kv_heads;
+    l.block_size = block_size;
+    l.group = num_heads / num_kv_heads;
+    l.ctas = 1;
+    l.split = true;
+    l.stream = st;
+    return dispatch_decode(l, dtype, head_dim);
+}
+
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, pa_dtype dtype, pa_stream_t stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "sizes must be positive (num_pairs >= 0)");
+    if (pa_status s = check_geometry(dtype, head_dim, block_size)) return s;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !block_mapping) return fail(PA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(k_cache) || !aligned16(v_cache))
+        return fail(PA_ERR_INVALID_ARG, "caches must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (validate_enabled()) {
+        std::vector<int64_t> mp;
+        if (!copy_to_host(mp, block_mapping, (size_t)num_pairs * 2, st))
+            return fail(PA_ERR_CUDA, "validation copy failed");
+        std::unordered_set<int64_t> dsts, srcs;
+        for (int i = 0; i < num_pairs; ++i) {
+            for (int k = 0; k < 2; ++k)
+                if (mp[2 * i + k] < 0 || mp[2 * i + k] >= num_blocks)
+                    return fail(PA_ERR_BAD_BLOCK_ID, "block_mapping[%d] outside the pool", i);
+            srcs.insert(mp[2 * i]);
+            if (!dsts.insert(mp[2 * i + 1]).second)
+                return fail(PA_ERR_BAD_BLOCK_ID, "destination %lld repeated",
+                            (long long)mp[2 * i + 1]);
+        }
+        for (int64_t d : dsts)
+            if (srcs.count(d))
+                return fail(PA_ERR_BAD_BLOCK_ID, "block %lld is both source and destination",
+                            (long long)d);
+    }
+    const int64_t block_bytes = (int64_t)block_size * num_kv_heads * head_dim * elem_size(dtype);
+    return launch_copy_blocks(k_cache, v_cache, block_mapping, num_pairs, block_bytes, num_blocks,
+                              st);
+}
+
+}  // extern "C"

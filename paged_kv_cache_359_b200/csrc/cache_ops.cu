@@ -1,0 +1,125 @@
+// Cache write (reshape_and_cache) and copy-on-write block copy kernels, plus
+// the library's device-side error word.
+//
+// reshape_and_cache: a generated token's key and value rows go into the row
+// its slot names ("vLLM内存管理与PagedAttention精讲" ch.2 §2.4.2, a new block
+// only when the current one is full; "VLLM中PagedAttention如何降低显存碎片？"
+// §四 flow: allocate a free page, update the mapping).  With the cache laid
+// out [num_blocks][block_size][kv_heads][head_dim], slot s is one contiguous
+// row of kv_heads * head_dim elements, so the write is a 16-byte-vector row
+// copy.
+//
+// copy_blocks: copy-on-write of a shared block ("vLLM内存管理与PagedAttention
+// 精讲" §2.4.3): block dst <- block src for keys and values; a block is one
+// contiguous run of block_size * kv_heads * head_dim elements.
+#include "common.cuh"
+#include "internal.h"
+
+namespace pa {
+
+__device__ unsigned g_device_error_word;
+
+namespace {
+
+__global__ void __launch_bounds__(128)
+    reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict__ value,
+                             uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                             const int64_t* __restrict__ slots, int num_tokens, int row_vecs,
+                             int64_t num_slots, unsigned* err) {
+    for (int t = blockIdx.x; t < num_tokens; t += gridDim.x) {
+        const int64_t s = slots[t];
+        if (s < 0) continue;
+        if (s >= num_slots) {
+            if (threadIdx.x == 0) raise_error(err, PA_DEVERR_SLOT);
+            continue;
+        }
+        const uint4* ks = key + (size_t)t * row_vecs;
+        const uint4* vs = value + (size_t)t * row_vecs;
+        uint4* kd = k_cache + (size_t)s * row_vecs;
+        uint4* vd = v_cache + (size_t)s * row_vecs;
+        for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) {
+            kd[i] = ks[i];
+            vd[i] = vs[i];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+                       const int64_t* __restrict__ mapping, int64_t block_vecs, int num_blocks,
+                       unsigned* err) {
+    const int pair = blockIdx.x;
+    const int64_t src = mapping[2 * pair], dst = mapping[2 * pair + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) raise_error(err, PA_DEVERR_COPY_ID);
+        return;
+    }
+    const uint4* ks = k_cache + src * block_vecs;
+    const uint4* vs = v_cache + src * block_vecs;
+    uint4* kd = k_cache + dst * block_vecs;
+    uint4* vd = v_cache + dst * block_vecs;
+    for (int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; i < block_vecs;
+         i += (int64_t)gridDim.y * blockDim.x) {
+        kd[i] = ks[i];
+        vd[i] = vs[i];
+    }
+}
+
+}  // namespace
+
+unsigned* device_error_word() {
+    static unsigned* cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cached[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+        cached[dev] = static_cast<unsigned*>(p);
+    }
+    return cached[dev];
+}
+
+int num_sms() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+pa_status launch_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                                   void* v_cache, const int64_t* slots, int num_tokens,
+                                   int64_t row_bytes, int64_t num_slots, cudaStream_t stream) {
+    if (num_tokens == 0) return PA_OK;
+    unsigned* err = device_error_word();
+    if (!err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    const int grid = num_tokens < 8 * num_sms() ? num_tokens : 8 * num_sms();
+    reshape_and_cache_kernel<<<grid, 128, 0, stream>>>(
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slots, num_tokens,
+        (int)(row_bytes / 16), num_slots, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reshape_and_cache launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+}
+
+pa_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping, int num_pairs,
+                             int64_t block_bytes, int num_blocks, cudaStream_t stream) {
+    if (num_pairs == 0) return PA_OK;
+    unsigned* err = device_error_word();
+    if (!err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    const int64_t vecs = block_bytes / 16;
+    int chunks = (int)(vecs / 1024);
+    chunks = chunks < 1 ? 1 : (chunks > 32 ? 32 : chunks);
+    copy_blocks_kernel<<<dim3(num_pairs, chunks), 256, 0, stream>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), mapping, vecs, num_blocks, err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "copy_blocks launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+}
+
+}  // namespace pa

@@ -1,0 +1,4 @@
+// Decode kernel instances for f32, head_dim 64 (all block sizes and group sizes).
+#include "launch.cuh"
+
+PA_DEFINE_DECODE_LAUNCHER(launch_decode_f32_d64, float, 64)

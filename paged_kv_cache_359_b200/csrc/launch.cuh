@@ -1,0 +1,117 @@
+// Host-side launch of the paged decode kernels for one (dtype, head_dim);
+// dispatches block_size and group size to template instances.
+#pragma once
+
+#include <atomic>
+#include <type_traits>
+
+#include "decode.cuh"
+#include "internal.h"
+
+namespace pa {
+
+struct DecodeLaunch {
+    DecodeArgs args;
+    const void* k_cache;
+    const void* v_cache;
+    int num_seqs;
+    int num_kv_heads;
+    int block_size;
+    int group;
+    int ctas;          // pa_decode: CTAs (one cluster) per (sequence, kv head)
+    bool split;
+    cudaStream_t stream;
+};
+
+// Opt a kernel into `bytes` of dynamic shared memory, once per device.
+// `done` must be distinct for every kernel (one static per instantiation).
+template <class K>
+inline pa_status allow_smem(K kernel, int bytes, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_relaxed) & bit) return PA_OK;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+        return fail(PA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    done.fetch_or(bit);
+    return PA_OK;
+}
+
+template <typename T, int D, int BS, int G>
+pa_status launch_decode_g(const DecodeLaunch& l) {
+    using Gm = Geom<T, D, BS, G>;
+    constexpr pa_dtype DT = std::is_same<T, float>::value ? PA_DTYPE_F32 : PA_DTYPE_BF16;
+    CUtensorMap mk, mv;
+    if (pa_status s = encode_cache_map(&mk, l.k_cache, DT, D, l.num_kv_heads, BS,
+                                       l.args.num_blocks, Gm::R))
+        return s;
+    if (pa_status s = encode_cache_map(&mv, l.v_cache, DT, D, l.num_kv_heads, BS,
+                                       l.args.num_blocks, Gm::R))
+        return s;
+    if (l.split && l.args.part_tokens % Gm::R != 0)
+        return fail(PA_ERR_INVALID_ARG, "partition must be a multiple of %d tokens", Gm::R);
+
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(Gm::NW * 32);
+    cfg.dynamicSmemBytes = Gm::SMEM_BYTES;
+    cfg.stream = l.stream;
+    cudaError_t e;
+    if (l.split) {
+        static std::atomic<unsigned long long> done{0};
+        auto kern = paged_decode_kernel<T, D, BS, G, Mode::Split>;
+        if (pa_status s = allow_smem(kern, Gm::SMEM_BYTES, done)) return s;
+        cfg.gridDim = dim3(l.args.max_parts, l.num_kv_heads, l.num_seqs);
+        e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
+        if (e == cudaSuccess) {
+            lse_reduce_kernel<T, D><<<dim3(l.num_seqs * l.args.num_heads, D / 32), 256, 0,
+                                      l.stream>>>(l.args);
+            e = cudaGetLastError();
+        }
+    } else {
+        static std::atomic<unsigned long long> done{0};
+        auto kern = paged_decode_kernel<T, D, BS, G, Mode::Decode>;
+        if (pa_status s = allow_smem(kern, Gm::SMEM_BYTES, done)) return s;
+        cfg.gridDim = dim3(l.ctas, l.num_kv_heads, l.num_seqs);
+        if (l.ctas > 1) {
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = l.ctas;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+        }
+        e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
+    }
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+}
+
+template <typename T, int D, int BS>
+pa_status launch_decode_bs(const DecodeLaunch& l) {
+    switch (l.group) {
+        case 1: return launch_decode_g<T, D, BS, 1>(l);
+        case 2: return launch_decode_g<T, D, BS, 2>(l);
+        case 4: return launch_decode_g<T, D, BS, 4>(l);
+        case 8: return launch_decode_g<T, D, BS, 8>(l);
+        default: return fail(PA_ERR_UNSUPPORTED, "group size %d not built", l.group);
+    }
+}
+
+template <typename T, int D>
+pa_status launch_decode_td(const DecodeLaunch& l) {
+    switch (l.block_size) {
+        case 8: return launch_decode_bs<T, D, 8>(l);
+        case 16: return launch_decode_bs<T, D, 16>(l);
+        case 32: return launch_decode_bs<T, D, 32>(l);
+        default: return fail(PA_ERR_UNSUPPORTED, "block_size %d not built", l.block_size);
+    }
+}
+
+}  // namespace pa
+
+#define PA_DEFINE_DECODE_LAUNCHER(NAME, T, D) \
+    namespace pa {                            \
+    pa_status NAME(const DecodeLaunch& l) { return launch_decode_td<T, D>(l); } \
+    }

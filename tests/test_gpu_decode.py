@@ -1,0 +1,160 @@
+"""GPU parity for pa_decode and pa_decode_split against the fp64 oracle:
+every built (dtype, head_dim, block_size, group) combination on small ragged
+batches, the workload shapes at full size on sampled sequences, permutation
+invariance, cluster splits, and poisoned rows."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pa_inputs
+import paged_kv_cache_359_b200 as pa
+from gpu_common import (assert_close, device_clean, oracle_decode, run_decode, same_bits,
+                        tables_via_oracle_allocator)
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_decode_append_decode():
+    """3 sequences (5, 16, 37 tokens), fp32: decode, append one token per
+    sequence through the allocator and reshape_and_cache, decode again."""
+    problem = pa_inputs.tiny()
+    data = pa_inputs.materialize(problem, "cuda")
+    assert_close(run_decode(data, problem), oracle_decode(data, problem))
+    device_clean()
+
+    alloc, tables, lengths = tables_via_oracle_allocator(problem)
+    assert all(list(problem.block_tables[i, :len(t)]) == t for i, t in enumerate(tables))
+    slots, cows = oracle.append_slots(alloc, tables, lengths)
+    new = pa_inputs.step_tokens(3, 4, 4, 64, "f32", problem.seed, 0, "cuda")
+    k_ref, v_ref = oracle.reshape_and_cache(new["key"].cpu(), new["value"].cpu(),
+                                            data["k_cache"].cpu(), data["v_cache"].cpu(), slots)
+    pa.pa_reshape_and_cache(new["key"], new["value"], data["k_cache"], data["v_cache"],
+                            torch.tensor(slots, dtype=torch.int64, device="cuda"))
+    problem.context_lens = np.array(lengths, dtype=np.int32)
+    for i, t in enumerate(tables):
+        problem.block_tables[i, :len(t)] = t
+    data["block_tables"] = torch.from_numpy(problem.block_tables).cuda()
+    data["context_lens"] = torch.from_numpy(problem.context_lens).cuda()
+    data["q"] = new["q"]
+    got = run_decode(data, problem)
+    ref = oracle.paged_decode(new["q"].cpu(), k_ref, v_ref, problem.block_tables,
+                              problem.context_lens, problem.scale)
+    assert_close(got, ref)
+    device_clean()
+
+
+COMBOS = [(dt, d, bs, g) for dt in ("bf16", "f32") for d in (64, 128, 256)
+          for bs in (8, 16, 32) for g in (1, 2, 4, 8)]
+
+
+@pytest.mark.parametrize("dtype,d,bs,g", COMBOS)
+def test_decode_all_instances_small(dtype, d, bs, g):
+    hk = 2
+    problem = pa_inputs.random_small(COMBOS.index((dtype, d, bs, g)), num_seqs=5, max_len=150,
+                                     num_heads=hk * g, num_kv_heads=hk, head_dim=d,
+                                     block_size=bs, dtype=dtype, zero_len=True)
+    problem.context_lens[0] = 1             # single token
+    problem.context_lens[1] = 0             # empty sequence
+    problem.context_lens[2] = bs            # exactly one full block
+    data = pa_inputs.materialize(problem, "cuda")
+    ref = oracle_decode(data, problem)
+    assert_close(run_decode(data, problem), ref)
+    assert_close(run_decode(data, problem, split=True, partition=2 * bs), ref)
+    device_clean()
+
+
+@pytest.mark.parametrize("ctas", [1, 2, 4, 8])
+def test_cluster_split_agrees(ctas):
+    problem = pa_inputs.random_small(77, num_seqs=6, max_len=900, num_heads=16, num_kv_heads=4,
+                                     head_dim=128, block_size=16, dtype="bf16")
+    problem.context_lens[0] = 3
+    data = pa_inputs.materialize(problem, "cuda")
+    ref = oracle_decode(data, problem)
+    pa.pa_set_option("decode_split_ctas", ctas)
+    try:
+        assert_close(run_decode(data, problem), ref)
+    finally:
+        pa.pa_set_option("decode_split_ctas", 0)
+    device_clean()
+
+
+def test_permutation_invariance_bitwise():
+    """The same logical tokens under three physical placements give the same
+    bits: the kernel's arithmetic depends on logical order only."""
+    rng = np.random.default_rng(5)
+    length, hk, d, bs, hq = 333, 8, 128, 16, 32
+    n = -(-length // bs)
+    key = torch.randn((n * bs, hk, d), device="cuda").to(torch.bfloat16)
+    val = torch.randn((n * bs, hk, d), device="cuda").to(torch.bfloat16)
+    q = torch.randn((1, hq, d), device="cuda").to(torch.bfloat16)
+    outs = []
+    for trial in range(3):
+        nb = n + 50
+        perm = rng.permutation(nb)[:n]
+        kc = torch.full((nb, bs, hk, d), float("nan"), device="cuda", dtype=torch.bfloat16)
+        vc = kc.clone()
+        kc[torch.from_numpy(perm).cuda()] = key.view(n, bs, hk, d)
+        vc[torch.from_numpy(perm).cuda()] = val.view(n, bs, hk, d)
+        table = torch.from_numpy(perm.astype(np.int32)[None]).cuda()
+        out = torch.empty_like(q)
+        pa.pa_decode(out, q, kc, vc, table, torch.tensor([length], dtype=torch.int32,
+                                                         device="cuda"), d ** -0.5)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert same_bits(outs[0], outs[1]) and same_bits(outs[0], outs[2])
+    device_clean()
+
+
+def test_mha_workload_sampled():
+    """Batch 64, 32 q = 32 kv heads, lengths U[128, 2048], 8192-block pool."""
+    problem = pa_inputs.mha()
+    data = pa_inputs.materialize(problem, "cuda")
+    got = run_decode(data, problem)
+    seqs = [0, 1, 17, 40, 63, int(np.argmax(problem.context_lens))]
+    ref = oracle_decode(data, problem, seqs=seqs)
+    assert_close(got[seqs], ref[seqs])
+    device_clean()
+
+
+def test_gqa_workload_sampled():
+    """Batch 256, 32 q / 8 kv heads, lognormal lengths, pool 110 % of use."""
+    problem = pa_inputs.gqa()
+    data = pa_inputs.materialize(problem, "cuda")
+    got = run_decode(data, problem)
+    lens = problem.context_lens
+    seqs = sorted({0, 5, 99, 255, int(np.argmax(lens)), int(np.argmin(lens))})
+    ref = oracle_decode(data, problem, seqs=seqs)
+    assert_close(got[seqs], ref[seqs])
+    got_split = run_decode(data, problem, split=True, partition=512)
+    assert_close(got_split[seqs], ref[seqs])
+    assert not torch.isnan(got).any()
+    device_clean()
+
+
+def test_split_partition_sizes():
+    problem = pa_inputs.random_small(3, num_seqs=7, max_len=3000, num_heads=32, num_kv_heads=8,
+                                     head_dim=128, block_size=16, dtype="bf16")
+    data = pa_inputs.materialize(problem, "cuda")
+    ref = oracle_decode(data, problem)
+    for part in (16, 64, 512, 4096):
+        assert_close(run_decode(data, problem, split=True, partition=part), ref)
+    device_clean()
+
+
+def test_long_context_split():
+    """Sequences of 262144 and 1048576 tokens, 32 q / 8 kv heads, 512-token
+    partitions merged by log-sum-exp; every output against the oracle."""
+    problem = pa_inputs.long_context()
+    data = pa_inputs.materialize(problem, "cuda")
+    got = run_decode(data, problem, split=True, partition=512)
+    got1 = run_decode(data, problem, split=False)       # single pass (cluster split)
+    kc, vc, q = data["k_cache"].cpu(), data["v_cache"].cpu(), data["q"].cpu()
+    del data
+    for s in range(problem.num_seqs):
+        ref = oracle.paged_decode(q[s:s + 1], kc, vc, problem.block_tables[s:s + 1],
+                                  problem.context_lens[s:s + 1], problem.scale)
+        assert_close(got[s:s + 1], ref)
+        assert_close(got1[s:s + 1], ref)
+    device_clean()
