@@ -1,0 +1,622 @@
+#!/usr/bin/env python
+"""Paged-decode benchmark: KV-read GB/s and tokens/s on B200, as a fraction of
+the HBM roofline.
+
+One step of the decode loop (the whole hot path for one batch):
+  host allocator appends one token to every sequence (new block when the last
+  one is full, copy-on-write when it is shared) -> pa_copy_blocks for any
+  copy-on-write pairs -> pa_reshape_and_cache writes the new tokens' K/V ->
+  pa_decode (or pa_decode_split) attends every query head over its sequence.
+
+Default workload: GQA decode, batch 256, 32 q / 8 kv heads, head_dim 128,
+block 16, bf16, lognormal context lengths (median 1024, sigma 0.5, cap 8192),
+pool 110 % of the blocks in use, synthetic N(0,1) data.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+                  [--workload gqa|mha|long] [--kernel decode|split]
+
+Reported line (rank 0):
+  value      KV-read GB/s over the K timed steps, inputs resident in HBM
+             (per-step allocator outputs are computed before timing), max
+             over ranks, whole job (all replicas).
+  e2e        the same metric through the public API with host buffers: the
+             live allocator on the host, pinned H2D copies of each step's
+             q / new K,V / slots / lengths / table, and a D2H read of the
+             step's output, all inside the timed region.
+  roofline   the decode kernel: algorithmic bytes per launch / mean launch
+             time (CUDA events on the launching stream) vs measured HBM GB/s.
+  cpu_baseline  the fp64 oracle on the host's cores, bounded sample.
+Multi-GPU: the decode path is not sharded; N GPUs run N independent replicas
+("scaling": "weak"), one process per GPU, timings max-reduced over NCCL.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import pa_inputs  # noqa: E402
+
+METRIC = "paged decode KV-read GB/s and tokens/s at 1 B200, as fraction of HBM peak"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+KERNEL_SOURCES = ["paged_kv_cache_359_b200/csrc/decode.cuh",
+                  "paged_kv_cache_359_b200/csrc/common.cuh",
+                  "paged_kv_cache_359_b200/csrc/launch.cuh"]
+TRAFFIC_SUMMARY = "profiles/decode_gqa_b256_traffic.txt"
+
+
+# --------------------------------------------------------------------------
+# ranks
+# --------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(world, backend):
+    if world > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_scalar(x: float, op: str, world: int, device) -> float:
+    """max or sum of a scalar over ranks (identity at world size 1)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    red = torch.distributed.ReduceOp.MAX if op == "max" else torch.distributed.ReduceOp.SUM
+    torch.distributed.all_reduce(t, op=red)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# --------------------------------------------------------------------------
+# clocks (NVML, sampled in a thread during the timed region)
+# --------------------------------------------------------------------------
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            handle = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                handle = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._h = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # no NVML: report no clocks rather than guess
+            self._nv = None
+            self.error = f"nvml unavailable: {e}"
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in REASON_BITS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+               "samples": len(self.samples), "source": "nvml"}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+# --------------------------------------------------------------------------
+# workload
+# --------------------------------------------------------------------------
+
+def make_problem(name: str, extra_tokens: int, rank: int):
+    if name == "gqa":
+        return pa_inputs.gqa(extra_tokens=extra_tokens)
+    if name == "mha":
+        p = pa_inputs.mha(max_len=2048 + extra_tokens,
+                          num_blocks=8192 + 64 * (-(-extra_tokens // 16) + 1))
+        return p
+    if name == "long":
+        p = pa_inputs.long_context()
+        # room for the appended tokens
+        extra_blocks = 2 * (-(-extra_tokens // 16) + 1)
+        nb = p.num_blocks + extra_blocks
+        rng = np.random.default_rng(p.seed + 11)
+        order = rng.permutation(nb).astype(np.int32)
+        max_blocks = p.max_blocks_per_seq + extra_blocks
+        tables = pa_inputs.tables_from_order(p.context_lens, order, 16, max_blocks)
+        p.num_blocks, p.free_order, p.block_tables = nb, order, tables
+        return p
+    raise ValueError(f"unknown workload {name}")
+
+
+def decode_kv_bytes(lens: np.ndarray, problem) -> int:
+    return int(lens.astype(np.int64).sum()) * problem.num_kv_heads * problem.head_dim * 2 * \
+        problem.elem_bytes
+
+
+def decode_alg_bytes(lens: np.ndarray, problem) -> int:
+    """K/V rows read + q read + out written + block-table entries + lengths."""
+    s = len(lens)
+    qo = 2 * s * problem.num_heads * problem.head_dim * problem.elem_bytes
+    tab = 4 * int(sum(-(-int(x) // problem.block_size) for x in lens)) + 4 * s
+    return decode_kv_bytes(lens, problem) + qo + tab
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """(DRAM bytes, algorithmic bytes) of the decode launch in the committed
+    ncu summary, if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, TRAFFIC_SUMMARY)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    if fields.get("kernel_sources_sha256_16") != kernel_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"]), float(fields["alg_bytes_of_captured_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs: torch copy, read+write)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
+
+
+class DecodeLoop:
+    """State of one replica's decode loop: cache pool, host allocator, tables."""
+
+    def __init__(self, problem, device, kernel: str, partition: int):
+        import paged_kv_cache_359_b200 as pa
+        self.pa = pa
+        self.p = problem
+        self.device = device
+        self.kernel = kernel
+        self.partition = partition
+        data = pa_inputs.materialize(problem, device)
+        self.k_cache, self.v_cache = data["k_cache"], data["v_cache"]
+        self.q0 = data["q"]
+        s, cap = problem.num_seqs, problem.max_blocks_per_seq
+        self.alloc = pa.BlockAllocator(problem.num_blocks, problem.block_size, problem.free_order)
+        self.tables = np.full((s, cap), -1, dtype=np.int32)
+        self.lens = np.zeros(s, dtype=np.int32)
+        for i in range(s):
+            _, _, ln = self.alloc.extend(self.tables[i], 0, int(problem.context_lens[i]),
+                                         want_slots=False)
+            self.lens[i] = ln
+        n = -(-self.lens // problem.block_size)
+        for i in range(s):
+            assert (self.tables[i, :n[i]] == problem.block_tables[i, :n[i]]).all()
+        self.out = torch.empty_like(self.q0)
+        self.ws = None
+        self.max_len_cap = cap * problem.block_size
+
+    def workspace(self, max_len):
+        need = self.pa.pa_decode_split_workspace_bytes(self.p.num_seqs, self.p.num_heads,
+                                                       self.p.head_dim, max_len, self.partition)
+        if self.ws is None or self.ws.numel() < need:
+            self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self.ws
+
+    def launches_per_step(self, n_cow: int) -> int:
+        return (1 if n_cow else 0) + 1 + (2 if self.kernel == "split" else 1)
+
+    def decode(self, q, tables_d, lens_d, max_len):
+        if self.kernel == "split":
+            self.pa.pa_decode_split(self.out, q, self.k_cache, self.v_cache, tables_d, lens_d,
+                                    self.p.scale, max_len, self.partition, self.workspace(max_len))
+        else:
+            self.pa.pa_decode(self.out, q, self.k_cache, self.v_cache, tables_d, lens_d,
+                              self.p.scale)
+
+
+def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_index: int):
+    """Allocator outputs for every step are computed up front and uploaded;
+    the timed region holds only device work on inputs resident in HBM."""
+    pa, p, dev = loop.pa, loop.p, loop.device
+    total = steps + warmup
+    slots, cows, tabs, lens = [], [], [], []
+    for _ in range(total):
+        sl, cw = loop.alloc.append_slots(loop.tables, loop.lens)
+        slots.append(sl.copy())
+        cows.append(cw.astype(np.int64))
+        tabs.append(loop.tables.copy())
+        lens.append(loop.lens.copy())
+    slots_d = torch.from_numpy(np.stack(slots)).to(dev)
+    tabs_d = torch.from_numpy(np.stack(tabs)).to(dev)
+    lens_d = torch.from_numpy(np.stack(lens)).to(dev)
+    cows_d = [torch.from_numpy(c).to(dev) if len(c) else None for c in cows]
+    keys, vals, qs = [], [], []
+    for st in range(total):
+        t = pa_inputs.step_tokens(p.num_seqs, p.num_heads, p.num_kv_heads, p.head_dim, p.dtype,
+                                  p.seed, st, dev)
+        keys.append(t["key"]); vals.append(t["value"]); qs.append(t["q"])
+    max_lens = [int(x.max()) for x in lens]
+    stream = torch.cuda.current_stream()
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+
+    def step(i, timed_index=None):
+        if cows_d[i] is not None:
+            pa.pa_copy_blocks(loop.k_cache, loop.v_cache, cows_d[i])
+        pa.pa_reshape_and_cache(keys[i], vals[i], loop.k_cache, loop.v_cache, slots_d[i])
+        if timed_index is not None:
+            dec_ev[timed_index][0].record(stream)
+        loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
+        if timed_index is not None:
+            dec_ev[timed_index][1].record(stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev_index) as clocks:
+        t0.record(stream)
+        for j in range(steps):
+            step(warmup + j, j)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    flags = pa.pa_device_error(clear=True)
+    if flags:
+        raise RuntimeError(f"device error word 0x{flags:x} during the timed region")
+    ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+    timed_lens = lens[warmup:]
+    kv = sum(decode_kv_bytes(x, p) for x in timed_lens)
+    alg = [decode_alg_bytes(x, p) for x in timed_lens]
+    launches = sum(loop.launches_per_step(len(c)) for c in cows[warmup:])
+    return {"ms": ms, "kv_bytes": kv, "dec_ms": dec_ms, "dec_alg_bytes": alg,
+            "launches": launches, "clocks": clocks.summary(),
+            "tokens": steps * p.num_seqs,
+            "cow_pairs": int(sum(len(c) for c in cows[warmup:]))}
+
+
+def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int):
+    """Through the public API from host buffers: live allocator, pinned H2D of
+    every step's inputs, D2H of every step's output, all timed."""
+    pa, p, dev = loop.pa, loop.p, loop.device
+    total = steps + warmup
+    pin = lambda t: t.pin_memory()
+    host = []
+    for st in range(total):
+        t = pa_inputs.step_tokens(p.num_seqs, p.num_heads, p.num_kv_heads, p.head_dim, p.dtype,
+                                  p.seed + 1, st, "cpu")
+        host.append((pin(t["q"]), pin(t["key"]), pin(t["value"])))
+    s, cap = loop.tables.shape
+    tables_h = torch.from_numpy(loop.tables).pin_memory()
+    lens_h = torch.from_numpy(loop.lens).pin_memory()
+    tables_np, lens_np = tables_h.numpy(), lens_h.numpy()
+    slots_h = torch.zeros(s, dtype=torch.int64).pin_memory()
+    cows_h = torch.zeros((s, 2), dtype=torch.int64).pin_memory()
+    out_h = torch.empty(tuple(loop.out.shape), dtype=loop.out.dtype).pin_memory()
+    q_d = torch.empty_like(loop.q0)
+    k_d = torch.empty((s, p.num_kv_heads, p.head_dim), dtype=loop.q0.dtype, device=dev)
+    v_d = torch.empty_like(k_d)
+    tables_d = torch.empty((s, cap), dtype=torch.int32, device=dev)
+    lens_d = torch.empty(s, dtype=torch.int32, device=dev)
+    slots_d = torch.empty(s, dtype=torch.int64, device=dev)
+    cows_d = torch.empty((s, 2), dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+    h2d = d2h = 0
+    kv = 0
+
+    def step(i):
+        nonlocal h2d, d2h, kv
+        sl, cw = loop.alloc.append_slots(tables_np, lens_np)
+        slots_h.numpy()[:] = sl
+        n = len(cw)
+        if n:
+            cows_h.numpy()[:n] = cw
+        q_h, k_h, v_h = host[i]
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        slots_d.copy_(slots_h, non_blocking=True)
+        lens_d.copy_(lens_h, non_blocking=True)
+        tables_d.copy_(tables_h, non_blocking=True)
+        nb = (q_h.numel() * q_h.element_size() + 2 * k_h.numel() * k_h.element_size() +
+              8 * s + 4 * s + 4 * s * cap)
+        if n:
+            cows_d[:n].copy_(cows_h[:n], non_blocking=True)
+            nb += 16 * n
+            pa.pa_copy_blocks(loop.k_cache, loop.v_cache, cows_d[:n])
+        pa.pa_reshape_and_cache(k_d, v_d, loop.k_cache, loop.v_cache, slots_d)
+        loop.decode(q_d, tables_d, lens_d, int(lens_np.max()))
+        out_h.copy_(loop.out, non_blocking=True)
+        stream.synchronize()
+        return nb, out_h.numel() * out_h.element_size(), decode_kv_bytes(lens_np, p)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for j in range(steps):
+        a, b, c = step(warmup + j)
+        h2d += a; d2h += b; kv += c
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return {"ms": t0.elapsed_time(t1), "kv_bytes": kv, "h2d": h2d / steps, "d2h": d2h / steps}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_sample_seconds(problem, k_cache, v_cache, q, tables, lens, seqs):
+    import oracle
+    t = time.perf_counter()
+    oracle.paged_decode(q, k_cache, v_cache, tables, lens, problem.scale, seqs=seqs)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(loop: DecodeLoop, budget_s: float = 15.0):
+    """The oracle, as it stands, on this host's cores: whole-batch decode
+    steps over the current cache until about ``budget_s`` of CPU work."""
+    p = loop.p
+    kc, vc, q = loop.k_cache.cpu(), loop.v_cache.cpu(), loop.q0.cpu()
+    tables, lens = loop.tables.copy(), loop.lens.copy()
+    seqs_all = list(range(p.num_seqs))
+    done_bytes, done_secs, steps = 0, 0.0, 0
+    chunk = max(1, p.num_seqs // 8)
+    i = 0
+    while done_secs < budget_s and steps < 8 * 8:
+        seqs = seqs_all[(i * chunk) % p.num_seqs:][:chunk]
+        i += 1
+        done_secs += oracle_sample_seconds(p, kc, vc, q, tables, lens, seqs)
+        done_bytes += decode_kv_bytes(lens[seqs], p)
+        steps += 1
+    return {"value": done_bytes / done_secs / 1e9, "unit": "GB/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"{steps} chunks of {chunk} sequences ({done_secs:.1f} s of fp64 oracle "
+                      f"decode over the current cache; host os.cpu_count()={os.cpu_count()})",
+            "tokens_per_s": steps * chunk / done_secs}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the oracle times the same decode loop on the host's
+    cores; each step appends one token per sequence (oracle allocator and
+    cache write) and decodes a rotating sample of the batch."""
+    import oracle
+    if world > 1 and rank != 0:
+        return
+    extra = args.steps + args.warmup + 2
+    p = make_problem(args.workload, extra, 0)
+    data = pa_inputs.materialize(p, "cpu")
+    kc, vc = data["k_cache"], data["v_cache"]
+    alloc = oracle.BlockAllocator(p.num_blocks, p.block_size, p.free_order)
+    tables, lens = [], []
+    for x in p.context_lens:
+        t = []
+        _, _, ln = oracle.extend(alloc, t, 0, int(x))
+        tables.append(t)
+        lens.append(ln)
+    sample = max(1, min(p.num_seqs, args.ref_sample))
+    total_bytes, total_s, tokens = 0, 0.0, 0
+    for st in range(args.warmup + args.steps):
+        new = pa_inputs.step_tokens(p.num_seqs, p.num_heads, p.num_kv_heads, p.head_dim, p.dtype,
+                                    p.seed, st, "cpu")
+        t0 = time.perf_counter()
+        slots, cows = oracle.append_slots(alloc, tables, lens)
+        if cows:
+            kc, vc = oracle.copy_blocks(kc, vc, cows)
+        kc, vc = oracle.reshape_and_cache(new["key"], new["value"], kc, vc, slots)
+        seqs = [(st * sample + j) % p.num_seqs for j in range(sample)]
+        tab = np.full((p.num_seqs, max(len(t) for t in tables)), -1, dtype=np.int32)
+        for i, t in enumerate(tables):
+            tab[i, :len(t)] = t
+        oracle.paged_decode(new["q"], kc, vc, tab, lens, p.scale, seqs=seqs)
+        dt = time.perf_counter() - t0
+        if st >= args.warmup:
+            total_s += dt
+            total_bytes += decode_kv_bytes(np.asarray(lens)[seqs], p)
+            tokens += sample
+    value = total_bytes / total_s / 1e9
+    cores = torch.get_num_threads()
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total_s / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(p, args),
+        "cpu_baseline": {"kind": "oracle", "cores": cores, "value": round(value, 4),
+                         "unit": "GB/s",
+                         "sample": f"each step: allocator + cache write for all {p.num_seqs} "
+                                   f"sequences, fp64 decode of {sample} of them (rotating)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "tokens_per_s": round(tokens / total_s, 2),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(p, args):
+    lens = p.context_lens
+    return {"workload": {"gqa": "gqa_decode_b256", "mha": "mha_decode_b64",
+                         "long": "long_context_split"}[args.workload],
+            "num_seqs": p.num_seqs, "num_heads": p.num_heads, "num_kv_heads": p.num_kv_heads,
+            "head_dim": p.head_dim, "block_size": p.block_size, "num_blocks": p.num_blocks,
+            "context_len_median": int(np.median(lens)), "context_len_max": int(lens.max()),
+            "context_tokens": int(lens.astype(np.int64).sum()),
+            "kernel": args.kernel, "partition": args.partition,
+            "l2": "inputs larger than L2 (KV cache %.2f GB vs 126 MB L2), no flush" %
+                  (decode_kv_bytes(lens, p) / 1e9)}
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["gqa", "mha", "long"], default="gqa")
+    ap.add_argument("--kernel", choices=["decode", "split"], default=None)
+    ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-sample", type=int, default=64,
+                    help="sequences decoded per step by the reference arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.kernel is None:
+        args.kernel = "split" if args.workload == "long" else "decode"
+    rank, world, local = dist_env()
+    if world != args.gpus and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+
+    if args.impl == "reference":
+        dist_init(world, "gloo")
+        try:
+            run_reference(args, rank, world)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    try:
+        extra = 2 * (args.steps + args.warmup) + 4
+        p = make_problem(args.workload, extra, rank)
+        loop = DecodeLoop(p, dev, args.kernel, args.partition)
+        res = run_device_timed(loop, args.steps, args.warmup, world, local)
+        e2e = None if args.no_e2e else run_e2e(loop, args.steps, args.warmup, world)
+
+        ms = reduce_scalar(res["ms"], "max", world, dev)
+        kv_all = reduce_scalar(res["kv_bytes"], "sum", world, dev)
+        tokens_all = reduce_scalar(res["tokens"], "sum", world, dev)
+        secs = ms / 1e3
+        value = kv_all / secs / 1e9
+        dec_mean_ms = statistics.fmean(res["dec_ms"])
+        dec_alg = statistics.fmean(res["dec_alg_bytes"])
+        achieved = dec_alg / (dec_mean_ms / 1e3) / 1e9
+        peak, peak_src = hbm_peak()
+        cap = measured_traffic()
+        # scaled from the captured launch to this run's mean launch by
+        # algorithmic bytes (DRAM traffic grows with the tokens read)
+        traffic = None if cap is None else round(cap[0] * dec_alg / cap[1])
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if p.dtype == "bf16" else "f32",
+            "data": "synthetic", "config": workload_config(p, args),
+            "tokens_per_s": round(tokens_all / secs, 1),
+            "frac_of_nominal_8tbps": round(value / NOMINAL_HBM_GBS, 4),
+            "roofline": {"bound": "hbm", "kernel": "pa_decode" if args.kernel == "decode"
+                         else "pa_decode_split (partition + reduce)",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                         "frac_of_nominal_8tbps": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "traffic": traffic,
+                         "alg_bytes_per_launch": int(dec_alg),
+                         "mean_launch_ms": round(dec_mean_ms, 5)},
+            "gpu_launches": int(reduce_scalar(res["launches"], "sum", world, dev)),
+            "clocks": res["clocks"],
+            "cow_pairs_timed": res["cow_pairs"],
+        }
+        if e2e is not None:
+            e2e_ms = reduce_scalar(e2e["ms"], "max", world, dev)
+            e2e_kv = reduce_scalar(e2e["kv_bytes"], "sum", world, dev)
+            line["e2e"] = {"value": round(e2e_kv / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+                           "h2d_bytes_per_step": int(e2e["h2d"]),
+                           "d2h_bytes_per_step": int(e2e["d2h"]),
+                           "ms_per_step": round(e2e_ms / args.steps, 4)}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(loop)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

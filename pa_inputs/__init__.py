@@ -200,11 +200,16 @@ def prefix(block_size: int = 16, head_dim: int = 128, aligned: bool = False,
 
 def random_small(seed: int, num_seqs: int, max_len: int, num_heads: int,
                  num_kv_heads: int, head_dim: int, block_size: int, dtype: str,
-                 slack_blocks: int = 3, zero_len: bool = False) -> PagedProblem:
-    """Small random problems for parity sweeps (ragged lengths, optional L=0)."""
+                 slack_blocks: int = 3, zero_len: bool = False,
+                 fixed: Optional[dict] = None) -> PagedProblem:
+    """Small random problems for parity sweeps (ragged lengths, optional L=0).
+    ``fixed`` pins chosen sequences' lengths ({index: length}) before the
+    tables are built."""
     rng = np.random.default_rng(SEED_BASE + 1000 + seed)
     lo = 0 if zero_len else 1
     lengths = rng.integers(lo, max_len + 1, size=num_seqs).astype(np.int32)
+    for i, n in (fixed or {}).items():
+        lengths[i] = n
     in_use = int(sum(blocks_for(x, block_size) for x in lengths))
     nb = in_use + slack_blocks
     max_blocks = blocks_for(max_len, block_size) + 1

@@ -115,12 +115,17 @@ pa_status check_decode_args(void* out, const void* q, const void* kc, const void
     return PA_OK;
 }
 
+// CTAs per (sequence, kv head) for pa_decode.  Splitting costs a cluster
+// merge and shortens every CTA's stream, so it only pays when the grid
+// would otherwise leave SMs idle: grow the cluster while there are fewer
+// (sequence, kv head) pairs than two per SM and each CTA keeps at least
+// 1024 tokens of its sequence's capacity.
 int auto_decode_ctas(int num_seqs, int num_kv_heads, int max_blocks, int block_size) {
     const int64_t max_tokens = (int64_t)max_blocks * block_size;
     const int64_t work = (int64_t)num_seqs * num_kv_heads;
-    const int64_t target = 16LL * num_sms();
+    const int64_t target = 2LL * num_sms();
     int c = 1;
-    while (c < 8 && max_tokens / c > 2048 && work * c < target) c *= 2;
+    while (c < 8 && work * c < target && max_tokens / (2 * c) >= 1024) c *= 2;
     return c;
 }
 

@@ -52,12 +52,11 @@ COMBOS = [(dt, d, bs, g) for dt in ("bf16", "f32") for d in (64, 128, 256)
 @pytest.mark.parametrize("dtype,d,bs,g", COMBOS)
 def test_decode_all_instances_small(dtype, d, bs, g):
     hk = 2
+    # a single token, an empty sequence, exactly one full block, two ragged
     problem = pa_inputs.random_small(COMBOS.index((dtype, d, bs, g)), num_seqs=5, max_len=150,
                                      num_heads=hk * g, num_kv_heads=hk, head_dim=d,
-                                     block_size=bs, dtype=dtype, zero_len=True)
-    problem.context_lens[0] = 1             # single token
-    problem.context_lens[1] = 0             # empty sequence
-    problem.context_lens[2] = bs            # exactly one full block
+                                     block_size=bs, dtype=dtype, zero_len=True,
+                                     fixed={0: 1, 1: 0, 2: bs})
     data = pa_inputs.materialize(problem, "cuda")
     ref = oracle_decode(data, problem)
     assert_close(run_decode(data, problem), ref)
@@ -68,8 +67,7 @@ def test_decode_all_instances_small(dtype, d, bs, g):
 @pytest.mark.parametrize("ctas", [1, 2, 4, 8])
 def test_cluster_split_agrees(ctas):
     problem = pa_inputs.random_small(77, num_seqs=6, max_len=900, num_heads=16, num_kv_heads=4,
-                                     head_dim=128, block_size=16, dtype="bf16")
-    problem.context_lens[0] = 3
+                                     head_dim=128, block_size=16, dtype="bf16", fixed={0: 3})
     data = pa_inputs.materialize(problem, "cuda")
     ref = oracle_decode(data, problem)
     pa.pa_set_option("decode_split_ctas", ctas)

@@ -27,6 +27,7 @@ def build(problem):
     _, _, plen = oracle.extend(o, ot[0], 0, problem.prefix_len)
     _, _, plen_c = c.extend(ct[0], 0, problem.prefix_len)
     assert plen == plen_c
+    prefix_table = np.array(ot[0], dtype=np.int32)[None]   # before any copy-on-write
     n = -(-plen // bs)
     for i in range(1, s):
         ot[i] = oracle.fork(o, ot[0])
@@ -45,7 +46,7 @@ def build(problem):
     for i in range(s):
         tables[i, :len(ot[i])] = ot[i]
         assert list(ct[i, :len(ot[i])]) == ot[i]
-    return tables, np.array(lens, dtype=np.int32), slots, cows
+    return tables, np.array(lens, dtype=np.int32), slots, cows, prefix_table
 
 
 @pytest.mark.parametrize("aligned", [False, True])
@@ -53,7 +54,7 @@ def build(problem):
 @pytest.mark.parametrize("bs", [8, 16, 32])
 def test_prefix_sharing_copy_on_write(bs, d, aligned):
     problem = pa_inputs.prefix(bs, d, aligned=aligned)
-    tables, lens, slots, cows = build(problem)
+    tables, lens, slots, cows, prefix_table = build(problem)
     writers = int((problem.tail_lens > 0).sum())
     if aligned:
         assert not cows
@@ -64,7 +65,7 @@ def test_prefix_sharing_copy_on_write(bs, d, aligned):
 
     hk, dt = problem.num_kv_heads, pa_inputs.torch_dtype(problem.dtype)
     # pool: the prefix rows filled, everything else NaN
-    prefix_owned = pa_inputs.owned_rows(tables[:1], np.array([problem.prefix_len]), bs,
+    prefix_owned = pa_inputs.owned_rows(prefix_table, np.array([problem.prefix_len]), bs,
                                         problem.num_blocks)
     gen = pa_inputs.generator("cuda", problem.seed)
     kc = pa_inputs.poisoned_pool(problem.num_blocks, bs, hk, d, dt, gen, "cuda", prefix_owned)
