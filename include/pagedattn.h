@@ -160,6 +160,37 @@ pa_status pa_decode_split(void* out_d, const void* q_d,
                           pa_stream_t stream);
 
 /*
+ * pa_decode_split_noalloc -- pa_decode_split without a caller workspace.
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory where they decode: a plugin inside a host
+ * framework that owns all device memory and gives plugins none, or a
+ * serving process with a fixed memory budget that allows no allocation
+ * after start-up.  It takes pa_decode_split's arguments minus the workspace
+ * and uses a scratch array built into the library instead, so it allocates
+ * nothing (no cudaMalloc, no allocating library call).
+ *   Limit: a batch whose pa_decode_split_workspace_bytes(...) exceeds
+ *   PA_NOALLOC_SCRATCH_BYTES (16 MiB) is rejected with PA_ERR_UNSUPPORTED
+ *   before anything is launched.  Every GPU that loads the library holds
+ *   the 16 MiB until the process exits.
+ *   The first call on a device, with that device current, looks up the
+ *   scratch array's device address; make that first call before any
+ *   stream capture.
+ *   All calls share the one scratch array, which keeps the last call's
+ *   contents (nothing needs to start at zero).  Calls that overlap on the
+ *   GPU -- on different streams or from different host threads -- race on
+ *   it and corrupt each other's results: serialise them.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+
+pa_status pa_decode_split_noalloc(void* out_d, const void* q_d,
+                                  const void* k_cache_d, const void* v_cache_d,
+                                  const int32_t* block_tables_d, int max_blocks_per_seq,
+                                  const int32_t* context_lens_d, int num_seqs, int num_heads,
+                                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                  float scale, pa_dtype dtype, int max_context_len,
+                                  int partition_size, pa_stream_t stream);
+
+/*
  * pa_copy_blocks -- copy-on-write of shared blocks: for each pair
  * (src, dst) the whole key block and value block dst <- src ([course] 2.4.3:
  * a write to a block whose reference count exceeds one first copies it).

@@ -30,7 +30,7 @@ from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SP
 
 __all__ = [
     "pa_reshape_and_cache", "pa_decode", "pa_decode_split", "pa_decode_split_workspace_bytes",
-    "pa_copy_blocks", "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
+    "pa_decode_split_noalloc", "pa_copy_blocks", "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
     "PagedAttnError", "OutOfBlocks", "DEVERR_BITS",
 ]
 
@@ -112,6 +112,22 @@ def pa_decode_split(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                                 _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), s,
                                 hq, hk, d, bs, nb, float(scale), _dtype(q), int(max_context_len),
                                 int(partition_size), _ptr(workspace), nbytes, _stream(stream)))
+    return out
+
+
+def pa_decode_split_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            max_context_len, partition_size=512, stream=None):
+    """pa_decode_split for callers that cannot allocate device memory: the
+    library's built-in 16 MiB scratch replaces the caller workspace.  Calls
+    share that scratch, so calls that overlap on the GPU must not be issued."""
+    _dev(out, q, k_cache, v_cache, block_tables, context_lens)
+    s, hq, d = q.shape
+    nb, bs, hk, _ = k_cache.shape
+    check(lib().pa_decode_split_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(block_tables), block_tables.shape[1],
+                                        _ptr(context_lens), s, hq, hk, d, bs, nb, float(scale),
+                                        _dtype(q), int(max_context_len), int(partition_size),
+                                        _stream(stream)))
     return out
 
 
