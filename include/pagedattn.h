@@ -76,7 +76,7 @@ enum {
 
 typedef enum pa_option {
     PA_OPT_VALIDATE = 0,         /* 0/1: host-side index validation before launch */
-    PA_OPT_DECODE_SPLIT_CTAS = 1 /* pa_decode CTAs per (sequence, kv head): 0 = auto, 1, 2, 4, 8 */
+    PA_OPT_DECODE_SPLIT_CTAS = 1  /* pa_decode CTAs per (sequence, kv head): 0 = auto, 1, 2, 4, 8 */
 } pa_option;
 
 const char* pa_last_error(void);

@@ -155,7 +155,8 @@ pa_status fail(pa_status status, const char* fmt, ...) {
 }
 
 pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
-                           int num_kv_heads, int block_size, int num_blocks, int rows) {
+                           int num_kv_heads, int block_size, int num_blocks, int box_inner,
+                           int rows, bool swizzle128) {
     auto enc = tensor_map_encoder();
     if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     const cuuint64_t es = (cuuint64_t)elem_size(dtype);
@@ -163,13 +164,14 @@ pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, i
                           (cuuint64_t)num_blocks};
     cuuint64_t strides[3] = {head_dim * es, (cuuint64_t)num_kv_heads * head_dim * es,
                              (cuuint64_t)block_size * num_kv_heads * head_dim * es};
-    cuuint32_t box[4] = {(cuuint32_t)head_dim, 1, (cuuint32_t)rows, 1};
+    cuuint32_t box[4] = {(cuuint32_t)box_inner, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(map,
                      dtype == PA_DTYPE_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                            : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                      4, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return PA_OK;
@@ -291,6 +293,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     l.args.err = device_error_word();
     if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
     l.args.scale_log2 = scale * 1.4426950408889634f;
+    l.args.num_seqs = num_seqs;
     l.args.max_blocks = max_blocks_per_seq;
     l.args.max_tokens = max_blocks_per_seq * block_size;
     l.args.num_heads = num_heads;
@@ -305,6 +308,9 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     l.ctas = g_decode_ctas ? g_decode_ctas
                            : auto_decode_ctas(num_seqs, num_kv_heads, max_blocks_per_seq,
                                               block_size);
+    // one CTA per item: a longest-first grid; several CTAs per item: one
+    // cluster per (sequence, kv head)
+    l.args.sched = l.ctas > 1 ? SCHED_CLUSTER : SCHED_LPT;
     l.split = false;
     l.stream = st;
     return dispatch_decode(l, dtype, head_dim);
@@ -366,6 +372,7 @@ pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const v
     l.args.err = device_error_word();
     if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
     l.args.scale_log2 = scale * 1.4426950408889634f;
+    l.args.num_seqs = num_seqs;
     l.args.max_blocks = max_blocks_per_seq;
     l.args.max_tokens = max_blocks_per_seq * block_size;
     l.args.num_heads = num_heads;

@@ -7,39 +7,38 @@
 // query head h reads kv head h / G (G = num_heads / num_kv_heads).
 //
 // How (B200 design, not the pages' A100 sketch):
-//  * One CTA per (sequence, kv head[, partition or cluster rank]); all G
-//    query heads of the kv group share every K/V tile the CTA loads.
-//  * Work unit = R consecutive tokens of one block for one kv head: a K tile
-//    and a V tile of R rows x head_dim, each one 4-D TMA box
-//    {head_dim, 1, R, 1} over the cache viewed as
-//    [num_blocks][block_size][kv_heads][head_dim].  R is chosen so a tile is
-//    at most 4 KiB; with block_size 16 / head_dim 128 / bf16 a unit is one
-//    whole block.
+//  * Work item = (sequence, kv head): all G query heads of the kv group share
+//    every K/V tile the CTA loads.  pa_decode runs a persistent grid (about
+//    two CTAs per SM); every CTA sorts the context lengths in shared memory
+//    and takes items in snake order over the longest-first list, so long
+//    sequences start first and the CTAs finish together.  With few items a
+//    cluster of CTAs shares one item instead and merges through distributed
+//    shared memory; pa_decode_split gives every fixed token partition its
+//    own CTA and merges partitions with a log-sum-exp reduce kernel.
+//  * Unit = R consecutive tokens of one block for one kv head: a K tile and
+//    a V tile, each loaded by 4-D TMA boxes over the cache viewed as
+//    [num_blocks][block_size][kv_heads][head_dim].
 //  * Each of the NW warps owns a private ring of DEPTH stages with its own
 //    mbarriers: lane 0 issues the TMA loads DEPTH units ahead, all lanes wait
-//    on the stage's barrier (bounded), compute, and lane 0 refills the stage.
-//    Warps take units round-robin, so every warp streams independently and
-//    there is no CTA-wide barrier in the main loop.
+//    (bounded), compute, and lane 0 refills the stage.  Warps take units
+//    round-robin and stream independently; no CTA-wide barrier in the loop.
 //  * Block-table lookups are hoisted: every 32 units a warp loads the next 32
-//    block ids with one coalesced read (one id per lane) and hands them to
-//    lane 0 with a shuffle.
-//  * QK: a K row is spread over LPR lanes, 16 bytes per lane; each lane forms
-//    partial dot products for all G heads of its rows, then a butterfly
-//    reduce-scatter across the LPR lanes leaves every lane holding complete
-//    scores for a few (row, head) pairs.
-//  * Online softmax in fp32, in log2 units (q is pre-scaled by
-//    scale * log2 e), with a lazy running max: the accumulator is only
-//    rescaled when a score exceeds the current max by more than 2^8, which
-//    keeps exp2 arguments bounded and the result exact up to rounding.
-//  * PV: probabilities go through a tiny per-warp shared buffer so each lane
-//    reads the weights of its own rows, then fp32 FMAs into registers.
-//  * Warps merge through shared memory; the CTAs of a cluster (pa_decode on
-//    long sequences) merge through distributed shared memory; split-K
-//    partitions write (max, sum, unnormalised output) to a workspace for the
-//    log-sum-exp reduce kernel.
+//    block ids with one coalesced read and hands them to lane 0 by shuffle.
+//  * Online softmax in fp32, in log2 units, with a lazy running max: the
+//    accumulators are only rescaled when a score tops the current max by
+//    more than 2^8, which bounds every exp2 argument and keeps the result
+//    exact up to rounding.
+//  * Two unit policies.  MmaUnit (bf16, R = 16): QK^T and PV on the
+//    tensor cores with mma.sync m16n8k16 -- the G query rows of the group
+//    form the M side (padded to 16), tokens and head_dim the N/K sides; tiles
+//    arrive 128B-swizzled so ldmatrix reads them without bank conflicts.
+//    CoreUnit (fp32 caches, block 8): fp32 FMAs with 16-byte loads and a
+//    butterfly reduce-scatter across the lanes of a row.
 #pragma once
 
 #include <cooperative_groups.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -47,11 +46,19 @@ namespace pa {
 
 namespace cg = cooperative_groups;
 
-constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units: rescale when a score tops the max by 2^8
+constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
+constexpr int MAX_SORT = 1024;              // longest-first order up to this many sequences
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 __host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
+// pa_decode schedules.  LPT: one CTA per (sequence, kv head), CTA b runs the
+// item at position b of the longest-first list, so the hardware block
+// scheduler hands out the longest items first and back-fills SMs greedily
+// (longest-processing-time-first list scheduling).  CLUSTER: several CTAs
+// per item, merged through distributed shared memory (few, long items).
+enum Sched { SCHED_CLUSTER = 0, SCHED_LPT = 2 };
 
 struct DecodeArgs {
     void* out;                    // [S, Hq, D]
@@ -63,6 +70,7 @@ struct DecodeArgs {
     float* ws_o;                  // split: [S, Hq, max_parts, D] unnormalised output
     unsigned* err;                // device error word
     float scale_log2;             // scale * log2(e)
+    int num_seqs;
     int max_blocks;
     int max_tokens;               // max_blocks * block_size
     int num_heads;
@@ -70,352 +78,196 @@ struct DecodeArgs {
     int num_blocks;
     int part_tokens;              // split: partition size in tokens
     int max_parts;                // split: partitions per (sequence, head) in the workspace
+    int sched;                    // pa_decode: SCHED_CLUSTER or SCHED_LPT
 };
 
 enum class Mode { Decode, Split };
 
-template <typename T, int D, int BS, int G>
-struct Geom {
+// ============================================================ CoreUnit ==
+// fp32 FMA unit: a K/V row is spread over LPR lanes (16 bytes per lane), each
+// lane forms partial dot products for all G heads of its rows, a butterfly
+// reduce-scatter leaves every lane a few complete scores, probabilities go
+// through a per-warp shared buffer, PV is fp32 FMA into registers.
+template <typename T_, int D_, int BS_, int G_>
+struct CoreUnit {
+    using T = T_;
+    static constexpr int D = D_, BS = BS_, G = G_;
     static constexpr int ES = (int)sizeof(T);
-    static constexpr int VEC = 16 / ES;                 // elements per 16-byte vector
-    static constexpr int VPR = D / VEC;                 // vectors per K/V row
-    static constexpr int LPR = cmin(VPR, 32);           // lanes per row
-    static constexpr int VPL = VPR / LPR;               // vectors per lane per row
-    static constexpr int RPP = 32 / LPR;                // rows per warp pass
-    static constexpr int R = cmin(BS, cmax(RPP, 4096 / (D * ES)));   // rows per unit
+    static constexpr int VEC = 16 / ES;
+    static constexpr int VPR = D / VEC;
+    static constexpr int LPR = cmin(VPR, 32);
+    static constexpr int VPL = VPR / LPR;
+    static constexpr int RPP = 32 / LPR;
+    static constexpr int R = cmin(BS, cmax(RPP, 4096 / (D * ES)));
     static constexpr int PASSES = R / RPP;
-    static constexpr int N = PASSES * G;                // partial scores per lane per unit
+    static constexpr int N = PASSES * G;
     static constexpr int LOG_LPR = ilog2(LPR);
-    static constexpr int RS = cmin(LOG_LPR, ilog2(N));  // reduce-scatter steps
-    static constexpr int NH = N >> RS;                  // scores held per lane afterwards
-    static constexpr int DUP = LPR >> RS;               // lanes holding the same score
-    static constexpr int UNIT_BYTES = R * D * ES;       // one K (or V) tile
-    static constexpr int STAGE_BYTES = 2 * UNIT_BYTES;
-    static constexpr int NW = 4;                        // warps per CTA
-    static constexpr int DEPTH = cmin(8, cmax(3, 24576 / STAGE_BYTES));
-    static constexpr int STAGE_REGION = NW * DEPTH * STAGE_BYTES;
-    static constexpr int MERGE_FLOATS = (NW + 1) * G * (D + 2);
-    static constexpr int MAIN_REGION = cmax(STAGE_REGION, MERGE_FLOATS * 4);
-    static constexpr int PBUF_BYTES = NW * R * G * 4;
-    static constexpr int BAR_OFFSET = MAIN_REGION + PBUF_BYTES;
-    static constexpr int SMEM_BYTES = BAR_OFFSET + NW * DEPTH * 8;
-
+    static constexpr int RS = cmin(LOG_LPR, ilog2(N));
+    static constexpr int NH = N >> RS;
+    static constexpr int DUP = LPR >> RS;
+    static constexpr int BOX_INNER = D;
+    static constexpr int BOXES = 1;
+    static constexpr bool SWIZZLE128 = false;
+    static constexpr int PBUF_FLOATS = R * G;           // per warp
     static_assert(D % VEC == 0 && VPR % LPR == 0, "head_dim must be a multiple of 16 bytes");
     static_assert(BS % R == 0 && R % RPP == 0, "unit rows must tile the block");
     static_assert((N & (N - 1)) == 0, "power-of-two score count");
-    static_assert(MAIN_REGION % 16 == 0 && PBUF_BYTES % 16 == 0, "alignment");
-};
 
-// Process one unit (R rows of K and V) for one warp.
-template <typename T, int D, int BS, int G, bool MASKED>
-__device__ __forceinline__ void process_unit(
-    const T* __restrict__ ks, const T* __restrict__ vs, float* __restrict__ pbuf, int valid,
-    int lane, const float (&qf)[G][Geom<T, D, BS, G>::VPL][Geom<T, D, BS, G>::VEC],
-    float (&acc)[G][Geom<T, D, BS, G>::VPL][Geom<T, D, BS, G>::VEC], float (&m)[G],
-    float (&mh)[Geom<T, D, BS, G>::NH], float (&lh)[Geom<T, D, BS, G>::NH],
-    const int (&hg)[Geom<T, D, BS, G>::NH], const int (&hrow)[Geom<T, D, BS, G>::NH]) {
-    using Gm = Geom<T, D, BS, G>;
-    constexpr int VEC = Gm::VEC, VPL = Gm::VPL, LPR = Gm::LPR, RPP = Gm::RPP;
-    constexpr int PASSES = Gm::PASSES, N = Gm::N, NH = Gm::NH;
-    const int c = lane % LPR;
-    const int r = lane / LPR;
-
-    // ---- partial dot products q_g . k_row over this lane's slice of D ----
-    float x[N];
-#pragma unroll
-    for (int p = 0; p < PASSES; ++p) {
-        const int row = p * RPP + r;
-        float kf[VPL][VEC];
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-            const uint4 u = *reinterpret_cast<const uint4*>(ks + row * D + (v * LPR + c) * VEC);
-            Vec16<T>::to_float(u, kf[v]);
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float s = 0.f;
-#pragma unroll
-            for (int v = 0; v < VPL; ++v)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) s = fmaf(qf[g][v][e], kf[v][e], s);
-            x[p * G + g] = s;
-        }
-    }
-
-    // ---- butterfly reduce-scatter across the LPR lanes of a row ----
-#pragma unroll
-    for (int k = 0; k < Gm::RS; ++k) {
-        const int half = N >> (k + 1);
-        const bool upper = (lane >> k) & 1;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-            const float lo = x[i], hi = x[i + half];
-            const float send = upper ? lo : hi;
-            const float keep = upper ? hi : lo;
-            x[i] = keep + __shfl_xor_sync(FULL_MASK, send, 1 << k);
-        }
-    }
-#pragma unroll
-    for (int k = Gm::RS; k < Gm::LOG_LPR; ++k) x[0] += __shfl_xor_sync(FULL_MASK, x[0], 1 << k);
-
-    float sc[NH];
-#pragma unroll
-    for (int j = 0; j < NH; ++j) {
-        sc[j] = x[j];
-        if (MASKED && hrow[j] >= valid) sc[j] = -INFINITY;
-    }
-
-    // ---- lazy running max ----
-    bool grow = false;
-#pragma unroll
-    for (int j = 0; j < NH; ++j) grow |= sc[j] > mh[j] + RESCALE_THRESHOLD;
-    if (__any_sync(FULL_MASK, grow)) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float lm = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < NH; ++j)
-                if (hg[j] == g) lm = fmaxf(lm, sc[j]);
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1)
-                lm = fmaxf(lm, __shfl_xor_sync(FULL_MASK, lm, off));
-            const float mn = fmaxf(m[g], lm);
-            const float alpha = exp2_approx(m[g] - mn);
-            m[g] = mn;
-#pragma unroll
-            for (int v = 0; v < VPL; ++v)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[g][v][e] *= alpha;
-#pragma unroll
-            for (int j = 0; j < NH; ++j)
-                if (hg[j] == g) {
-                    lh[j] *= alpha;
-                    mh[j] = mn;
-                }
-        }
-    }
-
-    // ---- probabilities: keep the running sum, publish to the warp ----
-#pragma unroll
-    for (int j = 0; j < NH; ++j) {
-        const float pj = exp2_approx(sc[j] - mh[j]);
-        lh[j] += pj;
-        pbuf[hrow[j] * G + hg[j]] = pj;
-    }
-    __syncwarp();
-
-    // ---- PV ----
-#pragma unroll
-    for (int p = 0; p < PASSES; ++p) {
-        const int row = p * RPP + r;
-        float pv[G];
-        if constexpr (G % 4 == 0) {
-#pragma unroll
-            for (int g = 0; g < G; g += 4) {
-                const float4 w = *reinterpret_cast<const float4*>(pbuf + row * G + g);
-                pv[g] = w.x; pv[g + 1] = w.y; pv[g + 2] = w.z; pv[g + 3] = w.w;
-            }
-        } else if constexpr (G == 2) {
-            const float2 w = *reinterpret_cast<const float2*>(pbuf + row * G);
-            pv[0] = w.x; pv[1] = w.y;
-        } else {
-            pv[0] = pbuf[row];
-        }
-        float vf[VPL][VEC];
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) {
-            const uint4 u = *reinterpret_cast<const uint4*>(vs + row * D + (v * LPR + c) * VEC);
-            Vec16<T>::to_float(u, vf[v]);
-        }
-        if (MASKED && row >= valid) {
-            // rows past the end of the sequence may hold anything (NaN poison)
-#pragma unroll
-            for (int v = 0; v < VPL; ++v)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) vf[v][e] = 0.f;
-        }
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int v = 0; v < VPL; ++v)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[g][v][e] = fmaf(pv[g], vf[v][e], acc[g][v][e]);
-    }
-    __syncwarp();
-}
-
-template <typename T, int D, int BS, int G, Mode MODE>
-__global__ void __launch_bounds__(Geom<T, D, BS, G>::NW * 32)
-    paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
-    using Gm = Geom<T, D, BS, G>;
-    constexpr int NW = Gm::NW, DEPTH = Gm::DEPTH, R = Gm::R, VEC = Gm::VEC, VPL = Gm::VPL;
-    constexpr int LPR = Gm::LPR, NH = Gm::NH, N = Gm::N;
-    constexpr int NT = NW * 32;
-
-    const int seq = blockIdx.z;
-    const int kvh = blockIdx.y;
-    const int warp = threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
-
-    // ---- this CTA's share of the sequence, in units of R tokens ----
-    int L = a.context_lens[seq];
-    const int cap = a.max_tokens;
-    if (L < 0 || L > cap) {
-        if (threadIdx.x == 0) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
-        L = L < 0 ? 0 : cap;
-    }
-    const int total_units = (L + R - 1) / R;
-    int u_begin = 0, u_end = total_units, ctas = 1, crank = 0, part = 0, nparts = 1;
-    if constexpr (MODE == Mode::Split) {
-        part = blockIdx.x;
-        nparts = (L + a.part_tokens - 1) / a.part_tokens;
-        if (part >= cmax(nparts, 1)) return;            // whole CTA, before any barrier
-        if (nparts > a.max_parts) {
-            if (threadIdx.x == 0 && part == 0) raise_error(a.err, PA_DEVERR_WORKSPACE);
-            if (part > 0) return;
-            nparts = 1;                                  // degrade: partition 0 covers the rest
-            u_begin = 0;
-        } else {
-            u_begin = part * (a.part_tokens / R);
-            u_end = cmin(u_begin + a.part_tokens / R, total_units);
-        }
-    } else {
-        ctas = gridDim.x;
-        crank = blockIdx.x;
-    }
-    const int ustride = ctas * NW;
-    const int first = u_begin + crank + ctas * warp;
-    const int nk = first < u_end ? (u_end - first + ustride - 1) / ustride : 0;
-
-    extern __shared__ __align__(128) unsigned char smem[];
-    T* stage_base = reinterpret_cast<T*>(smem) + (size_t)warp * DEPTH * (2 * R * D);
-    float* pbuf = reinterpret_cast<float*>(smem + Gm::MAIN_REGION) + warp * R * G;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Gm::BAR_OFFSET) + warp * DEPTH;
-
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < DEPTH; ++s) mbar_init(&bars[s], 1);
-        fence_mbar_init();
-        if (warp == 0) {
-            prefetch_tensormap(&tm_k);
-            prefetch_tensormap(&tm_v);
-        }
-    }
-    __syncwarp();
-
-    const int c = lane % LPR;
-    const int r = lane / LPR;
-
-    // ---- queries of the kv group, pre-scaled into log2 units ----
     float qf[G][VPL][VEC];
-    {
-        const T* qb = reinterpret_cast<const T*>(a.q) +
-                      ((size_t)seq * a.num_heads + (size_t)kvh * G) * D;
+    float acc[G][VPL][VEC];
+    float m[G];
+    float mh[NH], lh[NH];
+    int hg[NH], hrow[NH];
+
+    __device__ __forceinline__ void begin(const T* qg, float scale_log2, int lane) {
+        const int c = lane % LPR, r = lane / LPR;
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
-                const uint4 u = *reinterpret_cast<const uint4*>(qb + g * D + (v * LPR + c) * VEC);
+                const uint4 u = *reinterpret_cast<const uint4*>(qg + g * D + (v * LPR + c) * VEC);
                 Vec16<T>::to_float(u, qf[g][v]);
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) qf[g][v][e] *= a.scale_log2;
+                for (int e = 0; e < VEC; ++e) {
+                    qf[g][v][e] *= scale_log2;
+                    acc[g][v][e] = 0.f;
+                }
             }
-    }
-
-    // ---- hoisted block-table window: lane i holds the block of unit k0+i ----
-    const int32_t* table = a.block_tables + (size_t)seq * a.max_blocks;
-    int win = 0;
-    auto load_window = [&](int k0) {
-        const int k = k0 + lane;
-        int id = 0;
-        if (k < nk) {
-            const int u = first + ustride * k;
-            id = __ldg(table + (u * R) / BS);
-            if (id < 0 || id >= a.num_blocks) {
-                raise_error(a.err, PA_DEVERR_BLOCK_ID);
-                id = a.num_blocks;        // out of the tensor map: TMA fills zeros
-            }
-        }
-        win = id;
-    };
-    auto issue = [&](int k, int id) {    // lane 0 only
-        const int s = k % DEPTH;
-        T* kdst = stage_base + (size_t)s * (2 * R * D);
-        const int u = first + ustride * k;
-        const int row0 = (u * R) % BS;
-        mbar_arrive_expect_tx(&bars[s], Gm::STAGE_BYTES);
-        tma_load_4d(kdst, &tm_k, &bars[s], 0, kvh, row0, id);
-        tma_load_4d(kdst + R * D, &tm_v, &bars[s], 0, kvh, row0, id);
-    };
-
-    load_window(0);
-    const int pro = cmin(DEPTH, nk);
-    for (int k = 0; k < pro; ++k) {
-        const int id = __shfl_sync(FULL_MASK, win, k);
-        if (lane == 0) issue(k, id);
-    }
-
-    // ---- per-lane softmax state ----
-    float m[G], acc[G][VPL][VEC], mh[NH], lh[NH];
-    int hg[NH], hrow[NH];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY;
-#pragma unroll
-        for (int v = 0; v < VPL; ++v)
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) acc[g][v][e] = 0.f;
-    }
-    {
+        for (int g = 0; g < G; ++g) m[g] = -INFINITY;
         int off = 0;
 #pragma unroll
-        for (int k = 0; k < Gm::RS; ++k) off += ((lane >> k) & 1) * (N >> (k + 1));
+        for (int k = 0; k < RS; ++k) off += ((lane >> k) & 1) * (N >> (k + 1));
 #pragma unroll
         for (int j = 0; j < NH; ++j) {
             const int gi = j + off;
             hg[j] = gi % G;
-            hrow[j] = (gi / G) * Gm::RPP + r;
+            hrow[j] = (gi / G) * RPP + r;
             mh[j] = -INFINITY;
             lh[j] = 0.f;
         }
     }
 
-    // ---- main loop over this warp's units ----
-    int k = 0;
-    bool failed = false;
-    for (; k < nk; ++k) {
-        const int s = k % DEPTH;
-        const uint32_t parity = (k / DEPTH) & 1;
-        const bool landed = __all_sync(FULL_MASK, mbar_wait_bounded(&bars[s], parity));
-        if (!landed) {
-            failed = true;
-            break;
+    template <bool MASKED>
+    __device__ __forceinline__ void unit(T* ks, T* vs, float* pbuf, int valid, int lane) {
+        const int c = lane % LPR, r = lane / LPR;
+        float x[N];
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) {
+            const int row = p * RPP + r;
+            float kf[VPL][VEC];
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                const uint4 u = *reinterpret_cast<const uint4*>(ks + row * D + (v * LPR + c) * VEC);
+                Vec16<T>::to_float(u, kf[v]);
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float s = 0.f;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) s = fmaf(qf[g][v][e], kf[v][e], s);
+                x[p * G + g] = s;
+            }
         }
-        const T* ks = stage_base + (size_t)s * (2 * R * D);
-        const int u = first + ustride * k;
-        const int valid = cmin(R, L - u * R);
-        if (valid == R)
-            process_unit<T, D, BS, G, false>(ks, ks + R * D, pbuf, valid, lane, qf, acc, m, mh,
-                                             lh, hg, hrow);
-        else
-            process_unit<T, D, BS, G, true>(ks, ks + R * D, pbuf, valid, lane, qf, acc, m, mh,
-                                            lh, hg, hrow);
-        const int kn = k + DEPTH;
-        if (kn < nk) {
-            if (kn % 32 == 0) load_window(kn);
-            const int id = __shfl_sync(FULL_MASK, win, kn % 32);
-            if (lane == 0) issue(kn, id);
+        // butterfly reduce-scatter across the LPR lanes of a row
+#pragma unroll
+        for (int k = 0; k < RS; ++k) {
+            const int half = N >> (k + 1);
+            const bool upper = (lane >> k) & 1;
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float lo = x[i], hi = x[i + half];
+                const float send = upper ? lo : hi;
+                const float keep = upper ? hi : lo;
+                x[i] = keep + __shfl_xor_sync(FULL_MASK, send, 1 << k);
+            }
         }
+#pragma unroll
+        for (int k = RS; k < LOG_LPR; ++k) x[0] += __shfl_xor_sync(FULL_MASK, x[0], 1 << k);
+
+        float sc[NH];
+#pragma unroll
+        for (int j = 0; j < NH; ++j) {
+            sc[j] = x[j];
+            if (MASKED && hrow[j] >= valid) sc[j] = -INFINITY;
+        }
+        bool grow = false;
+#pragma unroll
+        for (int j = 0; j < NH; ++j) grow |= sc[j] > mh[j] + RESCALE_THRESHOLD;
+        if (__any_sync(FULL_MASK, grow)) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float lm = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < NH; ++j)
+                    if (hg[j] == g) lm = fmaxf(lm, sc[j]);
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1)
+                    lm = fmaxf(lm, __shfl_xor_sync(FULL_MASK, lm, off));
+                const float mn = fmaxf(m[g], lm);
+                const float alpha = exp2_approx(m[g] - mn);
+                m[g] = mn;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[g][v][e] *= alpha;
+#pragma unroll
+                for (int j = 0; j < NH; ++j)
+                    if (hg[j] == g) {
+                        lh[j] *= alpha;
+                        mh[j] = mn;
+                    }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NH; ++j) {
+            const float pj = exp2_approx(sc[j] - mh[j]);
+            lh[j] += pj;
+            pbuf[hrow[j] * G + hg[j]] = pj;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) {
+            const int row = p * RPP + r;
+            float pv[G];
+            if constexpr (G % 4 == 0) {
+#pragma unroll
+                for (int g = 0; g < G; g += 4) {
+                    const float4 w = *reinterpret_cast<const float4*>(pbuf + row * G + g);
+                    pv[g] = w.x; pv[g + 1] = w.y; pv[g + 2] = w.z; pv[g + 3] = w.w;
+                }
+            } else if constexpr (G == 2) {
+                const float2 w = *reinterpret_cast<const float2*>(pbuf + row * G);
+                pv[0] = w.x; pv[1] = w.y;
+            } else {
+                pv[0] = pbuf[row];
+            }
+            float vf[VPL][VEC];
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                const uint4 u = *reinterpret_cast<const uint4*>(vs + row * D + (v * LPR + c) * VEC);
+                Vec16<T>::to_float(u, vf[v]);
+            }
+            if (MASKED && row >= valid) {
+                // rows past the end of the sequence may hold anything (NaN poison)
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) vf[v][e] = 0.f;
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[g][v][e] = fmaf(pv[g], vf[v][e], acc[g][v][e]);
+        }
+        __syncwarp();
     }
-    if (failed) {
-        // A load never landed: record it, wait (bounded) for this warp's
-        // other loads in flight so none lands after the CTA is gone, and
-        // contribute nothing.
-        if (lane == 0) raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
-        const int issued = cmin(nk, k + DEPTH);
-        for (int kk = k + 1; kk < issued; ++kk)
-            (void)mbar_wait_bounded(&bars[kk % DEPTH], (kk / DEPTH) & 1);
+
+    __device__ __forceinline__ void drop() {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             m[g] = -INFINITY;
@@ -428,54 +280,331 @@ __global__ void __launch_bounds__(Geom<T, D, BS, G>::NW * 32)
         for (int j = 0; j < NH; ++j) lh[j] = 0.f;
     }
 
-    // ---- finish the warp: sum rows across row groups, sums per head ----
+    // Warp partials into shared memory: wm/wl [NW][G], wacc [NW][G][D].
+    __device__ __forceinline__ void publish(float* wm, float* wl, float* wacc, int warp, int lane) {
+        const int c = lane % LPR, r = lane / LPR;
 #pragma unroll
-    for (int kk = Gm::LOG_LPR; kk < 5; ++kk)
+        for (int kk = LOG_LPR; kk < 5; ++kk)
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+            for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int v = 0; v < VPL; ++v)
+                for (int v = 0; v < VPL; ++v)
 #pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    acc[g][v][e] += __shfl_xor_sync(FULL_MASK, acc[g][v][e], 1 << kk);
-    float lsum[G];
+                    for (int e = 0; e < VEC; ++e)
+                        acc[g][v][e] += __shfl_xor_sync(FULL_MASK, acc[g][v][e], 1 << kk);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        float t = 0.f;
+        for (int g = 0; g < G; ++g) {
+            float t = 0.f;
 #pragma unroll
-        for (int j = 0; j < NH; ++j)
-            if (hg[j] == g) t += lh[j];
+            for (int j = 0; j < NH; ++j)
+                if (hg[j] == g) t += lh[j];
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) t += __shfl_xor_sync(FULL_MASK, t, off);
-        lsum[g] = t * (1.0f / Gm::DUP);
+            for (int off = 16; off >= 1; off >>= 1) t += __shfl_xor_sync(FULL_MASK, t, off);
+            if (lane == 0) {
+                wm[warp * G + g] = m[g];
+                wl[warp * G + g] = t * (1.0f / DUP);
+            }
+        }
+        if (r == 0)
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int v = 0; v < VPL; ++v)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e)
+                        wacc[(warp * G + g) * D + (v * LPR + c) * VEC + e] = acc[g][v][e];
+    }
+};
+
+// ============================================================= MmaUnit ==
+// Tensor-core unit for bf16: 16 tokens per unit.
+//   S[16 x 16] = Q[16 x D] K^T  (rows 0..G-1 = the group's query heads,
+//                               rows G..15 zero; 2 n-tiles of 8 tokens)
+//   O[16 x D] += P[16 x 16] V   (P = exp2(S - m) rounded to bf16; D/8 n-tiles)
+// The C fragment of the two S n-tiles is exactly the A fragment of P, so
+// probabilities never leave registers.  Thread `lane` owns row g = lane / 4
+// (its query head) and columns 2*(lane%4) + {0,1} of every n-tile.
+// K and V tiles arrive as head_dim/64 boxes of [16 rows][128 bytes] with the
+// 128-byte swizzle (16-byte chunk c of row r stored at chunk c ^ (r % 8)).
+template <int D_, int BS_, int G_>
+struct MmaUnit {
+    using T = __nv_bfloat16;
+    static constexpr int D = D_, BS = BS_, G = G_;
+    static constexpr int R = 16;
+    static constexpr int BOX_INNER = 64;
+    static constexpr int BOXES = D / 64;
+    static constexpr bool SWIZZLE128 = true;
+    static constexpr int KS = D / 16;            // QK k-steps
+    static constexpr int NT = D / 8;             // PV n-tiles
+    static constexpr int PBUF_FLOATS = 0;
+    static constexpr int BOX_BYTES = R * 128;
+    static_assert(G >= 1 && G <= 8 && BS % R == 0 && D % 64 == 0, "MmaUnit shape");
+
+    uint32_t qa[KS][2];     // A fragments of Q: row g, k-low and k-high halves
+    float o[NT][2];         // PV accumulators of row g (rows 8..15 are zero padding)
+    float m, l;             // row g: running max (log2 units) and this lane's partial sum
+    float scale_log2;
+
+    __device__ __forceinline__ void begin(const T* qg, float scale_log2_, int lane) {
+        scale_log2 = scale_log2_;
+        const int g = lane >> 2, c2 = 2 * (lane & 3);
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qg + g * D);
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            qa[k][0] = g < G ? __ldg(qrow + (16 * k + c2) / 2) : 0u;
+            qa[k][1] = g < G ? __ldg(qrow + (16 * k + 8 + c2) / 2) : 0u;
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = 0.f;
+        m = -INFINITY;
+        l = 0.f;
+    }
+
+    // byte offset of 16-byte chunk `chunk` (of D/8) in row `row` of a tile
+    static __device__ __forceinline__ uint32_t swz(int row, int chunk) {
+        return (uint32_t)((chunk >> 3) * BOX_BYTES + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+    }
+
+    template <bool MASKED>
+    __device__ __forceinline__ void unit(T* ks, T* vs, float*, int valid, int lane) {
+        const uint32_t kbase = smem_addr(ks), vbase = smem_addr(vs);
+        const int mi = lane >> 3, rr = lane & 7;
+        // ---- S = Q K^T: ldmatrix.x4 gives both n-tiles' B fragments for one k-step
+        float s0[2] = {0.f, 0.f}, s1[2] = {0.f, 0.f};
+        {
+            const int tok = 8 * (mi >> 1) + rr;
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                uint32_t b[4];
+                ldmatrix_x4(b, kbase + swz(tok, 2 * k + (mi & 1)));
+                mma_bf16_16816_top(s0[0], s0[1], qa[k][0], qa[k][1], b[0], b[1]);
+                mma_bf16_16816_top(s1[0], s1[1], qa[k][0], qa[k][1], b[2], b[3]);
+            }
+        }
+        const int c2 = 2 * (lane & 3);
+        float sc[4] = {s0[0] * scale_log2, s0[1] * scale_log2, s1[0] * scale_log2,
+                       s1[1] * scale_log2};
+        if (MASKED) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if ((j >> 1) * 8 + c2 + (j & 1) >= valid) sc[j] = -INFINITY;
+            // value rows past the end may hold NaN poison, and 0 * NaN = NaN
+            uint4* vz = reinterpret_cast<uint4*>(vs);
+            const int first = valid * 8, total = R * 8;        // 16-byte chunks per box
+#pragma unroll
+            for (int b = 0; b < BOXES; ++b)
+                for (int i = first + lane; i < total; i += 32)
+                    vz[b * (BOX_BYTES / 16) + i] = make_uint4(0u, 0u, 0u, 0u);
+            fence_proxy_async_smem();     // a later TMA load refills this stage
+            __syncwarp();
+        }
+        // ---- lazy running max over the row's 16 scores (4 lanes x 4)
+        const bool grow = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])) > m + RESCALE_THRESHOLD;
+        if (__any_sync(FULL_MASK, grow)) {
+            float rm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+            rm = fmaxf(rm, __shfl_xor_sync(FULL_MASK, rm, 1));
+            rm = fmaxf(rm, __shfl_xor_sync(FULL_MASK, rm, 2));
+            const float mn = fmaxf(m, rm);
+            const float alpha = exp2_approx(m - mn);
+            m = mn;
+            l *= alpha;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                o[n][0] *= alpha;
+                o[n][1] *= alpha;
+            }
+        }
+        float p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            p[j] = exp2_approx(sc[j] - m);
+            l += p[j];
+        }
+        const uint32_t pa0 = pack_bf16x2(p[0], p[1]);     // tokens c2, c2+1
+        const uint32_t pa2 = pack_bf16x2(p[2], p[3]);     // tokens 8+c2, 9+c2
+        // ---- O += P V: ldmatrix.x4.trans gives B fragments of two n-tiles
+        {
+            const int tok = 8 * (mi & 1) + rr;
+#pragma unroll
+            for (int j = 0; j < NT / 2; ++j) {
+                uint32_t b[4];
+                ldmatrix_x4_trans(b, vbase + swz(tok, 2 * j + (mi >> 1)));
+                mma_bf16_16816_top(o[2 * j][0], o[2 * j][1], pa0, pa2, b[0], b[1]);
+                mma_bf16_16816_top(o[2 * j + 1][0], o[2 * j + 1][1], pa0, pa2, b[2], b[3]);
+            }
+        }
+        __syncwarp();
+    }
+
+    __device__ __forceinline__ void drop() {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = 0.f;
+        m = -INFINITY;
+        l = 0.f;
+    }
+
+    __device__ __forceinline__ void publish(float* wm, float* wl, float* wacc, int warp, int lane) {
+        float lt = l;
+        lt += __shfl_xor_sync(FULL_MASK, lt, 1);
+        lt += __shfl_xor_sync(FULL_MASK, lt, 2);
+        const int g = lane >> 2, c2 = 2 * (lane & 3);
+        if (g < G) {
+            if ((lane & 3) == 0) {
+                wm[warp * G + g] = m;
+                wl[warp * G + g] = lt;
+            }
+            float* dst = wacc + (warp * G + g) * D + c2;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) *reinterpret_cast<float2*>(dst + 8 * n) =
+                make_float2(o[n][0], o[n][1]);
+        }
+    }
+};
+
+// Policy choice: tensor cores for bf16 whose blocks hold whole 16-token
+// units; fp32 FMAs otherwise (fp32 caches, 8-token blocks).
+template <typename T, int D, int BS, int G>
+using UnitFor = typename std::conditional<(std::is_same<T, __nv_bfloat16>::value &&
+                                           BS % 16 == 0),
+                                          MmaUnit<D, BS, G>, CoreUnit<T, D, BS, G>>::type;
+
+// ---------------------------------------------------- kernel geometry ----
+template <class U>
+struct Layout {
+    static constexpr int NW = 4;                                   // warps per CTA
+    static constexpr int UNIT_BYTES = U::R * U::D * (int)sizeof(typename U::T);
+    static constexpr int STAGE_BYTES = 2 * UNIT_BYTES;
+    static constexpr int DEPTH = cmin(8, cmax(2, 16384 / STAGE_BYTES));
+    static constexpr int STAGE_REGION = NW * DEPTH * STAGE_BYTES;
+    // warps merge in the drained ring: [NW][G] max, [NW][G] sum,
+    // [NW][G][D] output, then the cluster exchange [G], [G], [G][D]
+    static constexpr int MERGE_BYTES = (NW + 1) * U::G * (U::D + 2) * 4;
+    static constexpr int MAIN_REGION = cmax(STAGE_REGION, MERGE_BYTES);
+    static constexpr int PBUF_OFFSET = MAIN_REGION;
+    static constexpr int ORDER_OFFSET = PBUF_OFFSET + NW * U::PBUF_FLOATS * 4;
+    static constexpr int BAR_OFFSET = ORDER_OFFSET + (MAX_SORT + 4) * 4;
+    static constexpr int SMEM_BYTES = BAR_OFFSET + NW * DEPTH * 8 + 1024;   // + alignment slack
+    static_assert(MAIN_REGION % 1024 == 0 && STAGE_BYTES % 1024 == 0, "1 KiB aligned stages");
+    static_assert(BAR_OFFSET % 8 == 0, "mbarrier alignment");
+};
+
+// Per-CTA context shared by every item the CTA runs.
+template <class U>
+struct Ctx {
+    unsigned char* smem;
+    typename U::T* stages;     // this warp's ring
+    float* pbuf;               // this warp's probability buffer (CoreUnit)
+    uint64_t* bars;            // this warp's mbarriers
+    int warp, lane;
+    int ring;                  // units this warp has consumed so far
+};
+
+// Run one item: stream this CTA's share of (seq, kvh)'s units in
+// [u_begin, u_end), interleaved over `ctas` CTAs (this one is `crank`) and
+// over the NW warps, then merge the warps into shared memory.  Returns with
+// the CTA-merged (max, sum, unnormalised output) per (g, d) computed by
+// `epilogue`.  Every thread of the CTA must call it (it holds barriers).
+template <class U, class Epi>
+__device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
+                                         const CUtensorMap* tm_v, const DecodeArgs& a, int seq,
+                                         int kvh, int L, int u_begin, int u_end, int ctas,
+                                         int crank, Epi&& epilogue) {
+    using T = typename U::T;
+    using Ly = Layout<U>;
+    constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
+    const int warp = cx.warp, lane = cx.lane;
+    const int ustride = ctas * NW;
+    const int first = u_begin + crank + ctas * warp;
+    const int nk = first < u_end ? (u_end - first + ustride - 1) / ustride : 0;
+
+    U u;
+    u.begin(reinterpret_cast<const T*>(a.q) +
+                ((size_t)seq * a.num_heads + (size_t)kvh * G) * D,
+            a.scale_log2, lane);
+
+    const int32_t* table = a.block_tables + (size_t)seq * a.max_blocks;
+    int win = 0;
+    auto load_window = [&](int k0) {
+        const int k = k0 + lane;
+        int id = 0;
+        if (k < nk) {
+            const int uu = first + ustride * k;
+            id = __ldg(table + (uu * R) / U::BS);
+            if (id < 0 || id >= a.num_blocks) {
+                raise_error(a.err, PA_DEVERR_BLOCK_ID);
+                id = a.num_blocks;       // outside the tensor map: TMA fills zeros
+            }
+        }
+        win = id;
+    };
+    auto slot = [&](int k) { return (cx.ring + k) % DEPTH; };
+    auto issue = [&](int k, int id) {     // lane 0 only
+        const int s = slot(k);
+        T* kdst = cx.stages + (size_t)s * (2 * R * D);
+        const int uu = first + ustride * k;
+        const int row0 = (uu * R) % U::BS;
+        mbar_arrive_expect_tx(&cx.bars[s], Ly::STAGE_BYTES);
+#pragma unroll
+        for (int b = 0; b < U::BOXES; ++b) {
+            tma_load_4d(kdst + b * R * U::BOX_INNER, tm_k, &cx.bars[s], b * U::BOX_INNER, kvh,
+                        row0, id);
+            tma_load_4d(kdst + R * D + b * R * U::BOX_INNER, tm_v, &cx.bars[s],
+                        b * U::BOX_INNER, kvh, row0, id);
+        }
+    };
+
+    load_window(0);
+    const int pro = cmin(DEPTH, nk);
+    for (int k = 0; k < pro; ++k) {
+        const int id = __shfl_sync(FULL_MASK, win, k);
+        if (lane == 0) issue(k, id);
+    }
+    int k = 0;
+    bool failed = false;
+    for (; k < nk; ++k) {
+        const int s = slot(k);
+        const uint32_t parity = ((cx.ring + k) / DEPTH) & 1;
+        const bool landed = __all_sync(FULL_MASK, mbar_wait_bounded(&cx.bars[s], parity));
+        if (!landed) {
+            failed = true;
+            break;
+        }
+        T* ks = cx.stages + (size_t)s * (2 * R * D);
+        const int uu = first + ustride * k;
+        const int valid = cmin(R, L - uu * R);
+        if (valid == R)
+            u.template unit<false>(ks, ks + R * D, cx.pbuf, valid, lane);
+        else
+            u.template unit<true>(ks, ks + R * D, cx.pbuf, valid, lane);
+        const int kn = k + DEPTH;
+        if (kn < nk) {
+            if (kn % 32 == 0) load_window(kn);
+            const int id = __shfl_sync(FULL_MASK, win, kn % 32);
+            if (lane == 0) issue(kn, id);
+        }
+    }
+    if (failed) {
+        // A load never landed: record it, wait (bounded) for this warp's other
+        // loads in flight so none lands after the CTA moves on, contribute nothing.
+        if (lane == 0) raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+        const int issued = cmin(nk, k + DEPTH);
+        for (int kk = k + 1; kk < issued; ++kk)
+            (void)mbar_wait_bounded(&cx.bars[slot(kk)], ((cx.ring + kk) / DEPTH) & 1);
+        u.drop();
+        // keep the ring's phase bookkeeping consistent with what was issued
+        cx.ring += issued;
+    } else {
+        cx.ring += nk;
     }
 
     // ---- merge the warps (the merge area overlays the stage ring) ----
     __syncthreads();
-    float* wm = reinterpret_cast<float*>(smem);     // [NW][G]
-    float* wl = wm + NW * G;                         // [NW][G]
-    float* wacc = wl + NW * G;                       // [NW][G][D]
-    float* xch = wacc + NW * G * D;                  // [G] max, [G] sum, [G][D] acc
-    if (lane == 0)
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            wm[warp * G + g] = m[g];
-            wl[warp * G + g] = lsum[g];
-        }
-    if (r == 0)
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int v = 0; v < VPL; ++v)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    wacc[(warp * G + g) * D + (v * LPR + c) * VEC + e] = acc[g][v][e];
+    float* wm = reinterpret_cast<float*>(cx.smem);   // [NW][G]
+    float* wl = wm + NW * G;                           // [NW][G]
+    float* wacc = wl + NW * G;                         // [NW][G][D]
+    u.publish(wm, wl, wacc, warp, lane);
     __syncthreads();
-
-    T* out = reinterpret_cast<T*>(a.out);
-    const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
-    const bool cluster_merge = MODE == Mode::Decode && ctas > 1;
-    for (int idx = threadIdx.x; idx < G * D; idx += NT) {
+    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
         const int g = idx / D, d = idx % D;
         float big = -INFINITY;
 #pragma unroll
@@ -488,47 +617,208 @@ __global__ void __launch_bounds__(Geom<T, D, BS, G>::NW * 32)
             num = fmaf(e, wacc[(w * G + g) * D + d], num);
             den = fmaf(e, wl[w * G + g], den);
         }
-        if (cluster_merge) {
-            if (d == 0) {
-                xch[g] = big;
-                xch[G + g] = den;
-            }
-            xch[2 * G + g * D + d] = num;
-        } else if (MODE == Mode::Split && nparts > 1) {
-            const size_t slot = (head0 + g) * a.max_parts + part;
-            if (d == 0) {
-                a.ws_m[slot] = big;
-                a.ws_l[slot] = den;
-            }
-            a.ws_o[slot * D + d] = num;
-        } else {
-            store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+        epilogue(g, d, big, num, den, wacc + NW * G * D);
+    }
+    // the merge area overlays the stage ring, which TMA refills next
+    fence_proxy_async_smem();
+}
+
+template <class U, Mode MODE>
+__global__ void __launch_bounds__(Layout<U>::NW * 32)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
+    using T = typename U::T;
+    using Ly = Layout<U>;
+    constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
+    constexpr int NT = NW * 32;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+    // Split mode: a partition that does not exist leaves before anything else.
+    int seq = 0, kvh = 0, L = 0, part = 0, nparts = 1;
+    auto clamp_len = [&](int s) {
+        int x = a.context_lens[s];
+        if (x < 0 || x > a.max_tokens) {
+            if (threadIdx.x == 0) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
+            x = x < 0 ? 0 : a.max_tokens;
+        }
+        return x;
+    };
+    if constexpr (MODE == Mode::Split) {
+        seq = blockIdx.z;
+        kvh = blockIdx.y;
+        part = blockIdx.x;
+        L = clamp_len(seq);
+        nparts = (L + a.part_tokens - 1) / a.part_tokens;
+        if (part >= cmax(nparts, 1)) return;
+        if (nparts > a.max_parts) {
+            if (threadIdx.x == 0 && part == 0) raise_error(a.err, PA_DEVERR_WORKSPACE);
+            if (part > 0) return;
+            nparts = 1;                       // degrade: partition 0 covers everything
         }
     }
 
-    if constexpr (MODE == Mode::Decode) {
-        if (cluster_merge) {
-            cg::cluster_group cluster = cg::this_cluster();
-            cluster.sync();                              // every rank's xch is written
-            if (cluster.block_rank() == 0) {
-                for (int idx = threadIdx.x; idx < G * D; idx += NT) {
-                    const int g = idx / D, d = idx % D;
-                    float big = -INFINITY;
-                    for (int rk = 0; rk < ctas; ++rk)
-                        big = fmaxf(big, cluster.map_shared_rank(xch, rk)[g]);
-                    float num = 0.f, den = 0.f;
-                    for (int rk = 0; rk < ctas; ++rk) {
-                        const float* rx = cluster.map_shared_rank(xch, rk);
-                        const float mr = rx[g];
-                        const float e = mr == -INFINITY ? 0.f : exp2_approx(mr - big);
-                        num = fmaf(e, rx[2 * G + g * D + d], num);
-                        den = fmaf(e, rx[G + g], den);
-                    }
-                    store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
-                }
-            }
-            cluster.sync();                              // keep xch alive until rank 0 is done
+    Ctx<U> cx;
+    cx.smem = smem;
+    cx.stages = reinterpret_cast<T*>(smem) + (size_t)warp * DEPTH * (2 * R * D);
+    cx.pbuf = reinterpret_cast<float*>(smem + Ly::PBUF_OFFSET) + warp * U::PBUF_FLOATS;
+    cx.bars = reinterpret_cast<uint64_t*>(smem + Ly::BAR_OFFSET) + warp * DEPTH;
+    cx.warp = warp;
+    cx.lane = lane;
+    cx.ring = 0;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < DEPTH; ++s) mbar_init(&cx.bars[s], 1);
+        fence_mbar_init();
+        if (warp == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
         }
+    }
+    __syncwarp();
+
+    T* out = reinterpret_cast<T*>(a.out);
+
+    if constexpr (MODE == Mode::Split) {
+        const int pu = a.part_tokens / R;
+        const int total_units = (L + R - 1) / R;
+        const int u_begin = nparts == 1 && part == 0 ? 0 : part * pu;
+        const int u_end = nparts == 1 ? total_units : cmin(u_begin + pu, total_units);
+        const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
+        run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, u_begin, u_end, 1, 0,
+                    [&](int g, int d, float big, float num, float den, float*) {
+                        if (nparts > 1) {
+                            const size_t slot = (head0 + g) * a.max_parts + part;
+                            if (d == 0) {
+                                a.ws_m[slot] = big;
+                                a.ws_l[slot] = den;
+                            }
+                            a.ws_o[slot * D + d] = num;
+                        } else {
+                            store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                        }
+                    });
+        return;
+    } else {
+        if (a.sched == SCHED_CLUSTER) {
+            seq = blockIdx.z;
+            kvh = blockIdx.y;
+            L = clamp_len(seq);
+            const int ctas = gridDim.x;
+            const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
+            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, ctas, blockIdx.x,
+                        [&](int g, int d, float big, float num, float den, float* x) {
+                            // x: [G] max, [G] sum, [G][D] unnormalised output
+                            if (ctas > 1) {
+                                if (d == 0) {
+                                    x[g] = big;
+                                    x[G + g] = den;
+                                }
+                                x[2 * G + g * D + d] = num;
+                            } else {
+                                store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                            }
+                        });
+            if (ctas > 1) {
+                float* xch = reinterpret_cast<float*>(smem) + NW * G * (D + 2);
+                cg::cluster_group cluster = cg::this_cluster();
+                cluster.sync();                        // every rank's xch is written
+                if (cluster.block_rank() == 0) {
+                    for (int idx = threadIdx.x; idx < G * D; idx += NT) {
+                        const int g = idx / D, d = idx % D;
+                        float big = -INFINITY;
+                        for (int rk = 0; rk < ctas; ++rk)
+                            big = fmaxf(big, cluster.map_shared_rank(xch, rk)[g]);
+                        float num = 0.f, den = 0.f;
+                        for (int rk = 0; rk < ctas; ++rk) {
+                            const float* rx = cluster.map_shared_rank(xch, rk);
+                            const float mr = rx[g];
+                            const float e = mr == -INFINITY ? 0.f : exp2_approx(mr - big);
+                            num = fmaf(e, rx[2 * G + g * D + d], num);
+                            den = fmaf(e, rx[G + g], den);
+                        }
+                        store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                    }
+                }
+                cluster.sync();                        // keep xch alive until rank 0 is done
+            }
+            return;
+        }
+
+        if (a.sched == SCHED_LPT) {
+            // Which sequence sits at rank r = blockIdx.x / Hk of the list sorted
+            // by (length descending, index ascending)?  Warp 0 binary-searches
+            // the length value v at rank r (counts by warp reduction), then
+            // picks the k-th sequence of length v in index order by ballots.
+            const int S = a.num_seqs, Hk = a.num_kv_heads;
+            const int r = blockIdx.x / Hk;
+            int* pick = reinterpret_cast<int*>(smem + Ly::ORDER_OFFSET);
+            int* lens = pick + 1;                            // S lengths (S <= MAX_SORT)
+            if (S <= MAX_SORT)
+                for (int i = threadIdx.x; i < S; i += NT) {
+                    const int x = a.context_lens[i];
+                    if (x < 0 || x > a.max_tokens) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
+                    lens[i] = x < 0 ? 0 : (x > a.max_tokens ? a.max_tokens : x);
+                }
+            __syncthreads();
+            if (warp == 0) {
+                int found = r;                               // natural order beyond MAX_SORT
+                if (S <= MAX_SORT) {
+                    const int per_lane = (S + 31) / 32;
+                    int top = 0;
+                    for (int j = 0; j < per_lane; ++j) {
+                        const int i = lane + 32 * j;
+                        if (i < S) top = max(top, lens[i]);
+                    }
+                    top = (int)__reduce_max_sync(FULL_MASK, (unsigned)top);
+                    int lo = 0, hi = top + 1;        // count(len >= lo) > r >= count(len >= hi)
+                    while (hi - lo > 1) {
+                        const int mid = lo + (hi - lo) / 2;
+                        int cnt = 0;
+                        for (int j = 0; j < per_lane; ++j) {
+                            const int i = lane + 32 * j;
+                            cnt += i < S && lens[i] >= mid;
+                        }
+                        if ((int)__reduce_add_sync(FULL_MASK, (unsigned)cnt) > r)
+                            lo = mid;
+                        else
+                            hi = mid;
+                    }
+                    int gt = 0;
+                    for (int j = 0; j < per_lane; ++j) {
+                        const int i = lane + 32 * j;
+                        gt += i < S && lens[i] > lo;
+                    }
+                    const int k = r - (int)__reduce_add_sync(FULL_MASK, (unsigned)gt);
+                    int base = 0;
+                    found = -1;
+                    for (int j = 0; j < per_lane; ++j) {
+                        const int i = lane + 32 * j;
+                        const bool eq = i < S && lens[i] == lo;
+                        const unsigned ball = __ballot_sync(FULL_MASK, eq);
+                        const int before = __popc(ball & ((1u << lane) - 1u));
+                        if (eq && base + before == k) found = i;
+                        base += __popc(ball);
+                    }
+                    found = (int)__reduce_max_sync(FULL_MASK, (unsigned)(found + 1)) - 1;
+                }
+                if (lane == 0) *pick = found;
+            }
+            __syncthreads();
+            seq = *pick;
+            kvh = blockIdx.x % Hk;
+            L = S <= MAX_SORT ? lens[seq] : clamp_len(seq);
+            const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
+            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, 1, 0,
+                        [&](int g, int d, float big, float num, float den, float*) {
+                            store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                        });
+            return;
+        }
+
     }
 }
 

@@ -23,9 +23,11 @@ namespace pa {
 struct DecodeArgs;
 
 // Encode a 4-D tensor map over a [num_blocks][block_size][kv_heads][head_dim]
-// cache with a {head_dim, 1, rows, 1} box (no swizzle, no multicast).
+// cache with a {box_inner, 1, rows, 1} box, optionally with the 128-byte
+// shared-memory swizzle (box_inner * element size must then be 128 bytes).
 pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
-                           int num_kv_heads, int block_size, int num_blocks, int rows);
+                           int num_kv_heads, int block_size, int num_blocks, int box_inner,
+                           int rows, bool swizzle128);
 
 // Device error word of the current device (address from cudaGetSymbolAddress).
 unsigned* device_error_word();

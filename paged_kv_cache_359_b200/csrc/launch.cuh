@@ -40,28 +40,29 @@ inline pa_status allow_smem(K kernel, int bytes, std::atomic<unsigned long long>
 
 template <typename T, int D, int BS, int G>
 pa_status launch_decode_g(const DecodeLaunch& l) {
-    using Gm = Geom<T, D, BS, G>;
+    using U = UnitFor<T, D, BS, G>;
+    using Ly = Layout<U>;
     constexpr pa_dtype DT = std::is_same<T, float>::value ? PA_DTYPE_F32 : PA_DTYPE_BF16;
     CUtensorMap mk, mv;
     if (pa_status s = encode_cache_map(&mk, l.k_cache, DT, D, l.num_kv_heads, BS,
-                                       l.args.num_blocks, Gm::R))
+                                       l.args.num_blocks, U::BOX_INNER, U::R, U::SWIZZLE128))
         return s;
     if (pa_status s = encode_cache_map(&mv, l.v_cache, DT, D, l.num_kv_heads, BS,
-                                       l.args.num_blocks, Gm::R))
+                                       l.args.num_blocks, U::BOX_INNER, U::R, U::SWIZZLE128))
         return s;
-    if (l.split && l.args.part_tokens % Gm::R != 0)
-        return fail(PA_ERR_INVALID_ARG, "partition must be a multiple of %d tokens", Gm::R);
+    if (l.split && l.args.part_tokens % U::R != 0)
+        return fail(PA_ERR_INVALID_ARG, "partition must be a multiple of %d tokens", U::R);
 
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
-    cfg.blockDim = dim3(Gm::NW * 32);
-    cfg.dynamicSmemBytes = Gm::SMEM_BYTES;
+    cfg.blockDim = dim3(Ly::NW * 32);
+    cfg.dynamicSmemBytes = Ly::SMEM_BYTES;
     cfg.stream = l.stream;
     cudaError_t e;
     if (l.split) {
         static std::atomic<unsigned long long> done{0};
-        auto kern = paged_decode_kernel<T, D, BS, G, Mode::Split>;
-        if (pa_status s = allow_smem(kern, Gm::SMEM_BYTES, done)) return s;
+        auto kern = paged_decode_kernel<U, Mode::Split>;
+        if (pa_status s = allow_smem(kern, Ly::SMEM_BYTES, done)) return s;
         cfg.gridDim = dim3(l.args.max_parts, l.num_kv_heads, l.num_seqs);
         e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
         if (e == cudaSuccess) {
@@ -71,16 +72,20 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
         }
     } else {
         static std::atomic<unsigned long long> done{0};
-        auto kern = paged_decode_kernel<T, D, BS, G, Mode::Decode>;
-        if (pa_status s = allow_smem(kern, Gm::SMEM_BYTES, done)) return s;
-        cfg.gridDim = dim3(l.ctas, l.num_kv_heads, l.num_seqs);
-        if (l.ctas > 1) {
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = l.ctas;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
+        auto kern = paged_decode_kernel<U, Mode::Decode>;
+        if (pa_status s = allow_smem(kern, Ly::SMEM_BYTES, done)) return s;
+        if (l.args.sched == SCHED_LPT) {
+            cfg.gridDim = dim3((unsigned)((long long)l.num_seqs * l.num_kv_heads));
+        } else {
+            cfg.gridDim = dim3(l.ctas, l.num_kv_heads, l.num_seqs);
+            if (l.ctas > 1) {
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = l.ctas;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+            }
         }
         e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
     }

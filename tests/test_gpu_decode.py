@@ -156,3 +156,26 @@ def test_long_context_split():
         assert_close(got[s:s + 1], ref)
         assert_close(got1[s:s + 1], ref)
     device_clean()
+
+
+@pytest.mark.parametrize("hq,hk", [(8, 2), (4, 4)])
+def test_large_batch_beyond_the_sorted_range(hq, hk):
+    """1100 short sequences: more than the kernel sorts in shared memory,
+    so items run in natural order; still every output is checked."""
+    problem = pa_inputs.random_small(500 + hq, num_seqs=1100, max_len=40, num_heads=hq,
+                                     num_kv_heads=hk, head_dim=64, block_size=16, dtype="bf16",
+                                     zero_len=True)
+    data = pa_inputs.materialize(problem, "cuda")
+    assert_close(run_decode(data, problem), oracle_decode(data, problem))
+    device_clean()
+
+
+def test_longest_first_order_with_length_ties():
+    """The longest-first grid on a ragged GQA batch whose lengths repeat
+    (duplicated lengths exercise the index tie-break of the rank search)."""
+    problem = pa_inputs.random_small(808, num_seqs=96, max_len=700, num_heads=32,
+                                     num_kv_heads=8, head_dim=128, block_size=16, dtype="bf16",
+                                     fixed={i: 333 for i in range(0, 96, 7)})
+    data = pa_inputs.materialize(problem, "cuda")
+    assert_close(run_decode(data, problem), oracle_decode(data, problem))
+    device_clean()
