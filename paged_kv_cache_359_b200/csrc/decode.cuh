@@ -517,11 +517,6 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
     const int first = u_begin + crank + ctas * warp;
     const int nk = first < u_end ? (u_end - first + ustride - 1) / ustride : 0;
 
-    U u;
-    u.begin(reinterpret_cast<const T*>(a.q) +
-                ((size_t)seq * a.num_heads + (size_t)kvh * G) * D,
-            a.scale_log2, lane);
-
     const int32_t* table = a.block_tables + (size_t)seq * a.max_blocks;
     int win = 0;
     auto load_window = [&](int k0) {
@@ -559,6 +554,11 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
         const int id = __shfl_sync(FULL_MASK, win, k);
         if (lane == 0) issue(k, id);
     }
+    // the queries load while the first tiles are in flight
+    U u;
+    u.begin(reinterpret_cast<const T*>(a.q) +
+                ((size_t)seq * a.num_heads + (size_t)kvh * G) * D,
+            a.scale_log2, lane);
     int k = 0;
     bool failed = false;
     for (; k < nk; ++k) {
