@@ -22,7 +22,10 @@ Reported line (rank 0):
   e2e        the same metric through the public API with host buffers: the
              live allocator on the host, pinned H2D copies of each step's
              q / new K,V / slots / lengths / table, and a D2H read of the
-             step's output, all inside the timed region.
+             step's output, all inside the timed region; uploads and
+             downloads run on their own streams, double-buffered,
+             overlapping the neighbouring steps' kernels as a serving loop
+             would.
   roofline   the decode kernel: algorithmic bytes per launch / mean launch
              time (CUDA events on the launching stream) vs measured HBM GB/s.
   cpu_baseline  the fp64 oracle on the host's cores, bounded sample.
@@ -127,18 +130,23 @@ class ClockSampler:
             self._nv = None
             self.error = f"nvml unavailable: {e}"
 
-    def _run(self):
+    def sample(self):
+        """One reading of the SM clock and the active clock-event reasons."""
+        if self._nv is None:
+            return
         nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for b, name in REASON_BITS.items():
-                    if bits & b:
-                        self.reasons.add(name)
-            except Exception as e:
-                self.error = str(e)
-                return
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for b, name in REASON_BITS.items():
+                if bits & b:
+                    self.reasons.add(name)
+        except Exception as e:
+            self.error = str(e)
+
+    def _run(self):
+        while not self._stop.is_set() and self.error is None:
+            self.sample()
             time.sleep(self.period)
 
     def __enter__(self):
@@ -331,6 +339,7 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
         for j in range(steps):
             step(warmup + j, j)
         t1.record(stream)
+        clocks.sample()                # the host is ahead: the GPU is still in the region
         torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -349,74 +358,151 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
             "cow_pairs": int(sum(len(c) for c in cows[warmup:]))}
 
 
+def _segments(spec):
+    """Byte offsets of 256-byte-aligned segments: spec = [(name, nbytes), ...]."""
+    off, out = 0, {}
+    for name, nbytes in spec:
+        out[name] = (off, nbytes)
+        off += (nbytes + 255) // 256 * 256
+    return out, off
+
+
+def _view(buf, seg, dtype, shape):
+    off, nbytes = seg
+    return buf[off:off + nbytes].view(dtype).view(shape)
+
+
 def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int):
-    """Through the public API from host buffers: live allocator, pinned H2D of
-    every step's inputs, D2H of every step's output, all timed."""
+    """Through the public API from host buffers, as a serving loop runs it.
+
+    Every step: the host allocator appends a token to every sequence, writing
+    the block table, lengths, slots and copy-on-write pairs straight into a
+    pinned metadata buffer; the step's inputs go host->device from pinned
+    memory (one copy for q and the new K/V rows, one for the metadata); the
+    kernels run; the step's output comes back device->host and is read on the
+    host.  Copies run on a second stream with double-buffered device inputs,
+    so step i+1's upload and step i-1's download overlap step i's kernels; the
+    timed region spans every copy of every timed step."""
     pa, p, dev = loop.pa, loop.p, loop.device
     total = steps + warmup
-    pin = lambda t: t.pin_memory()
+    s, cap = loop.tables.shape
+    dt = loop.q0.dtype
+    esz = loop.q0.element_size()
+    qshape = (s, p.num_heads, p.head_dim)
+    kshape = (s, p.num_kv_heads, p.head_dim)
+    in_seg, in_bytes = _segments([("q", s * p.num_heads * p.head_dim * esz),
+                                  ("k", s * p.num_kv_heads * p.head_dim * esz),
+                                  ("v", s * p.num_kv_heads * p.head_dim * esz)])
+    meta_seg, meta_bytes = _segments([("tables", s * cap * 4), ("lens", s * 4), ("slots", s * 8),
+                                      ("cows", s * 2 * 8)])
     host = []
     for st in range(total):
         t = pa_inputs.step_tokens(p.num_seqs, p.num_heads, p.num_kv_heads, p.head_dim, p.dtype,
                                   p.seed + 1, st, "cpu")
-        host.append((pin(t["q"]), pin(t["key"]), pin(t["value"])))
-    s, cap = loop.tables.shape
-    tables_h = torch.from_numpy(loop.tables).pin_memory()
-    lens_h = torch.from_numpy(loop.lens).pin_memory()
-    tables_np, lens_np = tables_h.numpy(), lens_h.numpy()
-    slots_h = torch.zeros(s, dtype=torch.int64).pin_memory()
-    cows_h = torch.zeros((s, 2), dtype=torch.int64).pin_memory()
-    out_h = torch.empty(tuple(loop.out.shape), dtype=loop.out.dtype).pin_memory()
-    q_d = torch.empty_like(loop.q0)
-    k_d = torch.empty((s, p.num_kv_heads, p.head_dim), dtype=loop.q0.dtype, device=dev)
-    v_d = torch.empty_like(k_d)
-    tables_d = torch.empty((s, cap), dtype=torch.int32, device=dev)
-    lens_d = torch.empty(s, dtype=torch.int32, device=dev)
-    slots_d = torch.empty(s, dtype=torch.int64, device=dev)
-    cows_d = torch.empty((s, 2), dtype=torch.int64, device=dev)
-    stream = torch.cuda.current_stream()
-    h2d = d2h = 0
-    kv = 0
+        hb = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+        _view(hb, in_seg["q"], dt, qshape).copy_(t["q"])
+        _view(hb, in_seg["k"], dt, kshape).copy_(t["key"])
+        _view(hb, in_seg["v"], dt, kshape).copy_(t["value"])
+        host.append(hb)
+    meta_h = torch.zeros(meta_bytes, dtype=torch.uint8).pin_memory()
+    tables_np = _view(meta_h, meta_seg["tables"], torch.int32, (s, cap)).numpy()
+    lens_np = _view(meta_h, meta_seg["lens"], torch.int32, (s,)).numpy()
+    slots_np = _view(meta_h, meta_seg["slots"], torch.int64, (s,)).numpy()
+    cows_np = _view(meta_h, meta_seg["cows"], torch.int64, (s, 2)).numpy()
+    tables_np[:] = loop.tables             # the allocator continues from here, in place
+    lens_np[:] = loop.lens
+    comp = torch.cuda.current_stream()
+    up = torch.cuda.Stream(device=dev)      # host -> device
+    down = torch.cuda.Stream(device=dev)    # device -> host, so uploads never queue behind it
+    meta_up = torch.cuda.Event()
 
-    def step(i):
-        nonlocal h2d, d2h, kv
+    class Buf:
+        def __init__(self):
+            self.inp = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+            self.meta = torch.empty(meta_bytes, dtype=torch.uint8, device=dev)
+            self.q = _view(self.inp, in_seg["q"], dt, qshape)
+            self.k = _view(self.inp, in_seg["k"], dt, kshape)
+            self.v = _view(self.inp, in_seg["v"], dt, kshape)
+            self.tables = _view(self.meta, meta_seg["tables"], torch.int32, (s, cap))
+            self.lens = _view(self.meta, meta_seg["lens"], torch.int32, (s,))
+            self.slots = _view(self.meta, meta_seg["slots"], torch.int64, (s,))
+            self.cows = _view(self.meta, meta_seg["cows"], torch.int64, (s, 2))
+            self.out = torch.empty_like(loop.out)
+            self.out_h = torch.empty(tuple(loop.out.shape), dtype=loop.out.dtype).pin_memory()
+            self.h2d, self.done, self.d2h = (torch.cuda.Event(), torch.cuda.Event(),
+                                             torch.cuda.Event())
+            self.used = False
+
+    bufs = [Buf(), Buf()]
+    counts = {"h2d": 0, "d2h": 0, "kv": 0}
+    pending = []
+
+    def read_back(upto_all=False):
+        while pending and (upto_all or len(pending) > 1):
+            b = pending.pop(0)
+            b.d2h.synchronize()
+            float(b.out_h.view(-1)[0])                 # the host reads the result
+
+    def step(i, count):
+        b = bufs[i % 2]
+        meta_up.synchronize()                          # last step's metadata upload is done
         sl, cw = loop.alloc.append_slots(tables_np, lens_np)
-        slots_h.numpy()[:] = sl
+        slots_np[:] = sl
         n = len(cw)
         if n:
-            cows_h.numpy()[:n] = cw
-        q_h, k_h, v_h = host[i]
-        q_d.copy_(q_h, non_blocking=True)
-        k_d.copy_(k_h, non_blocking=True)
-        v_d.copy_(v_h, non_blocking=True)
-        slots_d.copy_(slots_h, non_blocking=True)
-        lens_d.copy_(lens_h, non_blocking=True)
-        tables_d.copy_(tables_h, non_blocking=True)
-        nb = (q_h.numel() * q_h.element_size() + 2 * k_h.numel() * k_h.element_size() +
-              8 * s + 4 * s + 4 * s * cap)
+            cows_np[:n] = cw
+        with torch.cuda.stream(up):
+            if b.used:
+                up.wait_event(b.done)                  # step i-2 is done with buffer b
+            b.inp.copy_(host[i], non_blocking=True)
+            b.meta.copy_(meta_h, non_blocking=True)
+            meta_up.record(up)
+            b.h2d.record(up)
+        comp.wait_event(b.h2d)
         if n:
-            cows_d[:n].copy_(cows_h[:n], non_blocking=True)
-            nb += 16 * n
-            pa.pa_copy_blocks(loop.k_cache, loop.v_cache, cows_d[:n])
-        pa.pa_reshape_and_cache(k_d, v_d, loop.k_cache, loop.v_cache, slots_d)
-        loop.decode(q_d, tables_d, lens_d, int(lens_np.max()))
-        out_h.copy_(loop.out, non_blocking=True)
-        stream.synchronize()
-        return nb, out_h.numel() * out_h.element_size(), decode_kv_bytes(lens_np, p)
+            pa.pa_copy_blocks(loop.k_cache, loop.v_cache, b.cows[:n], stream=comp)
+        pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
+        if loop.kernel == "split":
+            mx = int(lens_np.max())
+            pa.pa_decode_split(b.out, b.q, loop.k_cache, loop.v_cache, b.tables, b.lens,
+                               p.scale, mx, loop.partition, loop.workspace(mx), stream=comp)
+        else:
+            pa.pa_decode(b.out, b.q, loop.k_cache, loop.v_cache, b.tables, b.lens, p.scale,
+                         stream=comp)
+        b.done.record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(b.done)
+            b.out_h.copy_(b.out, non_blocking=True)
+            b.d2h.record(down)
+        b.used = True
+        pending.append(b)
+        read_back()
+        if count:
+            counts["h2d"] += in_bytes + meta_bytes
+            counts["d2h"] += b.out_h.numel() * b.out_h.element_size()
+            counts["kv"] += decode_kv_bytes(lens_np, p)
 
     for i in range(warmup):
-        step(i)
+        step(i, False)
+    read_back(True)
     torch.cuda.synchronize()
     barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
+    t0.record(comp)
+    up.wait_event(t0)
+    down.wait_event(t0)
     for j in range(steps):
-        a, b, c = step(warmup + j)
-        h2d += a; d2h += b; kv += c
-    t1.record(stream)
+        step(warmup + j, True)
+    for b in pending:
+        comp.wait_event(b.d2h)
+    t1.record(comp)
+    read_back(True)
     torch.cuda.synchronize()
     barrier(world)
-    return {"ms": t0.elapsed_time(t1), "kv_bytes": kv, "h2d": h2d / steps, "d2h": d2h / steps}
+    loop.tables[:] = tables_np
+    loop.lens[:] = lens_np
+    return {"ms": t0.elapsed_time(t1), "kv_bytes": counts["kv"], "h2d": counts["h2d"] / steps,
+            "d2h": counts["d2h"] / steps}
 
 
 # --------------------------------------------------------------------------
