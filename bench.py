@@ -194,6 +194,63 @@ def make_problem(name: str, extra_tokens: int, rank: int):
     raise ValueError(f"unknown workload {name}")
 
 
+def build_prefix_loop(device, extra_tokens: int, kernel: str, partition: int):
+    """64 sequences forked from one 2040-token prefix (block 16, head_dim 128,
+    32 q / 8 kv heads, bf16), tails U[0, 512]: the parent's prefix is
+    written, the children fork it, every sequence appends its tail through
+    the allocator (the shared half-full last block is copied on first write),
+    then one pa_copy_blocks and one pa_reshape_and_cache fill the cache."""
+    import paged_kv_cache_359_b200 as pa
+    pp = pa_inputs.prefix(16, 128, extra_tokens=extra_tokens)
+    bs, hk, d, s = pp.block_size, pp.num_kv_heads, pp.head_dim, pp.num_seqs
+    cap = pp.max_blocks_per_seq
+    alloc = pa.BlockAllocator(pp.num_blocks, bs, pp.free_order)
+    tables = np.full((s, cap), -1, dtype=np.int32)
+    lens = np.zeros(s, dtype=np.int32)
+    pre_slots, _, lens[0] = alloc.extend(tables[0], 0, pp.prefix_len)
+    n = -(-pp.prefix_len // bs)
+    for i in range(1, s):
+        alloc.fork(tables[0], n, tables[i])
+        lens[i] = lens[0]
+    slots, cows = [], []
+    for i in range(s):
+        sl, cow, lens[i] = alloc.extend(tables[i], int(lens[i]), int(pp.tail_lens[i]))
+        slots.append(sl)
+        if cow is not None:
+            cows.append(cow)
+    dt = pa_inputs.torch_dtype(pp.dtype)
+    gen = pa_inputs.generator(device, pp.seed)
+    kc = pa_inputs.poisoned_pool(pp.num_blocks, bs, hk, d, dt, gen, device,
+                                 np.zeros((pp.num_blocks, bs), bool))
+    vc = pa_inputs.poisoned_pool(pp.num_blocks, bs, hk, d, dt, gen, device,
+                                 np.zeros((pp.num_blocks, bs), bool))
+    pk, pv = pa_inputs.token_rows(pp.prefix_len, hk, d, pp.dtype, pp.seed + 2, device)
+    pa.pa_reshape_and_cache(pk, pv, kc, vc, torch.from_numpy(pre_slots).to(device))
+    if cows:
+        pa.pa_copy_blocks(kc, vc, torch.tensor(cows, dtype=torch.int64, device=device))
+    all_slots = np.concatenate(slots) if slots else np.zeros(0, np.int64)
+    tk, tv = pa_inputs.token_rows(len(all_slots), hk, d, pp.dtype, pp.seed + 3, device)
+    pa.pa_reshape_and_cache(tk, tv, kc, vc, torch.from_numpy(all_slots).to(device))
+    q0 = pa_inputs.randn((s, pp.num_heads, d), dt, gen, device)
+    torch.cuda.synchronize()
+    problem = pa_inputs.PagedProblem(
+        name="prefix", num_heads=pp.num_heads, num_kv_heads=hk, head_dim=d, block_size=bs,
+        num_blocks=pp.num_blocks, dtype=pp.dtype, context_lens=lens.copy(),
+        free_order=pp.free_order, block_tables=tables.copy(), seed=pp.seed, scale=pp.scale)
+    loop = DecodeLoop(problem, device, kernel, partition,
+                      state=(kc, vc, q0, alloc, tables, lens))
+    return loop
+
+
+def unique_kv_bytes(tables: np.ndarray, lens: np.ndarray, problem) -> int:
+    """K/V bytes of the distinct physical blocks the batch reads."""
+    bs = problem.block_size
+    blocks = set()
+    for i, n in enumerate(lens):
+        blocks.update(tables[i, :-(-int(n) // bs)].tolist())
+    return len(blocks) * bs * problem.num_kv_heads * problem.head_dim * 2 * problem.elem_bytes
+
+
 def decode_kv_bytes(lens: np.ndarray, problem) -> int:
     return int(lens.astype(np.int64).sum()) * problem.num_kv_heads * problem.head_dim * 2 * \
         problem.elem_bytes
@@ -248,13 +305,20 @@ def hbm_peak():
 class DecodeLoop:
     """State of one replica's decode loop: cache pool, host allocator, tables."""
 
-    def __init__(self, problem, device, kernel: str, partition: int):
+    def __init__(self, problem, device, kernel: str, partition: int, state=None):
         import paged_kv_cache_359_b200 as pa
         self.pa = pa
         self.p = problem
         self.device = device
         self.kernel = kernel
         self.partition = partition
+        self.ws = None
+        if state is not None:            # a prebuilt batch (the prefix workload)
+            (self.k_cache, self.v_cache, self.q0, self.alloc, self.tables,
+             self.lens) = state
+            self.out = torch.empty_like(self.q0)
+            self.max_len_cap = self.tables.shape[1] * problem.block_size
+            return
         data = pa_inputs.materialize(problem, device)
         self.k_cache, self.v_cache = data["k_cache"], data["v_cache"]
         self.q0 = data["q"]
@@ -292,7 +356,8 @@ class DecodeLoop:
                               self.p.scale)
 
 
-def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_index: int):
+def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_index: int,
+                     unique: bool = False):
     """Allocator outputs for every step are computed up front and uploaded;
     the timed region holds only device work on inputs resident in HBM."""
     pa, p, dev = loop.pa, loop.p, loop.device
@@ -352,7 +417,9 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     kv = sum(decode_kv_bytes(x, p) for x in timed_lens)
     alg = [decode_alg_bytes(x, p) for x in timed_lens]
     launches = sum(loop.launches_per_step(len(c)) for c in cows[warmup:])
-    return {"ms": ms, "kv_bytes": kv, "dec_ms": dec_ms, "dec_alg_bytes": alg,
+    uniq = (sum(unique_kv_bytes(t, l, p) for t, l in zip(tabs[warmup:], timed_lens))
+            if unique else None)
+    return {"ms": ms, "kv_bytes": kv, "dec_ms": dec_ms, "dec_alg_bytes": alg, "unique": uniq,
             "launches": launches, "clocks": clocks.summary(),
             "tokens": steps * p.num_seqs,
             "cow_pairs": int(sum(len(c) for c in cows[warmup:]))}
@@ -599,7 +666,8 @@ def run_reference(args, rank, world):
 def workload_config(p, args):
     lens = p.context_lens
     return {"workload": {"gqa": "gqa_decode_b256", "mha": "mha_decode_b64",
-                         "long": "long_context_split"}[args.workload],
+                         "long": "long_context_split",
+                         "prefix": "prefix_sharing_b64"}[args.workload],
             "num_seqs": p.num_seqs, "num_heads": p.num_heads, "num_kv_heads": p.num_kv_heads,
             "head_dim": p.head_dim, "block_size": p.block_size, "num_blocks": p.num_blocks,
             "context_len_median": int(np.median(lens)), "context_len_max": int(lens.max()),
@@ -617,7 +685,7 @@ def main():
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["gqa", "mha", "long"], default="gqa")
+    ap.add_argument("--workload", choices=["gqa", "mha", "long", "prefix"], default="gqa")
     ap.add_argument("--kernel", choices=["decode", "split"], default=None)
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--no-e2e", action="store_true")
@@ -634,6 +702,8 @@ def main():
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE {world}")
 
     if args.impl == "reference":
+        if args.workload == "prefix":
+            ap.error("the reference arm times the gqa, mha and long workloads")
         dist_init(world, "gloo")
         try:
             run_reference(args, rank, world)
@@ -649,9 +719,14 @@ def main():
     dist_init(world, "nccl")
     try:
         extra = 2 * (args.steps + args.warmup) + 4
-        p = make_problem(args.workload, extra, rank)
-        loop = DecodeLoop(p, dev, args.kernel, args.partition)
-        res = run_device_timed(loop, args.steps, args.warmup, world, local)
+        if args.workload == "prefix":
+            loop = build_prefix_loop(dev, extra, args.kernel, args.partition)
+            p = loop.p
+        else:
+            p = make_problem(args.workload, extra, rank)
+            loop = DecodeLoop(p, dev, args.kernel, args.partition)
+        res = run_device_timed(loop, args.steps, args.warmup, world, local,
+                               unique=args.workload == "prefix")
         e2e = None if args.no_e2e else run_e2e(loop, args.steps, args.warmup, world)
 
         ms = reduce_scalar(res["ms"], "max", world, dev)
@@ -687,6 +762,11 @@ def main():
             "clocks": res["clocks"],
             "cow_pairs_timed": res["cow_pairs"],
         }
+        if res["unique"] is not None:
+            # the shared prefix is read by every sharer: `value` counts each
+            # read (logical bytes), unique bytes count each physical block once
+            line["unique_kv_gbs"] = round(res["unique"] / secs / 1e9, 2)
+            line["unique_kv_bytes_per_step"] = int(res["unique"] / args.steps)
         if e2e is not None:
             e2e_ms = reduce_scalar(e2e["ms"], "max", world, dev)
             e2e_kv = reduce_scalar(e2e["kv_bytes"], "sum", world, dev)

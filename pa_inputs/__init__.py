@@ -183,13 +183,17 @@ class PrefixProblem:
 
 
 def prefix(block_size: int = 16, head_dim: int = 128, aligned: bool = False,
-           num_seqs: int = 64, shared: int = 2048, max_tail: int = 512) -> PrefixProblem:
+           num_seqs: int = 64, shared: int = 2048, max_tail: int = 512,
+           extra_tokens: int = 0) -> PrefixProblem:
+    """``extra_tokens`` reserves pool and table room for that many appended
+    tokens per sequence (a decode loop over the forked batch)."""
     seed = SEED_BASE + 4 + 100 * block_size + head_dim + (7 if aligned else 0)
     rng = np.random.default_rng(seed)
     plen = shared if aligned else shared - block_size // 2
     tails = rng.integers(0, max_tail + 1, size=num_seqs).astype(np.int32)
-    per_seq = blocks_for(plen + max_tail, block_size) + 1
-    nb = blocks_for(plen, block_size) + num_seqs * (blocks_for(max_tail, block_size) + 2)
+    per_seq = blocks_for(plen + max_tail + extra_tokens, block_size) + 1
+    nb = blocks_for(plen, block_size) + num_seqs * (blocks_for(max_tail + extra_tokens,
+                                                                block_size) + 2)
     order = shuffled_pool(rng, nb)
     return PrefixProblem(block_size=block_size, head_dim=head_dim, num_heads=32,
                          num_kv_heads=8, num_seqs=num_seqs, prefix_len=plen,
