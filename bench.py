@@ -313,6 +313,7 @@ class DecodeLoop:
         self.kernel = kernel
         self.partition = partition
         self.ws = None
+        self.fused = False
         if state is not None:            # a prebuilt batch (the prefix workload)
             (self.k_cache, self.v_cache, self.q0, self.alloc, self.tables,
              self.lens) = state
@@ -345,6 +346,8 @@ class DecodeLoop:
         return self.ws
 
     def launches_per_step(self, n_cow: int) -> int:
+        if self.fused:
+            return (1 if n_cow else 0) + 1
         return (1 if n_cow else 0) + 1 + (2 if self.kernel == "split" else 1)
 
     def decode(self, q, tables_d, lens_d, max_len):
@@ -386,10 +389,15 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     def step(i, timed_index=None):
         if cows_d[i] is not None:
             pa.pa_copy_blocks(loop.k_cache, loop.v_cache, cows_d[i])
-        pa.pa_reshape_and_cache(keys[i], vals[i], loop.k_cache, loop.v_cache, slots_d[i])
+        if not loop.fused:
+            pa.pa_reshape_and_cache(keys[i], vals[i], loop.k_cache, loop.v_cache, slots_d[i])
         if timed_index is not None:
             dec_ev[timed_index][0].record(stream)
-        loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
+        if loop.fused:
+            pa.pa_decode_append(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
+                                slots_d[i], tabs_d[i], lens_d[i], p.scale)
+        else:
+            loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
         if timed_index is not None:
             dec_ev[timed_index][1].record(stream)
 
@@ -528,12 +536,16 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int):
         comp.wait_event(b.h2d)
         if n:
             pa.pa_copy_blocks(loop.k_cache, loop.v_cache, b.cows[:n], stream=comp)
-        pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
-        if loop.kernel == "split":
+        if loop.fused:
+            pa.pa_decode_append(b.out, b.q, b.k, b.v, loop.k_cache, loop.v_cache, b.slots,
+                                b.tables, b.lens, p.scale, stream=comp)
+        elif loop.kernel == "split":
+            pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
             mx = int(lens_np.max())
             pa.pa_decode_split(b.out, b.q, loop.k_cache, loop.v_cache, b.tables, b.lens,
                                p.scale, mx, loop.partition, loop.workspace(mx), stream=comp)
         else:
+            pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
             pa.pa_decode(b.out, b.q, loop.k_cache, loop.v_cache, b.tables, b.lens, p.scale,
                          stream=comp)
         b.done.record(comp)
@@ -672,7 +684,8 @@ def workload_config(p, args):
             "head_dim": p.head_dim, "block_size": p.block_size, "num_blocks": p.num_blocks,
             "context_len_median": int(np.median(lens)), "context_len_max": int(lens.max()),
             "context_tokens": int(lens.astype(np.int64).sum()),
-            "kernel": args.kernel, "partition": args.partition,
+            "kernel": args.kernel + ("+append (fused)" if args.fused else ""),
+            "partition": args.partition,
             "l2": "inputs larger than L2 (KV cache %.2f GB vs 126 MB L2), no flush" %
                   (decode_kv_bytes(lens, p) / 1e9)}
 
@@ -688,6 +701,8 @@ def main():
     ap.add_argument("--workload", choices=["gqa", "mha", "long", "prefix"], default="gqa")
     ap.add_argument("--kernel", choices=["decode", "split"], default=None)
     ap.add_argument("--partition", type=int, default=512)
+    ap.add_argument("--fused", action="store_true",
+                    help="pa_decode_append: the cache write fused into the decode launch")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-sample", type=int, default=64,
@@ -697,6 +712,8 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.kernel is None:
         args.kernel = "split" if args.workload == "long" else "decode"
+    if args.fused and args.kernel != "decode":
+        ap.error("--fused fuses the cache write into pa_decode (not the split kernel)")
     rank, world, local = dist_env()
     if world != args.gpus and world > 1:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE {world}")
@@ -725,6 +742,7 @@ def main():
         else:
             p = make_problem(args.workload, extra, rank)
             loop = DecodeLoop(p, dev, args.kernel, args.partition)
+        loop.fused = args.fused
         res = run_device_timed(loop, args.steps, args.warmup, world, local,
                                unique=args.workload == "prefix")
         e2e = None if args.no_e2e else run_e2e(loop, args.steps, args.warmup, world)
@@ -750,8 +768,9 @@ def main():
             "data": "synthetic", "config": workload_config(p, args),
             "tokens_per_s": round(tokens_all / secs, 1),
             "frac_of_nominal_8tbps": round(value / NOMINAL_HBM_GBS, 4),
-            "roofline": {"bound": "hbm", "kernel": "pa_decode" if args.kernel == "decode"
-                         else "pa_decode_split (partition + reduce)",
+            "roofline": {"bound": "hbm",
+                         "kernel": ("pa_decode_append" if args.fused else "pa_decode")
+                         if args.kernel == "decode" else "pa_decode_split (partition + reduce)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "frac_of_nominal_8tbps": round(achieved / NOMINAL_HBM_GBS, 4),

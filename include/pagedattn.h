@@ -133,6 +133,28 @@ pa_status pa_decode(void* out_d, const void* q_d,
                     float scale, pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * pa_decode_append -- pa_reshape_and_cache of one new token per sequence
+ * followed by pa_decode, in one launch (the decode loop's step: the new
+ * token is stored, then attended to along with the rest of its sequence;
+ * [course] 2.4.2 and 2.5, [csdn-QA] 四 flow: update the mapping, then run
+ * the attention kernel).
+ *   key_d, value_d   [num_seqs, num_kv_heads, head_dim]: sequence s's new row
+ *   slot_mapping_d   int64 [num_seqs]: its slot (-1: sequence s gains no token)
+ *   k_cache_d, v_cache_d  written at those slots, then read
+ * Other arguments as pa_decode; context_lens already count the new token.
+ * Preconditions: each new slot is its sequence's last position (the slot of
+ * token context_lens[s]-1) and lies in a block no other sequence reads --
+ * the allocator's copy-on-write guarantees both.  Validate mode checks the
+ * first.  Out-of-pool slots are skipped and set PA_DEVERR_SLOT.
+ */
+pa_status pa_decode_append(void* out_d, const void* q_d, const void* key_d,
+                           const void* value_d, void* k_cache_d, void* v_cache_d,
+                           const int64_t* slot_mapping_d, const int32_t* block_tables_d,
+                           int max_blocks_per_seq, const int32_t* context_lens_d, int num_seqs,
+                           int num_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float scale, pa_dtype dtype, pa_stream_t stream);
+
+/*
  * pa_decode_split -- long-context decode in fixed token partitions merged by
  * log-sum-exp ("PagedAttention V2 ... block-wise computation",
  * [csdn-QA] 四, last paragraph; sequences up to 1M tokens, [tech] 1).

@@ -10,6 +10,7 @@ Functions carry the C names:
 
 * ``pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping)``
 * ``pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale)``
+* ``pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, ...)``
 * ``pa_decode_split(out, q, ..., max_context_len, partition_size, workspace)``
 * ``pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size)``
 * ``pa_copy_blocks(k_cache, v_cache, block_mapping)``
@@ -29,7 +30,7 @@ from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SP
                       PA_OPT_VALIDATE, PagedAttnError, check, lib)
 
 __all__ = [
-    "pa_reshape_and_cache", "pa_decode", "pa_decode_split", "pa_decode_split_workspace_bytes",
+    "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_split", "pa_decode_split_workspace_bytes",
     "pa_decode_split_noalloc", "pa_copy_blocks", "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
     "PagedAttnError", "OutOfBlocks", "DEVERR_BITS",
 ]
@@ -87,6 +88,22 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, strea
     check(lib().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                           block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb,
                           float(scale), _dtype(q), _stream(stream)))
+    return out
+
+
+def pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, block_tables,
+                     context_lens, scale, stream=None):
+    """pa_reshape_and_cache of one new row per sequence (key/value [S, Hk, D],
+    slot_mapping int64 [S], -1 = none) then pa_decode, in one launch."""
+    _dev(out, q, key, value, k_cache, v_cache, slot_mapping, block_tables, context_lens)
+    s, hq, d = q.shape
+    nb, bs, hk, _ = k_cache.shape
+    if slot_mapping.dtype != torch.int64:
+        raise ValueError("slot_mapping must be int64")
+    check(lib().pa_decode_append(_ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_cache),
+                                 _ptr(v_cache), _ptr(slot_mapping), _ptr(block_tables),
+                                 block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb,
+                                 float(scale), _dtype(q), _stream(stream)))
     return out
 
 

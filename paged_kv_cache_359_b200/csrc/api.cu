@@ -269,22 +269,52 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache
                                     row_bytes, num_slots, st);
 }
 
-pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                    const int32_t* block_tables, int max_blocks_per_seq,
-                    const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
-                    int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
-                    pa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// pa_decode, optionally with the fused append of one new token per sequence.
+pa_status decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                      int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+                      const void* new_k, const void* new_v, const int64_t* new_slots,
+                      pa_stream_t stream) {
     if (pa_status s = check_decode_args(out, q, k_cache, v_cache, block_tables,
                                         max_blocks_per_seq, context_lens, num_seqs, num_heads,
                                         num_kv_heads, head_dim, block_size, num_blocks, dtype,
                                         scale))
         return s;
     if (num_seqs == 0) return PA_OK;
+    const bool append = new_slots != nullptr;
+    if (append && (!new_k || !new_v || !aligned16(new_k) || !aligned16(new_v)))
+        return fail(PA_ERR_INVALID_ARG, "key and value rows must be 16-byte aligned device pointers");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (validate_enabled())
+    if (validate_enabled()) {
         if (pa_status s = validate_decode(block_tables, max_blocks_per_seq, context_lens,
                                           num_seqs, block_size, num_blocks, st))
             return s;
+        if (append) {
+            std::vector<int32_t> t, l;
+            std::vector<int64_t> sl;
+            if (!copy_to_host(l, context_lens, (size_t)num_seqs, st) ||
+                !copy_to_host(t, block_tables, (size_t)num_seqs * max_blocks_per_seq, st) ||
+                !copy_to_host(sl, new_slots, (size_t)num_seqs, st))
+                return fail(PA_ERR_CUDA, "validation copy failed");
+            for (int s = 0; s < num_seqs; ++s) {
+                if (sl[s] < 0) continue;
+                const int pos = l[s] - 1;
+                const int64_t want =
+                    pos < 0 ? -2
+                            : (int64_t)t[(size_t)s * max_blocks_per_seq + pos / block_size] *
+                                      block_size + pos % block_size;
+                if (sl[s] != want)
+                    return fail(PA_ERR_BAD_BLOCK_ID,
+                                "new slot of sequence %d is %lld, its last position is slot %lld",
+                                s, (long long)sl[s], (long long)want);
+            }
+        }
+    }
     DecodeLaunch l = {};
     l.args.out = out;
     l.args.q = q;
@@ -299,6 +329,11 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     l.args.num_heads = num_heads;
     l.args.num_kv_heads = num_kv_heads;
     l.args.num_blocks = num_blocks;
+    l.args.new_k = new_k;
+    l.args.new_v = new_v;
+    l.args.new_slots = new_slots;
+    l.args.k_cache = const_cast<void*>(k_cache);
+    l.args.v_cache = const_cast<void*>(v_cache);
     l.k_cache = k_cache;
     l.v_cache = v_cache;
     l.num_seqs = num_seqs;
@@ -314,6 +349,32 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     l.split = false;
     l.stream = st;
     return dispatch_decode(l, dtype, head_dim);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, int max_blocks_per_seq,
+                    const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
+                    int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+                    pa_stream_t stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       scale, dtype, nullptr, nullptr, nullptr, stream);
+}
+
+pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value,
+                           void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                           const int32_t* block_tables, int max_blocks_per_seq,
+                           const int32_t* context_lens, int num_seqs, int num_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           float scale, pa_dtype dtype, pa_stream_t stream) {
+    if (num_seqs > 0 && !slot_mapping) return fail(PA_ERR_INVALID_ARG, "null slot_mapping");
+    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       scale, dtype, key, value, slot_mapping, stream);
 }
 
 size_t pa_decode_split_workspace_bytes(int num_seqs, int num_heads, int head_dim,

@@ -174,6 +174,12 @@ __device__ __forceinline__ void mma_bf16_16816_top(float& d0, float& d1, uint32_
     (void)x3;
 }
 
+// Order this thread's earlier generic-proxy global-memory writes before later
+// async-proxy (TMA) reads of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (TMA) accesses to the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -79,7 +79,41 @@ struct DecodeArgs {
     int part_tokens;              // split: partition size in tokens
     int max_parts;                // split: partitions per (sequence, head) in the workspace
     int sched;                    // pa_decode: SCHED_CLUSTER or SCHED_LPT
+    // fused append (pa_decode_append): the new token of sequence s, rows
+    // new_k/new_v [S, Hk, D], goes to slot new_slots[s] (-1: none) before
+    // the sequence is read; null when not appending
+    const void* new_k;
+    const void* new_v;
+    const int64_t* new_slots;
+    void* k_cache;                // written only by the fused append
+    void* v_cache;
 };
+
+// Fused append: the CTA of (seq, kvh) writes kv head kvh's part of the new
+// token's key and value rows into the cache, then makes the writes visible
+// to its own TMA loads.  Only this sequence reads the new token's block (a
+// shared block is copied before it is written), so no other CTA can race
+// with the write.  The caller follows with a CTA (or cluster) barrier.
+template <typename T, int D, int BS>
+__device__ __forceinline__ void append_row(const DecodeArgs& a, int seq, int kvh, void* k_cache,
+                                           void* v_cache) {
+    constexpr int NV = D * (int)sizeof(T) / 16;          // 16-byte vectors per head row
+    const int64_t slot = a.new_slots[seq];
+    if (slot < 0) return;
+    if (slot >= (int64_t)a.num_blocks * BS) {
+        if (threadIdx.x == 0) raise_error(a.err, PA_DEVERR_SLOT);
+        return;
+    }
+    const size_t src = ((size_t)seq * a.num_kv_heads + kvh) * NV;
+    const size_t dst = ((size_t)slot * a.num_kv_heads + kvh) * NV;
+    for (int i = threadIdx.x; i < 2 * NV; i += blockDim.x) {
+        const bool val = i >= NV;
+        const int j = val ? i - NV : i;
+        const uint4 x = reinterpret_cast<const uint4*>(val ? a.new_v : a.new_k)[src + j];
+        reinterpret_cast<uint4*>(val ? v_cache : k_cache)[dst + j] = x;
+    }
+    fence_proxy_async_global();
+}
 
 enum class Mode { Decode, Split };
 
@@ -708,6 +742,13 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             kvh = blockIdx.y;
             L = clamp_len(seq);
             const int ctas = gridDim.x;
+            if (a.new_slots) {
+                if (blockIdx.x == 0) append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
+                if (ctas > 1)
+                    cg::this_cluster().sync();         // every rank loads after the write
+                else
+                    __syncthreads();
+            }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
             run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, ctas, blockIdx.x,
                         [&](int g, int d, float big, float num, float den, float* x) {
@@ -811,6 +852,10 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             seq = *pick;
             kvh = blockIdx.x % Hk;
             L = S <= MAX_SORT ? lens[seq] : clamp_len(seq);
+            if (a.new_slots) {
+                append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
+                __syncthreads();                       // the loads below see the new row
+            }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
             run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, 1, 0,
                         [&](int g, int d, float big, float num, float den, float*) {
