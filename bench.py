@@ -239,6 +239,11 @@ def build_prefix_loop(device, extra_tokens: int, kernel: str, partition: int):
         free_order=pp.free_order, block_tables=tables.copy(), seed=pp.seed, scale=pp.scale)
     loop = DecodeLoop(problem, device, kernel, partition,
                       state=(kc, vc, q0, alloc, tables, lens))
+    shared = (pp.prefix_len // bs) * bs            # whole blocks no one has copied
+    shared -= shared % 16
+    loop.groups = {"starts": torch.tensor([0, s], dtype=torch.int32, device=device),
+                   "prefix": torch.tensor([shared], dtype=torch.int32, device=device),
+                   "max_size": s, "max_prefix": shared}
     return loop
 
 
@@ -348,10 +353,20 @@ class DecodeLoop:
     def launches_per_step(self, n_cow: int) -> int:
         if self.fused:
             return (1 if n_cow else 0) + 1
-        return (1 if n_cow else 0) + 1 + (2 if self.kernel == "split" else 1)
+        per = {"split": 2, "cascade": 2}.get(self.kernel, 1)
+        return (1 if n_cow else 0) + 1 + per
 
     def decode(self, q, tables_d, lens_d, max_len):
-        if self.kernel == "split":
+        if self.kernel == "cascade":
+            g = self.groups
+            need = self.pa.pa_decode_shared_prefix_workspace_bytes(
+                self.p.num_seqs, self.p.num_heads, self.p.head_dim, g["max_prefix"])
+            if self.ws is None or self.ws.numel() < need:
+                self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self.pa.pa_decode_shared_prefix(self.out, q, self.k_cache, self.v_cache, tables_d,
+                                            lens_d, self.p.scale, g["starts"], g["prefix"],
+                                            g["max_size"], g["max_prefix"], self.ws)
+        elif self.kernel == "split":
             self.pa.pa_decode_split(self.out, q, self.k_cache, self.v_cache, tables_d, lens_d,
                                     self.p.scale, max_len, self.partition, self.workspace(max_len))
         else:
@@ -539,11 +554,12 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int):
         if loop.fused:
             pa.pa_decode_append(b.out, b.q, b.k, b.v, loop.k_cache, loop.v_cache, b.slots,
                                 b.tables, b.lens, p.scale, stream=comp)
-        elif loop.kernel == "split":
+        elif loop.kernel in ("split", "cascade"):
             pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
-            mx = int(lens_np.max())
-            pa.pa_decode_split(b.out, b.q, loop.k_cache, loop.v_cache, b.tables, b.lens,
-                               p.scale, mx, loop.partition, loop.workspace(mx), stream=comp)
+            saved_out, loop.out = loop.out, b.out
+            with torch.cuda.stream(comp):
+                loop.decode(b.q, b.tables, b.lens, int(lens_np.max()))
+            loop.out = saved_out
         else:
             pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
             pa.pa_decode(b.out, b.q, loop.k_cache, loop.v_cache, b.tables, b.lens, p.scale,
@@ -699,7 +715,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["gqa", "mha", "long", "prefix"], default="gqa")
-    ap.add_argument("--kernel", choices=["decode", "split"], default=None)
+    ap.add_argument("--kernel", choices=["decode", "split", "cascade"], default=None)
     ap.add_argument("--partition", type=int, default=512)
     ap.add_argument("--fused", action="store_true",
                     help="pa_decode_append: the cache write fused into the decode launch")
@@ -714,6 +730,8 @@ def main():
         args.kernel = "split" if args.workload == "long" else "decode"
     if args.fused and args.kernel != "decode":
         ap.error("--fused fuses the cache write into pa_decode (not the split kernel)")
+    if args.kernel == "cascade" and args.workload != "prefix":
+        ap.error("--kernel cascade needs the prefix workload (its sequences share a prefix)")
     rank, world, local = dist_env()
     if world != args.gpus and world > 1:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE {world}")
@@ -769,8 +787,10 @@ def main():
             "tokens_per_s": round(tokens_all / secs, 1),
             "frac_of_nominal_8tbps": round(value / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm",
-                         "kernel": ("pa_decode_append" if args.fused else "pa_decode")
-                         if args.kernel == "decode" else "pa_decode_split (partition + reduce)",
+                         "kernel": {"decode": "pa_decode_append" if args.fused else "pa_decode",
+                                    "split": "pa_decode_split (partition + reduce)",
+                                    "cascade": "pa_decode_shared_prefix (shared pass, then own "
+                                               "tokens merged)"}[args.kernel],
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "frac_of_nominal_8tbps": round(achieved / NOMINAL_HBM_GBS, 4),

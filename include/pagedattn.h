@@ -213,6 +213,43 @@ pa_status pa_decode_split_noalloc(void* out_d, const void* q_d,
                                   int partition_size, pa_stream_t stream);
 
 /*
+ * pa_decode_shared_prefix -- decode of a batch whose sequences come in groups
+ * sharing a prefix: sequences [group_starts[g], group_starts[g+1]) all start
+ * with the same prefix_lens[g] tokens in the same physical blocks (forks of
+ * one prompt: [course] 2.4.3 block tables pointing at the same physical
+ * blocks; [csdn-QA] 三 item 8 shared prefix pages).  Same result as
+ * pa_decode.  First the members of a group attend over the shared prefix
+ * together -- members x G query rows form one dense contraction per kv head,
+ * so each prefix block comes from HBM once per kv head (once per 64 query
+ * rows from L2) instead of once per sequence -- leaving per-chunk partial
+ * results in the workspace; then
+ * pa_decode's kernel covers each sequence's own tokens and merges those
+ * partials (log-sum-exp) into the output.  Two launches.
+ *   group_starts_d   int32 [num_groups + 1], ascending, 0 .. num_seqs (the
+ *                    groups cover every sequence; a group of one with prefix
+ *                    0 is a plain sequence)
+ *   prefix_lens_d    int32 [num_groups]: shared tokens, whole blocks and a
+ *                    multiple of 16, at most max_prefix_len; every member is
+ *                    at least that long and has the same first
+ *                    prefix_lens[g] / block_size table entries
+ *   max_group_size   >= every group's size
+ *   workspace_d      >= pa_decode_shared_prefix_workspace_bytes(...) bytes
+ * bf16 and block_size 16 or 32 only (else PA_ERR_UNSUPPORTED).  Validate
+ * mode checks every precondition above.
+ */
+size_t pa_decode_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                               int max_prefix_len);
+
+pa_status pa_decode_shared_prefix(void* out_d, const void* q_d, const void* k_cache_d,
+                                  const void* v_cache_d, const int32_t* block_tables_d,
+                                  int max_blocks_per_seq, const int32_t* context_lens_d,
+                                  int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                  const int32_t* group_starts_d, const int32_t* prefix_lens_d,
+                                  int num_groups, int max_group_size, int max_prefix_len,
+                                  void* workspace_d, size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * pa_copy_blocks -- copy-on-write of shared blocks: for each pair
  * (src, dst) the whole key block and value block dst <- src ([course] 2.4.3:
  * a write to a block whose reference count exceeds one first copies it).

@@ -13,6 +13,7 @@ Functions carry the C names:
 * ``pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, ...)``
 * ``pa_decode_split(out, q, ..., max_context_len, partition_size, workspace)``
 * ``pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size)``
+* ``pa_decode_shared_prefix(out, q, ..., group_starts, prefix_lens, ...)``
 * ``pa_copy_blocks(k_cache, v_cache, block_mapping)``
 * ``pa_device_error(clear=True)``, ``pa_set_option(name, value)``
 
@@ -31,7 +32,8 @@ from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SP
 
 __all__ = [
     "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_split", "pa_decode_split_workspace_bytes",
-    "pa_decode_split_noalloc", "pa_copy_blocks", "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
+    "pa_decode_split_noalloc", "pa_decode_shared_prefix",
+    "pa_decode_shared_prefix_workspace_bytes", "pa_copy_blocks", "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
     "PagedAttnError", "OutOfBlocks", "DEVERR_BITS",
 ]
 
@@ -145,6 +147,34 @@ def pa_decode_split_noalloc(out, q, k_cache, v_cache, block_tables, context_lens
                                         _ptr(context_lens), s, hq, hk, d, bs, nb, float(scale),
                                         _dtype(q), int(max_context_len), int(partition_size),
                                         _stream(stream)))
+    return out
+
+
+def pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, head_dim,
+                                            max_prefix_len) -> int:
+    return int(lib().pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                             max_prefix_len))
+
+
+def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                            group_starts, prefix_lens, max_group_size, max_prefix_len,
+                            workspace=None, stream=None):
+    """Decode of a batch whose sequences come in groups sharing a prefix:
+    group_starts int32 [G+1] (device), prefix_lens int32 [G] (device, whole
+    blocks, multiples of 16).  Same result as pa_decode."""
+    _dev(out, q, k_cache, v_cache, block_tables, context_lens, group_starts, prefix_lens)
+    s, hq, d = q.shape
+    nb, bs, hk, _ = k_cache.shape
+    need = pa_decode_shared_prefix_workspace_bytes(s, hq, d, max_prefix_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _dev(workspace)
+    check(lib().pa_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb, float(scale), _dtype(q),
+        _ptr(group_starts), _ptr(prefix_lens), prefix_lens.shape[0], int(max_group_size),
+        int(max_prefix_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
     return out
 
 

@@ -51,6 +51,10 @@ SIGNATURES = {
     "pa_decode_split_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
                                          _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _c_int,
                                          _c_int, _vp]),
+    "pa_decode_shared_prefix_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "pa_decode_shared_prefix": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp,
+                                         _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
     "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _vp]),
     "pa_alloc_create": (_vp, [_c_int, _c_int, _i32p]),

@@ -441,6 +441,7 @@ pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const v
     l.args.num_blocks = num_blocks;
     l.args.part_tokens = partition_size;
     l.args.max_parts = (int)parts64;
+    l.args.slot_stride = (int)parts64;
     l.k_cache = k_cache;
     l.v_cache = v_cache;
     l.num_seqs = num_seqs;
@@ -449,6 +450,118 @@ pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const v
     l.group = num_heads / num_kv_heads;
     l.ctas = 1;
     l.split = true;
+    l.stream = st;
+    return dispatch_decode(l, dtype, head_dim);
+}
+
+size_t pa_decode_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                               int max_prefix_len) {
+    if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_prefix_len < 0) return 0;
+    const size_t chunks = (size_t)((max_prefix_len + PREFIX_CHUNK_TOKENS - 1) / PREFIX_CHUNK_TOKENS);
+    const size_t rows = (size_t)num_seqs * num_heads * (chunks ? chunks : 1);
+    return 2 * align256(rows * sizeof(float)) + rows * head_dim * sizeof(float);
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  int max_blocks_per_seq, const int32_t* context_lens,
+                                  int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                  const int32_t* group_starts, const int32_t* prefix_lens,
+                                  int num_groups, int max_group_size, int max_prefix_len,
+                                  void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+    if (pa_status s = check_decode_args(out, q, k_cache, v_cache, block_tables,
+                                        max_blocks_per_seq, context_lens, num_seqs, num_heads,
+                                        num_kv_heads, head_dim, block_size, num_blocks, dtype,
+                                        scale))
+        return s;
+    if (dtype != PA_DTYPE_BF16 || block_size % 16 != 0)
+        return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs bf16 and block_size 16 or 32");
+    if (num_groups <= 0 || max_group_size <= 0 || max_prefix_len < 0 ||
+        (int64_t)max_prefix_len > (int64_t)max_blocks_per_seq * block_size)
+        return fail(PA_ERR_INVALID_ARG, "bad group or prefix bounds");
+    if ((int64_t)num_groups * ((max_group_size * (num_heads / num_kv_heads) +
+                                PREFIX_ROWS_PER_CTA - 1) / PREFIX_ROWS_PER_CTA) > 65535)
+        return fail(PA_ERR_UNSUPPORTED, "too many groups x row blocks for one launch");
+    if (num_seqs == 0) return PA_OK;
+    if (!group_starts || !prefix_lens) return fail(PA_ERR_INVALID_ARG, "null group arrays");
+    const size_t need = pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                                max_prefix_len);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+        return fail(PA_ERR_INVALID_ARG, "workspace needs %zu bytes, 16-byte aligned", need);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (validate_enabled()) {
+        if (pa_status s = validate_decode(block_tables, max_blocks_per_seq, context_lens,
+                                          num_seqs, block_size, num_blocks, st))
+            return s;
+        std::vector<int32_t> gs, pl, t, l;
+        if (!copy_to_host(gs, group_starts, (size_t)num_groups + 1, st) ||
+            !copy_to_host(pl, prefix_lens, (size_t)num_groups, st) ||
+            !copy_to_host(l, context_lens, (size_t)num_seqs, st) ||
+            !copy_to_host(t, block_tables, (size_t)num_seqs * max_blocks_per_seq, st))
+            return fail(PA_ERR_CUDA, "validation copy failed");
+        if (gs[0] != 0 || gs[num_groups] != num_seqs)
+            return fail(PA_ERR_BAD_BLOCK_ID, "groups must cover sequences 0..num_seqs-1");
+        for (int g = 0; g < num_groups; ++g) {
+            if (gs[g + 1] <= gs[g] || gs[g + 1] - gs[g] > max_group_size)
+                return fail(PA_ERR_BAD_BLOCK_ID, "group %d is empty or above max_group_size", g);
+            if (pl[g] < 0 || pl[g] > max_prefix_len || pl[g] % 16 || pl[g] % block_size)
+                return fail(PA_ERR_BAD_BLOCK_ID, "prefix of group %d (%d) is not whole blocks "
+                            "of 16 tokens within max_prefix_len", g, pl[g]);
+            const int nb = pl[g] / block_size;
+            for (int s = gs[g]; s < gs[g + 1]; ++s) {
+                if (l[s] < pl[g])
+                    return fail(PA_ERR_BAD_BLOCK_ID, "sequence %d is shorter than its prefix", s);
+                for (int j = 0; j < nb; ++j)
+                    if (t[(size_t)s * max_blocks_per_seq + j] !=
+                        t[(size_t)gs[g] * max_blocks_per_seq + j])
+                        return fail(PA_ERR_BAD_BLOCK_ID,
+                                    "sequence %d does not share block %d of its group's prefix",
+                                    s, j);
+            }
+        }
+    }
+    const int chunks = (max_prefix_len + PREFIX_CHUNK_TOKENS - 1) / PREFIX_CHUNK_TOKENS;
+    const int group = num_heads / num_kv_heads;
+    const size_t rows = (size_t)num_seqs * num_heads * (size_t)(chunks ? chunks : 1);
+    char* ws = static_cast<char*>(workspace);
+    DecodeLaunch l = {};
+    l.args.out = out;
+    l.args.q = q;
+    l.args.block_tables = block_tables;
+    l.args.context_lens = context_lens;
+    l.args.ws_m = reinterpret_cast<float*>(ws);
+    l.args.ws_l = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
+    l.args.ws_o = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
+    l.args.err = device_error_word();
+    if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    l.args.scale_log2 = scale * 1.4426950408889634f;
+    l.args.num_seqs = num_seqs;
+    l.args.max_blocks = max_blocks_per_seq;
+    l.args.max_tokens = max_blocks_per_seq * block_size;
+    l.args.num_heads = num_heads;
+    l.args.num_kv_heads = num_kv_heads;
+    l.args.num_blocks = num_blocks;
+    l.args.group_starts = group_starts;
+    l.args.group_prefix = prefix_lens;
+    l.args.num_groups = num_groups;
+    l.args.chunk_tokens = PREFIX_CHUNK_TOKENS;
+    l.args.prefix_slot0 = 0;
+    l.args.slot_stride = chunks ? chunks : 1;
+    l.args.sched = SCHED_LPT;
+    l.k_cache = k_cache;
+    l.v_cache = v_cache;
+    l.num_seqs = num_seqs;
+    l.num_kv_heads = num_kv_heads;
+    l.block_size = block_size;
+    l.group = group;
+    l.ctas = 1;
+    l.split = false;
+    l.cascade = true;
+    l.max_chunks = chunks;
+    const int max_rows = max_group_size * group;
+    l.row_blocks = (max_rows + PREFIX_ROWS_PER_CTA - 1) / PREFIX_ROWS_PER_CTA;
+    l.consumers = cmin(PrefixCfg<64, 16, 1>::MAX_CONSUMERS, (max_rows + 15) / 16);
     l.stream = st;
     return dispatch_decode(l, dtype, head_dim);
 }

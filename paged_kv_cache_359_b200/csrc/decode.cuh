@@ -87,7 +87,31 @@ struct DecodeArgs {
     const int64_t* new_slots;
     void* k_cache;                // written only by the fused append
     void* v_cache;
+    // shared-prefix decode: sequences [group_starts[g], group_starts[g+1])
+    // share their first group_prefix[g] tokens.  The shared pass leaves one
+    // (max, sum, unnormalised output) per (sequence, head, prefix chunk) at
+    // workspace slots [prefix_slot0, prefix_slot0 + ceil(prefix / chunk_tokens));
+    // pa_decode's CTAs then cover only each sequence's own tokens and merge
+    // those chunks into their output.  null: off
+    const int32_t* group_starts;
+    const int32_t* group_prefix;
+    int num_groups;
+    int chunk_tokens;
+    int prefix_slot0;
+    int slot_stride;              // workspace slots per (sequence, head)
 };
+
+// Group of sequence `seq` (binary search over group_starts) and its shared
+// prefix length; 0 when no groups are given.
+__device__ __forceinline__ int shared_prefix_of(const DecodeArgs& a, int seq) {
+    if (!a.group_starts) return 0;
+    int lo = 0, hi = a.num_groups;           // group_starts[lo] <= seq < group_starts[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(a.group_starts + mid) <= seq) lo = mid; else hi = mid;
+    }
+    return __ldg(a.group_prefix + lo);
+}
 
 // Fused append: the CTA of (seq, kvh) writes kv head kvh's part of the new
 // token's key and value rows into the cache, then makes the writes visible
@@ -725,7 +749,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
         run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, u_begin, u_end, 1, 0,
                     [&](int g, int d, float big, float num, float den, float*) {
                         if (nparts > 1) {
-                            const size_t slot = (head0 + g) * a.max_parts + part;
+                            const size_t slot = (head0 + g) * a.slot_stride + part;
                             if (d == 0) {
                                 a.ws_m[slot] = big;
                                 a.ws_l[slot] = den;
@@ -802,7 +826,9 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                 for (int i = threadIdx.x; i < S; i += NT) {
                     const int x = a.context_lens[i];
                     if (x < 0 || x > a.max_tokens) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
-                    lens[i] = x < 0 ? 0 : (x > a.max_tokens ? a.max_tokens : x);
+                    const int len = x < 0 ? 0 : (x > a.max_tokens ? a.max_tokens : x);
+                    // order by the tokens this pass reads (own tokens with a shared prefix)
+                    lens[i] = len - cmin(shared_prefix_of(a, i), len);
                 }
             __syncthreads();
             if (warp == 0) {
@@ -851,19 +877,89 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             __syncthreads();
             seq = *pick;
             kvh = blockIdx.x % Hk;
-            L = S <= MAX_SORT ? lens[seq] : clamp_len(seq);
+            L = S <= MAX_SORT && !a.group_starts ? lens[seq] : clamp_len(seq);
+            const int tok0 = cmin(shared_prefix_of(a, seq), L);    // whole 16-token units
             if (a.new_slots) {
                 append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
                 __syncthreads();                       // the loads below see the new row
             }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
-            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, 1, 0,
-                        [&](int g, int d, float big, float num, float den, float*) {
+            const int nchunks = a.group_starts ? (tok0 + a.chunk_tokens - 1) / a.chunk_tokens : 0;
+            // chunk weights of the shared pass live after the exchange area
+            constexpr int XCH_FLOATS = (NW + 1) * G * (D + 2);
+            constexpr int MAX_STAGED_CHUNKS = (Ly::MAIN_REGION / 4 - XCH_FLOATS - G) / (2 * G);
+            const bool staged = nchunks > 0 && nchunks <= MAX_STAGED_CHUNKS;
+            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, tok0 / R, (L + R - 1) / R, 1, 0,
+                        [&](int g, int d, float big, float num, float den, float* x) {
+                            if (staged) {
+                                // keep this CTA's own part; merged below with the chunks
+                                if (d == 0) {
+                                    x[g] = big;
+                                    x[G + g] = den;
+                                }
+                                x[2 * G + g * D + d] = num;
+                                return;
+                            }
+                            if (nchunks) {
+                                // merge with the shared pass's chunks of this head
+                                const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0;
+                                float mm = big;
+                                for (int c = 0; c < nchunks; ++c) mm = fmaxf(mm, a.ws_m[b + c]);
+                                const float e = big == -INFINITY ? 0.f : exp2_approx(big - mm);
+                                num *= e;
+                                den *= e;
+                                for (int c = 0; c < nchunks; ++c) {
+                                    const float ec = exp2_approx(a.ws_m[b + c] - mm);
+                                    num = fmaf(ec, a.ws_o[(b + c) * D + d], num);
+                                    den = fmaf(ec, a.ws_l[b + c], den);
+                                }
+                            }
                             store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
                         });
+            if (staged) {
+                // merge this CTA's part with the shared pass's chunks: chunk
+                // maxima and sums staged once, weights once per head, then
+                // every output's chunk loads issued independently
+                float* x = reinterpret_cast<float*>(smem) + NW * G * (D + 2);
+                float* cw = x + 2 * G + G * D;           // [G][nchunks] weights, then sums
+                float* cl = cw + G * nchunks;
+                float* tot = cl + G * nchunks;           // [G] own weight, then total sum
+                __syncthreads();
+                for (int i = threadIdx.x; i < G * nchunks; i += NT) {
+                    const int g = i / nchunks, c = i % nchunks;
+                    const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0 + c;
+                    cw[i] = a.ws_m[b];
+                    cl[i] = a.ws_l[b];
+                }
+                __syncthreads();
+                if (threadIdx.x < G) {
+                    const int g = threadIdx.x;
+                    float mm = x[g];
+                    for (int c = 0; c < nchunks; ++c) mm = fmaxf(mm, cw[g * nchunks + c]);
+                    const float e0 = x[g] == -INFINITY ? 0.f : exp2_approx(x[g] - mm);
+                    float den = e0 * x[G + g];
+                    for (int c = 0; c < nchunks; ++c) {
+                        const float ec = exp2_approx(cw[g * nchunks + c] - mm);
+                        cw[g * nchunks + c] = ec;
+                        den = fmaf(ec, cl[g * nchunks + c], den);
+                    }
+                    tot[g] = e0;
+                    x[G + g] = den;
+                }
+                __syncthreads();
+                for (int idx = threadIdx.x; idx < G * D; idx += NT) {
+                    const int g = idx / D, d = idx % D;
+                    const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0;
+                    float num = tot[g] * x[2 * G + g * D + d];
+#pragma unroll 8
+                    for (int c = 0; c < nchunks; ++c)
+                        num = fmaf(cw[g * nchunks + c], a.ws_o[(b + c) * D + d], num);
+                    const float den = x[G + g];
+                    store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                }
+            }
             return;
         }
-
     }
 }
 
@@ -879,9 +975,10 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
     L = L < 0 ? 0 : cmin(L, a.max_tokens);
     const int nparts = (L + a.part_tokens - 1) / a.part_tokens;
     if (nparts <= 1 || nparts > a.max_parts) return;   // written directly by the partition kernel
-    const float* m = a.ws_m + (size_t)sh * a.max_parts;
-    const float* l = a.ws_l + (size_t)sh * a.max_parts;
-    const float* o = a.ws_o + (size_t)sh * a.max_parts * D;
+    const size_t base = (size_t)sh * a.slot_stride;
+    const float* m = a.ws_m + base;
+    const float* l = a.ws_l + base;
+    const float* o = a.ws_o + base * D;
 
     __shared__ float red[8];
     __shared__ float part_num[8][32];

@@ -7,6 +7,7 @@
 
 #include "decode.cuh"
 #include "internal.h"
+#include "prefix.cuh"
 
 namespace pa {
 
@@ -20,6 +21,12 @@ struct DecodeLaunch {
     int group;
     int ctas;          // pa_decode: CTAs (one cluster) per (sequence, kv head)
     bool split;
+    // shared-prefix decode: the shared pass runs first (grid max_chunks x Hk x
+    // groups * row_blocks, `consumers` + 1 warps), then the split pass
+    bool cascade;
+    int max_chunks;
+    int row_blocks;
+    int consumers;
     cudaStream_t stream;
 };
 
@@ -59,6 +66,35 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
     cfg.dynamicSmemBytes = Ly::SMEM_BYTES;
     cfg.stream = l.stream;
     cudaError_t e;
+    if (l.cascade) {
+        if constexpr (std::is_same<T, __nv_bfloat16>::value && BS % 16 == 0) {
+            using C = PrefixCfg<D, BS, G>;
+            static std::atomic<unsigned long long> done_p{0};
+            auto pk = shared_prefix_kernel<D, BS, G>;
+            if (pa_status s = allow_smem(pk, C::SMEM_BYTES, done_p)) return s;
+            // all of L1 as shared memory, so two CTAs fit an SM
+            cudaFuncSetAttribute(pk, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            CUtensorMap sk, sv;        // 128B-swizzled {64, 1, 16, 1} boxes
+            if (pa_status s = encode_cache_map(&sk, l.k_cache, DT, D, l.num_kv_heads, BS,
+                                               l.args.num_blocks, 64, 16, true))
+                return s;
+            if (pa_status s = encode_cache_map(&sv, l.v_cache, DT, D, l.num_kv_heads, BS,
+                                               l.args.num_blocks, 64, 16, true))
+                return s;
+            if (l.max_chunks > 0) {
+                cudaLaunchConfig_t pc = {};
+                pc.gridDim = dim3(l.max_chunks, l.num_kv_heads, l.args.num_groups * l.row_blocks);
+                pc.blockDim = dim3((l.consumers + 1) * 32);
+                pc.dynamicSmemBytes = C::SMEM_BYTES;
+                pc.stream = l.stream;
+                e = cudaLaunchKernelEx(&pc, pk, sk, sv, l.args, l.row_blocks);
+                if (e != cudaSuccess)
+                    return fail(PA_ERR_CUDA, "shared-prefix launch: %s", cudaGetErrorString(e));
+            }
+        } else {
+            return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs bf16 and 16 | block_size");
+        }
+    }
     if (l.split) {
         static std::atomic<unsigned long long> done{0};
         auto kern = paged_decode_kernel<U, Mode::Split>;
