@@ -263,6 +263,27 @@ pa_status pa_copy_blocks(void* k_cache_d, void* v_cache_d,
                          pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * pa_swap_blocks -- move whole blocks (keys and values) between two pools,
+ * typically the device cache and a pinned host cache: swapping pages out of
+ * HBM and back ([csdn-QA] 三 item 10: page migration through pinned memory
+ * and asynchronous copies).  For each pair (src, dst) of block_mapping,
+ * block dst of the destination pool <- block src of the source pool.
+ *   dst_k, dst_v, src_k, src_v  [num_blocks, block_size, kv_heads, head_dim]
+ *                    pools: device memory, or pinned host memory (device-
+ *                    mapped under unified addressing, as cudaHostAlloc /
+ *                    torch pin_memory give); pageable host memory returns
+ *                    PA_ERR_UNSUPPORTED
+ *   block_mapping    int64 [num_pairs, 2] (src, dst), device or pinned host
+ * One kernel moves every pair, 16 bytes per thread access, over the GPU's
+ * link for host pools.  Destinations must be distinct (validate mode checks);
+ * an id outside its pool skips the pair and sets PA_DEVERR_COPY_ID.
+ */
+pa_status pa_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                         const int64_t* block_mapping, int num_pairs, int num_kv_heads,
+                         int head_dim, int block_size, int src_num_blocks, int dst_num_blocks,
+                         pa_dtype dtype, pa_stream_t stream);
+
+/*
  * Host block allocator ([tech] 2.1 Block {ref_count, is_allocated} and the
  * pool descriptor, 4.2 immediate reclamation at ref_count 0 and a free pool;
  * [csdn-QA] 三 item 7 slab-style frames, item 8 shared prefix pages;

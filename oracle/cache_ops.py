@@ -9,7 +9,11 @@
   reference count exceeds one first copies the whole block (keys and values)
   into a fresh block ([course] §2.4.3 pitfall note).
 
-Both return new tensors and leave their inputs untouched.  Duplicate slots,
+* ``swap_blocks``: a page moves between two pools -- the device cache and a
+  pinned host cache -- whole blocks of keys and values ([csdn-QA] §三
+  item 10: page migration through pinned memory and asynchronous copies).
+
+All return new tensors and leave their inputs untouched.  Duplicate slots,
 duplicate destinations or a destination that is also a source are outside
 the definition (read as invalid input).
 """
@@ -42,4 +46,16 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping) -> 
     for src, dst in block_mapping:
         k_out[int(dst)] = k_cache[int(src)]
         v_out[int(dst)] = v_cache[int(src)]
+    return k_out, v_out
+
+
+def swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor,
+                dst_v: torch.Tensor, block_mapping) -> tuple:
+    """block_mapping: (src, dst) pairs; block dst of the destination pool
+    receives block src of the source pool.  Returns the new destination."""
+    k_out = dst_k.clone()
+    v_out = dst_v.clone()
+    for src, dst in block_mapping:
+        k_out[int(dst)] = src_k[int(src)]
+        v_out[int(dst)] = src_v[int(src)]
     return k_out, v_out

@@ -15,6 +15,7 @@ Functions carry the C names:
 * ``pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size)``
 * ``pa_decode_shared_prefix(out, q, ..., group_starts, prefix_lens, ...)``
 * ``pa_copy_blocks(k_cache, v_cache, block_mapping)``
+* ``pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping)``
 * ``pa_device_error(clear=True)``, ``pa_set_option(name, value)``
 
 and ``BlockAllocator`` wraps the host allocator (``pa_alloc_*`` / ``pa_seq_*``).
@@ -33,7 +34,8 @@ from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SP
 __all__ = [
     "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_split", "pa_decode_split_workspace_bytes",
     "pa_decode_split_noalloc", "pa_decode_shared_prefix",
-    "pa_decode_shared_prefix_workspace_bytes", "pa_copy_blocks", "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
+    "pa_decode_shared_prefix_workspace_bytes", "pa_copy_blocks", "pa_swap_blocks",
+    "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
     "PagedAttnError", "OutOfBlocks", "DEVERR_BITS",
 ]
 
@@ -187,6 +189,23 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
     check(lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping),
                                block_mapping.shape[0], hk, d, bs, nb, _dtype(k_cache),
                                _stream(stream)))
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None):
+    """Move blocks between pools (device cache <-> pinned host cache):
+    block_mapping int64 [P, 2] of (src, dst), device or pinned host."""
+    for t in (dst_k, dst_v, src_k, src_v, block_mapping):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError("pools and mapping must be on a CUDA device or in pinned memory")
+    if block_mapping.dtype != torch.int64:
+        raise ValueError("block_mapping must be int64")
+    nb_dst, bs, hk, d = dst_k.shape
+    nb_src = src_k.shape[0]
+    check(lib().pa_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v),
+                               _ptr(block_mapping), block_mapping.shape[0], hk, d, bs, nb_src,
+                               nb_dst, _dtype(dst_k), _stream(stream)))
 
 
 def pa_device_error(clear: bool = True, stream=None) -> int:

@@ -57,6 +57,8 @@ SIGNATURES = {
                                          _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
     "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _vp]),
+    "pa_swap_blocks": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                _c_int, _c_int, _vp]),
     "pa_alloc_create": (_vp, [_c_int, _c_int, _i32p]),
     "pa_alloc_destroy": (None, [_vp]),
     "pa_alloc_allocate": (_c_int, [_vp, _i32p]),

@@ -601,4 +601,63 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapp
                               st);
 }
 
+// Device-usable address of a pool: device or managed memory as is, pinned host
+// memory through its device mapping; null if the GPU cannot reach it.
+static void* device_view(const void* p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();                       // pageable memory reports an error: clear it
+        return nullptr;
+    }
+    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged)
+        return const_cast<void*>(p);
+    if (attr.type == cudaMemoryTypeHost && attr.devicePointer) {
+        // the mapping covers the whole allocation: offset the mapped base
+        const uintptr_t off = reinterpret_cast<uintptr_t>(p) -
+                              reinterpret_cast<uintptr_t>(attr.hostPointer);
+        return static_cast<char*>(attr.devicePointer) + off;
+    }
+    return nullptr;
+}
+
+pa_status pa_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                         const int64_t* block_mapping, int num_pairs, int num_kv_heads,
+                         int head_dim, int block_size, int src_num_blocks, int dst_num_blocks,
+                         pa_dtype dtype, pa_stream_t stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || src_num_blocks <= 0 || dst_num_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "sizes must be positive (num_pairs >= 0)");
+    if (pa_status s = check_geometry(dtype, head_dim, block_size)) return s;
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_k || !dst_v || !src_k || !src_v || !block_mapping)
+        return fail(PA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(dst_k) || !aligned16(dst_v) || !aligned16(src_k) || !aligned16(src_v))
+        return fail(PA_ERR_INVALID_ARG, "pools must be 16-byte aligned");
+    void* dk = device_view(dst_k);
+    void* dv = device_view(dst_v);
+    const void* sk = device_view(src_k);
+    const void* sv = device_view(src_v);
+    const void* mp = device_view(block_mapping);
+    if (!dk || !dv || !sk || !sv || !mp)
+        return fail(PA_ERR_UNSUPPORTED, "pools and mapping must be device memory or pinned "
+                    "(device-mapped) host memory");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (validate_enabled()) {
+        std::vector<int64_t> m;
+        if (!copy_to_host(m, static_cast<const int64_t*>(mp), (size_t)num_pairs * 2, st))
+            return fail(PA_ERR_CUDA, "validation copy failed");
+        std::unordered_set<int64_t> dsts;
+        for (int i = 0; i < num_pairs; ++i) {
+            if (m[2 * i] < 0 || m[2 * i] >= src_num_blocks || m[2 * i + 1] < 0 ||
+                m[2 * i + 1] >= dst_num_blocks)
+                return fail(PA_ERR_BAD_BLOCK_ID, "block_mapping[%d] outside its pool", i);
+            if (!dsts.insert(m[2 * i + 1]).second)
+                return fail(PA_ERR_BAD_BLOCK_ID, "destination %lld repeated",
+                            (long long)m[2 * i + 1]);
+        }
+    }
+    const int64_t block_bytes = (int64_t)block_size * num_kv_heads * head_dim * elem_size(dtype);
+    return launch_move_blocks(dk, dv, sk, sv, static_cast<const int64_t*>(mp), num_pairs,
+                              block_bytes, src_num_blocks, dst_num_blocks, PA_DEVERR_COPY_ID, st);
+}
+
 }  // extern "C"

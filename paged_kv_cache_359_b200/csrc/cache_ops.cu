@@ -44,20 +44,24 @@ __global__ void __launch_bounds__(128)
     }
 }
 
+// Block dst of the destination pool <- block src of the source pool, keys and
+// values; the pools are the same cache (copy-on-write) or a device cache and
+// a pinned host cache reached through its device-mapped address (swapping).
 __global__ void __launch_bounds__(256)
-    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
-                       const int64_t* __restrict__ mapping, int64_t block_vecs, int num_blocks,
-                       unsigned* err) {
+    move_blocks_kernel(uint4* __restrict__ dst_k, uint4* __restrict__ dst_v,
+                       const uint4* __restrict__ src_k, const uint4* __restrict__ src_v,
+                       const int64_t* __restrict__ mapping, int64_t block_vecs, int src_blocks,
+                       int dst_blocks, unsigned err_bits, unsigned* err) {
     const int pair = blockIdx.x;
     const int64_t src = mapping[2 * pair], dst = mapping[2 * pair + 1];
-    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
-        if (threadIdx.x == 0 && blockIdx.y == 0) raise_error(err, PA_DEVERR_COPY_ID);
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) raise_error(err, err_bits);
         return;
     }
-    const uint4* ks = k_cache + src * block_vecs;
-    const uint4* vs = v_cache + src * block_vecs;
-    uint4* kd = k_cache + dst * block_vecs;
-    uint4* vd = v_cache + dst * block_vecs;
+    const uint4* ks = src_k + src * block_vecs;
+    const uint4* vs = src_v + src * block_vecs;
+    uint4* kd = dst_k + dst * block_vecs;
+    uint4* vd = dst_v + dst * block_vecs;
     for (int64_t i = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; i < block_vecs;
          i += (int64_t)gridDim.y * blockDim.x) {
         kd[i] = ks[i];
@@ -107,19 +111,28 @@ pa_status launch_reshape_and_cache(const void* key, const void* value, void* k_c
     return PA_OK;
 }
 
-pa_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping, int num_pairs,
-                             int64_t block_bytes, int num_blocks, cudaStream_t stream) {
+pa_status launch_move_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                             const int64_t* mapping, int num_pairs, int64_t block_bytes,
+                             int src_blocks, int dst_blocks, unsigned err_bits,
+                             cudaStream_t stream) {
     if (num_pairs == 0) return PA_OK;
     unsigned* err = device_error_word();
     if (!err) return fail(PA_ERR_CUDA, "device error word unavailable");
     const int64_t vecs = block_bytes / 16;
     int chunks = (int)(vecs / 1024);
     chunks = chunks < 1 ? 1 : (chunks > 32 ? 32 : chunks);
-    copy_blocks_kernel<<<dim3(num_pairs, chunks), 256, 0, stream>>>(
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), mapping, vecs, num_blocks, err);
+    move_blocks_kernel<<<dim3(num_pairs, chunks), 256, 0, stream>>>(
+        static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), static_cast<const uint4*>(src_k),
+        static_cast<const uint4*>(src_v), mapping, vecs, src_blocks, dst_blocks, err_bits, err);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "copy_blocks launch: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "block move launch: %s", cudaGetErrorString(e));
     return PA_OK;
+}
+
+pa_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping, int num_pairs,
+                             int64_t block_bytes, int num_blocks, cudaStream_t stream) {
+    return launch_move_blocks(k_cache, v_cache, k_cache, v_cache, mapping, num_pairs, block_bytes,
+                              num_blocks, num_blocks, PA_DEVERR_COPY_ID, stream);
 }
 
 }  // namespace pa

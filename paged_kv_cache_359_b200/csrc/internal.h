@@ -50,5 +50,9 @@ pa_status launch_reshape_and_cache(const void* key, const void* value, void* k_c
                                    int64_t row_bytes, int64_t num_slots, cudaStream_t stream);
 pa_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping, int num_pairs,
                              int64_t block_bytes, int num_blocks, cudaStream_t stream);
+pa_status launch_move_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                             const int64_t* mapping, int num_pairs, int64_t block_bytes,
+                             int src_blocks, int dst_blocks, unsigned err_bits,
+                             cudaStream_t stream);
 
 }  // namespace pa

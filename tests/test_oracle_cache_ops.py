@@ -71,3 +71,24 @@ def test_copy_blocks_copies_whole_blocks_bitwise():
     untouched = [b for b in range(nb) if b not in (7, 9, 6)]
     assert _same_bits(k_out[untouched], kc[untouched])
     assert _same_bits(v_out[untouched], vc[untouched])
+
+
+def test_swap_blocks_round_trip_restores_every_bit():
+    """Swap a set of device blocks out to a host pool and back into other
+    device blocks: the moved blocks carry the same bits, nothing else in
+    either pool changes, and the library's index_copy gives the same pool."""
+    nb, hb, bs, hk, d = 20, 12, 16, 2, 8
+    kc, vc = _pool(nb, bs, hk, d, seed=21), _pool(nb, bs, hk, d, seed=22)
+    hk_pool, hv_pool = _pool(hb, bs, hk, d, seed=23), _pool(hb, bs, hk, d, seed=24)
+    out = [(3, 0), (7, 5), (11, 2)]
+    h_k, h_v = oracle.swap_blocks(kc, vc, hk_pool, hv_pool, out)
+    src = torch.tensor([s for s, _ in out])
+    dst = torch.tensor([t for _, t in out])
+    assert _same_bits(h_k, hk_pool.clone().index_copy_(0, dst, kc[src]))
+    assert _same_bits(h_v, hv_pool.clone().index_copy_(0, dst, vc[src]))
+    back = [(0, 15), (5, 16), (2, 17)]
+    k2, v2 = oracle.swap_blocks(h_k, h_v, kc, vc, back)
+    for (s0, _), (_, t1) in zip(out, back):
+        assert _same_bits(k2[t1], kc[s0]) and _same_bits(v2[t1], vc[s0])
+    keep = [b for b in range(nb) if b not in (15, 16, 17)]
+    assert _same_bits(k2[keep], kc[keep]) and _same_bits(v2[keep], vc[keep])
