@@ -173,9 +173,10 @@ class ClockSampler:
 # workload
 # --------------------------------------------------------------------------
 
-def make_problem(name: str, extra_tokens: int, rank: int):
+def make_problem(name: str, extra_tokens: int, rank: int, block_size=None, head_dim=None):
     if name == "gqa":
-        return pa_inputs.gqa(extra_tokens=extra_tokens)
+        return pa_inputs.gqa(extra_tokens=extra_tokens, block_size=block_size or 16,
+                             head_dim=head_dim or 128)
     if name == "mha":
         p = pa_inputs.mha(max_len=2048 + extra_tokens,
                           num_blocks=8192 + 64 * (-(-extra_tokens // 16) + 1))
@@ -448,6 +449,62 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
             "cow_pairs": int(sum(len(c) for c in cows[warmup:]))}
 
 
+def run_compaction(loop: DecodeLoop, reps: int = 5):
+    """Compaction after the timed loop (not part of a step): every other
+    sequence ends and is freed, the host allocator packs the live blocks
+    below (live + 1 %) blocks, pa_copy_blocks moves their data, the tables
+    are remapped, and the survivors decode over the shrunken pool to the same
+    output bits as before the move.  The copy is idempotent (its sources are
+    not overwritten), so it is repeated ``reps`` times for the timing."""
+    pa, p, dev = loop.pa, loop.p, loop.device
+    bs = p.block_size
+    keep = np.arange(0, p.num_seqs, 2)
+    for i in range(1, p.num_seqs, 2):
+        loop.alloc.free(loop.tables[i], int(-(-int(loop.lens[i]) // bs)))
+    tables, lens = loop.tables[keep].copy(), loop.lens[keep].copy()
+    q = loop.q0[torch.from_numpy(keep).to(dev)].contiguous()
+    out0 = torch.empty_like(q)
+    lens_d = torch.from_numpy(lens).to(dev)
+    pa.pa_decode(out0, q, loop.k_cache, loop.v_cache, torch.from_numpy(tables).to(dev), lens_d,
+                 p.scale)
+    live = sum(1 for r in loop.alloc.ref_counts() if r > 0)
+    before = loop.alloc.num_blocks
+    target = min(before, live + max(1, live // 100))
+    t0 = time.perf_counter()
+    moves = loop.alloc.compact(target)
+    host_ms = (time.perf_counter() - t0) * 1e3
+    t0 = time.perf_counter()
+    n_blocks = -(-lens // bs)
+    for t, n in zip(tables, n_blocks):
+        pa.BlockAllocator.remap(t, int(n), moves)
+    remap_ms = (time.perf_counter() - t0) * 1e3
+    moves_d = torch.from_numpy(moves.astype(np.int64)).to(dev)
+    stream = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    pa.pa_copy_blocks(loop.k_cache, loop.v_cache, moves_d)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(reps):
+        pa.pa_copy_blocks(loop.k_cache, loop.v_cache, moves_d)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    copy_ms = ev[0].elapsed_time(ev[1]) / reps
+    out1 = torch.empty_like(q)
+    pa.pa_decode(out1, q, loop.k_cache[:target], loop.v_cache[:target],
+                 torch.from_numpy(tables).to(dev), lens_d, p.scale)
+    torch.cuda.synchronize()
+    bits = torch.int16 if out0.element_size() == 2 else torch.int32
+    same = bool(torch.equal(out0.view(bits), out1.view(bits)))
+    blk = bs * p.num_kv_heads * p.head_dim * 2 * p.elem_bytes       # K and V of one block
+    moved = len(moves) * blk
+    return {"pool_blocks_before": before, "pool_blocks_after": target, "live_blocks": live,
+            "moves": len(moves), "released_gb": round((before - target) * blk / 1e9, 3),
+            "host_compact_ms": round(host_ms, 3), "host_remap_ms": round(remap_ms, 3),
+            "copy_ms": round(copy_ms, 4),
+            "copy_gbs_read_plus_write": round(2 * moved / (copy_ms / 1e3) / 1e9, 1),
+            "decode_bits_identical": same}
+
+
 def _segments(spec):
     """Byte offsets of 256-byte-aligned segments: spec = [(name, nbytes), ...]."""
     off, out = 0, {}
@@ -642,7 +699,7 @@ def run_reference(args, rank, world):
     if world > 1 and rank != 0:
         return
     extra = args.steps + args.warmup + 2
-    p = make_problem(args.workload, extra, 0)
+    p = make_problem(args.workload, extra, 0, args.block_size, args.head_dim)
     data = pa_inputs.materialize(p, "cpu")
     kc, vc = data["k_cache"], data["v_cache"]
     alloc = oracle.BlockAllocator(p.num_blocks, p.block_size, p.free_order)
@@ -700,6 +757,9 @@ def workload_config(p, args):
             "head_dim": p.head_dim, "block_size": p.block_size, "num_blocks": p.num_blocks,
             "context_len_median": int(np.median(lens)), "context_len_max": int(lens.max()),
             "context_tokens": int(lens.astype(np.int64).sum()),
+            # internal fragmentation: unused rows of each sequence's last block
+            "block_waste_frac": round(1.0 - float(lens.astype(np.int64).sum()) / float(sum(
+                -(-int(x) // p.block_size) * p.block_size for x in lens)), 5),
             "kernel": args.kernel + ("+append (fused)" if args.fused else ""),
             "partition": args.partition,
             "l2": "inputs larger than L2 (KV cache %.2f GB vs 126 MB L2), no flush" %
@@ -721,6 +781,12 @@ def main():
                     help="pa_decode_append: the cache write fused into the decode launch")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block-size", type=int, default=None,
+                    help="gqa workload: block size (default 16; the block-size study)")
+    ap.add_argument("--head-dim", type=int, default=None,
+                    help="gqa workload: head_dim (default 128)")
+    ap.add_argument("--compact", action="store_true",
+                    help="after the timed loop: free half the batch, compact the pool, report")
     ap.add_argument("--ref-sample", type=int, default=64,
                     help="sequences decoded per step by the reference arm")
     args = ap.parse_args()
@@ -730,6 +796,10 @@ def main():
         args.kernel = "split" if args.workload == "long" else "decode"
     if args.fused and args.kernel != "decode":
         ap.error("--fused fuses the cache write into pa_decode (not the split kernel)")
+    if args.compact and args.workload not in ("gqa", "mha"):
+        ap.error("--compact runs on the gqa and mha workloads")
+    if (args.block_size or args.head_dim) and args.workload != "gqa":
+        ap.error("--block-size / --head-dim apply to the gqa workload")
     if args.kernel == "cascade" and args.workload != "prefix":
         ap.error("--kernel cascade needs the prefix workload (its sequences share a prefix)")
     rank, world, local = dist_env()
@@ -758,7 +828,7 @@ def main():
             loop = build_prefix_loop(dev, extra, args.kernel, args.partition)
             p = loop.p
         else:
-            p = make_problem(args.workload, extra, rank)
+            p = make_problem(args.workload, extra, rank, args.block_size, args.head_dim)
             loop = DecodeLoop(p, dev, args.kernel, args.partition)
         loop.fused = args.fused
         res = run_device_timed(loop, args.steps, args.warmup, world, local,
@@ -774,7 +844,10 @@ def main():
         dec_alg = statistics.fmean(res["dec_alg_bytes"])
         achieved = dec_alg / (dec_mean_ms / 1e3) / 1e9
         peak, peak_src = hbm_peak()
-        cap = measured_traffic()
+        # the committed capture is of the default gqa decode launch
+        default_shape = (args.workload == "gqa" and args.kernel == "decode" and not args.fused
+                         and args.block_size in (None, 16) and args.head_dim in (None, 128))
+        cap = measured_traffic() if default_shape else None
         # scaled from the captured launch to this run's mean launch by
         # algorithmic bytes (DRAM traffic grows with the tokens read)
         traffic = None if cap is None else round(cap[0] * dec_alg / cap[1])
@@ -815,6 +888,8 @@ def main():
                            "ms_per_step": round(e2e_ms / args.steps, 4)}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(loop)
+        if args.compact:                     # last: it frees half the batch
+            line["compaction"] = run_compaction(loop)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -30,7 +30,9 @@
  *     element size ([course] 2.3).
  *   - Supported: dtype f32 or bf16 (q, key/value rows, caches and outputs
  *     share one dtype; arithmetic is fp32), head_dim in {64, 128, 256},
- *     block_size in {8, 16, 32}, num_heads / num_kv_heads in {1, 2, 4, 8}.
+ *     block_size in {8, 16, 32, 64, 128} ([course] 2.3 and 2.5: 16 by
+ *     default, 8 and 32 tried; [tech] 4.1: 32..128 suggested by head_dim),
+ *     num_heads / num_kv_heads in {1, 2, 4, 8}.
  *     Anything else returns PA_ERR_UNSUPPORTED.
  *   - Validation: with PA_VALIDATE=1 in the environment (or
  *     pa_set_option(PA_OPT_VALIDATE, 1)) the calls first copy the index
@@ -340,6 +342,24 @@ pa_status pa_seq_fork(pa_allocator* alloc, const int32_t* parent_table, int num_
 
 /* Drop the sequence's reference on each of its blocks. */
 pa_status pa_seq_free(pa_allocator* alloc, const int32_t* table, int num_table_blocks);
+
+/*
+ * Compaction (periodic defragmentation, [tech] 2.1 and 4.2 item 2).  With
+ * fixed-size blocks a free block serves any request, so compaction packs the
+ * live blocks below `target_num_blocks` so the pool's tail can be released:
+ * every live block at or above the target (ascending id) moves to a free
+ * block below it (ascending id), its reference count travels with it, and
+ * the pool shrinks to the target (the free stack keeps its order).  The
+ * (src, dst) pairs go to moves[0 .. 2 * *num_moves); the caller then copies
+ * the data (pa_copy_blocks with those pairs, int64 on the device) and
+ * rewrites every table (pa_seq_remap).  OUT_OF_BLOCKS (nothing changes)
+ * when more blocks are live than the target holds.
+ */
+pa_status pa_alloc_compact(pa_allocator* alloc, int target_num_blocks, int32_t* moves,
+                           int capacity, int* num_moves);
+
+/* Replace every entry of a host table that is a move's src by its dst. */
+pa_status pa_seq_remap(int32_t* table, int num_table_blocks, const int32_t* moves, int num_moves);
 
 #ifdef __cplusplus
 }

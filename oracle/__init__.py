@@ -32,12 +32,12 @@ from .attention import (attention, paged_decode, split_partials, lse_merge,
                         paged_decode_split)
 from .cache_ops import reshape_and_cache, copy_blocks, swap_blocks
 from .allocator import (BlockAllocator, OutOfBlocks, append_slot, append_slots,
-                        extend, fork, free_sequence)
+                        extend, fork, free_sequence, compact, remap)
 
 __all__ = [
     "physical_slot", "gather_sequence", "block_bytes",
     "attention", "paged_decode", "split_partials", "lse_merge", "paged_decode_split",
     "reshape_and_cache", "copy_blocks", "swap_blocks",
     "BlockAllocator", "OutOfBlocks", "append_slot", "append_slots", "extend", "fork",
-    "free_sequence",
+    "free_sequence", "compact", "remap",
 ]

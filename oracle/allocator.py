@@ -14,10 +14,22 @@
 * Copy-on-write: a write into a block whose count exceeds one first copies it
   into a fresh block ([course] §2.4.3 pitfall note).
 
+* Compaction: periodic defragmentation ([tech] §2.1 "defragmentation only
+  moves block pointers", §4.2 item 2 "defragment every 1000 iterations").
+  With fixed-size blocks a free block always serves any request, so the
+  useful form is packing live blocks below a target so the pool's tail can
+  be released: the data of each moved block is copied (the caller runs the
+  copies) and every pointer to it -- table entries -- is rewritten.
+
 Readings where the pages are silent:
 * Free pool order: a stack.  It starts as ``initial_free_order`` (element 0
   handed out first); a reclaimed block is pushed on top (LIFO).
 * Out of blocks: the call raises ``OutOfBlocks`` and changes nothing.
+* Compaction moves the live blocks at or above the target, in ascending id,
+  into the free blocks below it, in ascending id; the pool then holds
+  exactly the target number of blocks and its free stack lists the remaining
+  free blocks in their previous stack order.  It raises ``OutOfBlocks`` (and
+  changes nothing) when more blocks are live than the target holds.
 * Batched appends process sequences in ascending index; when many sequences
   share one partial block, each but the last one to write copies it, and the
   last one (which then holds the only reference) writes in place.
@@ -154,3 +166,28 @@ def fork(alloc: BlockAllocator, parent_table: list) -> list:
 def free_sequence(alloc: BlockAllocator, table: list) -> None:
     for block in table:
         alloc.decref(block)
+
+
+def compact(alloc: BlockAllocator, target: int) -> list:
+    """Shrink the pool to ``target`` blocks; returns the (src, dst) moves."""
+    if target < 0 or target > alloc.num_blocks:
+        raise ValueError("target outside [0, num_blocks]")
+    live_high = [b for b in range(target, alloc.num_blocks) if alloc.ref[b] > 0]
+    free_low = sorted(b for b in alloc.free if b < target)
+    if len(live_high) > len(free_low):
+        raise OutOfBlocks()
+    moves = list(zip(live_high, free_low[:len(live_high)]))
+    taken = {dst for _, dst in moves}
+    for src, dst in moves:
+        alloc.ref[dst] = alloc.ref[src]
+        alloc.ref[src] = 0
+    alloc.free = [b for b in alloc.free if b < target and b not in taken]
+    alloc.ref = alloc.ref[:target]
+    alloc.num_blocks = target
+    return moves
+
+
+def remap(table: list, moves) -> list:
+    """The table with every moved block replaced by its destination."""
+    where = {src: dst for src, dst in moves}
+    return [where.get(b, b) for b in table]

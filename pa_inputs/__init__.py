@@ -139,19 +139,21 @@ def gqa_lengths(rng: np.random.Generator, num_seqs: int, median: float = 1024.0,
 
 
 def gqa(num_seqs: int = 256, extra_tokens: int = 0, cap: int = 8192,
-        headroom: float = 1.10) -> PagedProblem:
+        headroom: float = 1.10, block_size: int = 16, head_dim: int = 128) -> PagedProblem:
     """GQA decode batch.  ``extra_tokens`` reserves pool room for that many
     appended tokens per sequence (a decode loop grows every sequence by one
     token per step); the pool holds ``headroom`` times the blocks in use at
-    the end of such a loop."""
+    the end of such a loop.  The lengths do not depend on ``block_size`` or
+    ``head_dim`` (the block-size study varies those over one length mix)."""
     seed = SEED_BASE + 2
     rng = np.random.default_rng(seed)
     lengths = gqa_lengths(rng, num_seqs, cap=cap)
     final = lengths.astype(np.int64) + extra_tokens
-    in_use = int(sum(blocks_for(x, 16) for x in final))
+    in_use = int(sum(blocks_for(x, block_size) for x in final))
     nb = int(math.ceil(headroom * in_use))
-    max_blocks = blocks_for(cap + extra_tokens, 16)
-    return _problem("gqa", lengths, 32, 8, 128, 16, nb, "bf16", seed, max_blocks, rng)
+    max_blocks = blocks_for(cap + extra_tokens, block_size)
+    return _problem("gqa", lengths, 32, 8, head_dim, block_size, nb, "bf16", seed, max_blocks,
+                    rng)
 
 
 def long_context(lengths=(262144, 1048576)) -> PagedProblem:

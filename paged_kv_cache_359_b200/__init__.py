@@ -331,3 +331,19 @@ class BlockAllocator:
 
     def free(self, table: np.ndarray, num_table_blocks: int):
         self._check(lib().pa_seq_free(self._h, _i32(table), num_table_blocks))
+
+    def compact(self, target_num_blocks: int) -> np.ndarray:
+        """Pack live blocks below the target; returns int32 [n, 2] (src, dst)
+        moves (copy them with pa_copy_blocks, rewrite tables with remap)."""
+        moves = np.zeros((max(self.num_blocks, 1), 2), dtype=np.int32)
+        n = ctypes.c_int(0)
+        self._check(lib().pa_alloc_compact(self._h, int(target_num_blocks), _i32(moves),
+                                           self.num_blocks, ctypes.byref(n)))
+        self.num_blocks = int(target_num_blocks)
+        return moves[: n.value].copy()
+
+    @staticmethod
+    def remap(table: np.ndarray, num_table_blocks: int, moves: np.ndarray) -> None:
+        """Rewrite a host table in place after a compaction."""
+        moves = np.ascontiguousarray(moves, dtype=np.int32)
+        check(lib().pa_seq_remap(_i32(table), num_table_blocks, _i32(moves), moves.shape[0]))

@@ -74,6 +74,8 @@ SIGNATURES = {
     "pa_seq_extend": (_c_int, [_vp, _i32p, _c_int, _intp, _c_int, _i64p, _i32p, _i32p]),
     "pa_seq_fork": (_c_int, [_vp, _i32p, _c_int, _i32p]),
     "pa_seq_free": (_c_int, [_vp, _i32p, _c_int]),
+    "pa_alloc_compact": (_c_int, [_vp, _c_int, _i32p, _c_int, _intp]),
+    "pa_seq_remap": (_c_int, [_i32p, _c_int, _i32p, _c_int]),
 }
 
 

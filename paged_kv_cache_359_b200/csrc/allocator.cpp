@@ -9,6 +9,13 @@
 // (a new block only when the current one is full; copy-on-write when a
 // shared block is written).
 //
+// Compaction ("PagedAttention技术解析" 2.1: defragmentation moves block
+// pointers; 4.2 item 2: periodic defragmentation): with fixed-size blocks a
+// free block serves any request, so the useful form is packing the live
+// blocks below a target so the pool's tail can be released; the caller
+// copies the moved blocks' data (pa_copy_blocks) and rewrites its tables
+// (pa_seq_remap).
+//
 // Every operation is O(1) per block touched; failing calls change nothing.
 #include <cstdint>
 #include <cstring>
@@ -247,6 +254,56 @@ pa_status pa_seq_fork(pa_allocator* a, const int32_t* parent, int n, int32_t* ch
     for (int i = 0; i < n; ++i) {
         ++a->ref[parent[i]];
         child[i] = parent[i];
+    }
+    return PA_OK;
+}
+
+pa_status pa_alloc_compact(pa_allocator* a, int target, int32_t* moves, int capacity,
+                           int* num_moves) {
+    if (!a || !num_moves || target < 0 || target > a->num_blocks || capacity < 0 ||
+        (capacity > 0 && !moves))
+        return pa::fail(PA_ERR_INVALID_ARG, "bad compaction arguments");
+    std::vector<int32_t> high, low;
+    for (int32_t b = target; b < a->num_blocks; ++b)
+        if (a->ref[b] > 0) high.push_back(b);
+    for (int32_t b = 0; b < target; ++b)
+        if (a->ref[b] == 0) low.push_back(b);       // ascending id
+    if (high.size() > low.size())
+        return pa::fail(PA_ERR_OUT_OF_BLOCKS, "%zu live blocks above %d, %zu free below", high.size(),
+                        target, low.size());
+    if ((int)high.size() > capacity)
+        return pa::fail(PA_ERR_INVALID_ARG, "moves need %zu entries, capacity %d", high.size(),
+                        capacity);
+    std::vector<uint8_t> taken(target, 0);
+    for (size_t i = 0; i < high.size(); ++i) {
+        moves[2 * i] = high[i];
+        moves[2 * i + 1] = low[i];
+        a->ref[low[i]] = a->ref[high[i]];
+        a->ref[high[i]] = 0;
+        taken[low[i]] = 1;
+    }
+    // free stack keeps its order, minus blocks at or above the target and
+    // the destinations just taken
+    std::vector<int32_t> stack;
+    stack.reserve(a->stack.size());
+    for (int32_t b : a->stack)
+        if (b < target && !taken[b]) stack.push_back(b);
+    a->stack.swap(stack);
+    a->ref.resize(target);
+    a->num_blocks = target;
+    *num_moves = (int)high.size();
+    return PA_OK;
+}
+
+pa_status pa_seq_remap(int32_t* table, int n, const int32_t* moves, int num_moves) {
+    if (n < 0 || num_moves < 0 || (n > 0 && !table) || (num_moves > 0 && !moves))
+        return pa::fail(PA_ERR_INVALID_ARG, "null argument");
+    std::unordered_map<int32_t, int32_t> where;
+    where.reserve((size_t)num_moves * 2);
+    for (int i = 0; i < num_moves; ++i) where[moves[2 * i]] = moves[2 * i + 1];
+    for (int i = 0; i < n; ++i) {
+        auto it = where.find(table[i]);
+        if (it != where.end()) table[i] = it->second;
     }
     return PA_OK;
 }

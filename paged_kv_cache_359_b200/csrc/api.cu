@@ -53,8 +53,9 @@ pa_status check_geometry(pa_dtype dt, int head_dim, int block_size) {
         return fail(PA_ERR_UNSUPPORTED, "dtype %d not supported", (int)dt);
     if (head_dim != 64 && head_dim != 128 && head_dim != 256)
         return fail(PA_ERR_UNSUPPORTED, "head_dim %d not built (64, 128, 256)", head_dim);
-    if (block_size != 8 && block_size != 16 && block_size != 32)
-        return fail(PA_ERR_UNSUPPORTED, "block_size %d not built (8, 16, 32)", block_size);
+    if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
+        block_size != 128)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d not built (8, 16, 32, 64, 128)", block_size);
     return PA_OK;
 }
 

@@ -146,6 +146,8 @@ pa_status launch_decode_td(const DecodeLaunch& l) {
         case 8: return launch_decode_bs<T, D, 8>(l);
         case 16: return launch_decode_bs<T, D, 16>(l);
         case 32: return launch_decode_bs<T, D, 32>(l);
+        case 64: return launch_decode_bs<T, D, 64>(l);
+        case 128: return launch_decode_bs<T, D, 128>(l);
         default: return fail(PA_ERR_UNSUPPORTED, "block_size %d not built", l.block_size);
     }
 }

@@ -55,7 +55,7 @@ def _decode(**over):
 @pytest.mark.parametrize("over,status", [
     (dict(hq=6, hk=4), 1),          # heads not a multiple of kv heads
     (dict(d=96), 2),                # head_dim not built
-    (dict(bs=64), 2),               # block size not built
+    (dict(bs=24), 2),               # block size not built
     (dict(hq=48, hk=2), 2),         # group size 24 not built
     (dict(out=0), 1),               # null pointer
     (dict(q=8), 1),                 # misaligned

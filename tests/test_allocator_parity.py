@@ -143,3 +143,48 @@ def test_random_operation_sequences(seed):
         same_state(c, o)
         for t, ot, ln in zip(ctabs, otabs, lens):
             assert list(t[: -(-ln // bs)]) == ot
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_compaction_matches_the_oracle(seed):
+    rng = random.Random(900 + seed)
+    bs, nb, cap = 8, 120, 20
+    order = list(range(nb))
+    rng.shuffle(order)
+    c, o = BlockAllocator(nb, bs, order), oracle.BlockAllocator(nb, bs, order)
+    ctabs, otabs, lens = [], [], []
+    for _ in range(10):
+        k = rng.randint(1, 6 * bs)
+        t = np.full(cap, -1, dtype=np.int32)
+        ot = []
+        c.extend(t, 0, k)
+        oracle.extend(o, ot, 0, k)
+        ctabs.append(t); otabs.append(ot); lens.append(k)
+    for i in (0, 3):
+        t = np.full(cap, -1, dtype=np.int32)
+        c.fork(ctabs[i], -(-lens[i] // bs), t)
+        ctabs.append(t); otabs.append(oracle.fork(o, otabs[i])); lens.append(lens[i])
+    for i in (2, 5, 7):
+        c.free(ctabs[i], -(-lens[i] // bs))
+        oracle.free_sequence(o, otabs[i])
+    keep = [i for i in range(len(ctabs)) if i not in (2, 5, 7)]
+    live = sum(1 for r in o.ref if r > 0)
+    target = live + rng.randint(0, 3)
+    cm = c.compact(target)
+    om = oracle.compact(o, target)
+    assert [tuple(m) for m in cm.tolist()] == om
+    for i in keep:
+        n = -(-lens[i] // bs)
+        BlockAllocator.remap(ctabs[i], n, cm)
+        assert list(ctabs[i][:n]) == oracle.remap(otabs[i], om)
+    assert c.free_order() == o.free_order()
+    assert c.ref_counts() == o.ref
+    # below the live count: refused, nothing changes
+    before = (c.free_order(), c.ref_counts())
+    with pytest.raises(OutOfBlocks):
+        c.compact(live - 1)
+    assert (c.free_order(), c.ref_counts()) == before and c.num_blocks == target
+    # remap leaves entries that are not a source alone
+    t = np.array([0, 5, 7], dtype=np.int32)
+    BlockAllocator.remap(t, 3, np.array([[7, 2], [9, 1]], dtype=np.int32))
+    assert list(t) == [0, 5, 2]

@@ -46,7 +46,7 @@ def test_tiny_decode_append_decode():
 
 
 COMBOS = [(dt, d, bs, g) for dt in ("bf16", "f32") for d in (64, 128, 256)
-          for bs in (8, 16, 32) for g in (1, 2, 4, 8)]
+          for bs in (8, 16, 32, 64, 128) for g in (1, 2, 4, 8)]
 
 
 @pytest.mark.parametrize("dtype,d,bs,g", COMBOS)

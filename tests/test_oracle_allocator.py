@@ -178,3 +178,52 @@ def test_random_operation_sequences_keep_invariants(seed):
         check_invariants(alloc, seqs)
         for t, length in zip(seqs, lens):
             assert len(t) == -(-length // bs)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_compaction_packs_live_blocks_below_the_target(seed):
+    """After compaction every table points below the target, every moved
+    block's count travelled with it, the pool invariants hold at the new
+    size, and the moves are distinct high sources onto distinct free low
+    destinations."""
+    rng = random.Random(500 + seed)
+    bs = rng.choice([4, 8])
+    nb = 96
+    order = list(range(nb))
+    rng.shuffle(order)
+    alloc = oracle.BlockAllocator(nb, bs, order)
+    seqs, lens = [], []
+    for _ in range(8):
+        t, length = [], 0
+        _, _, length = oracle.extend(alloc, t, 0, rng.randint(1, 5 * bs))
+        seqs.append(t)
+        lens.append(length)
+    for i in range(3):
+        seqs.append(oracle.fork(alloc, seqs[i]))
+        lens.append(lens[i])
+    for i in (1, 4):
+        oracle.free_sequence(alloc, seqs[i])
+    seqs = [t for i, t in enumerate(seqs) if i not in (1, 4)]
+    live = sum(1 for r in alloc.ref if r > 0)
+    counts = {b: alloc.ref[b] for b in range(nb) if alloc.ref[b] > 0}
+    target = live + rng.randint(0, 5)
+    moves = oracle.compact(alloc, target)
+    assert len({s for s, _ in moves}) == len(moves) == len({d for _, d in moves})
+    assert all(s >= target > d for s, d in moves)
+    seqs = [oracle.remap(t, moves) for t in seqs]
+    assert all(b < target for t in seqs for b in t)
+    where = dict(moves)
+    for b, c in counts.items():
+        assert alloc.ref[where.get(b, b)] == c
+    assert alloc.num_blocks == target
+    check_invariants(alloc, seqs)
+
+
+def test_compaction_beyond_the_live_blocks_changes_nothing():
+    alloc = oracle.BlockAllocator(10, 4)
+    t = []
+    oracle.extend(alloc, t, 0, 24)                     # 6 live blocks
+    before = (alloc.free_order(), list(alloc.ref))
+    with pytest.raises(oracle.OutOfBlocks):
+        oracle.compact(alloc, 5)
+    assert (alloc.free_order(), list(alloc.ref)) == before
