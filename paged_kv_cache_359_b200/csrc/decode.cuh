@@ -8,13 +8,14 @@
 //
 // How (B200 design, not the pages' A100 sketch):
 //  * Work item = (sequence, kv head): all G query heads of the kv group share
-//    every K/V tile the CTA loads.  pa_decode runs a persistent grid (about
-//    two CTAs per SM); every CTA sorts the context lengths in shared memory
-//    and takes items in snake order over the longest-first list, so long
-//    sequences start first and the CTAs finish together.  With few items a
-//    cluster of CTAs shares one item instead and merges through distributed
-//    shared memory; pa_decode_split gives every fixed token partition its
-//    own CTA and merges partitions with a log-sum-exp reduce kernel.
+//    every K/V tile the CTA loads.  pa_decode launches one CTA per item and
+//    CTA b finds, by a warp search over the context lengths, the item at
+//    position b of the longest-first list, so the hardware block scheduler
+//    starts the long sequences first and back-fills SMs with short ones.
+//    With few items a cluster of CTAs shares one item instead and merges
+//    through distributed shared memory; pa_decode_split gives every fixed
+//    token partition its own CTA and merges partitions with a log-sum-exp
+//    reduce kernel.
 //  * Unit = R consecutive tokens of one block for one kv head: a K tile and
 //    a V tile, each loaded by 4-D TMA boxes over the cache viewed as
 //    [num_blocks][block_size][kv_heads][head_dim].
@@ -529,9 +530,12 @@ using UnitFor = typename std::conditional<(std::is_same<T, __nv_bfloat16>::value
 // ---------------------------------------------------- kernel geometry ----
 template <class U>
 struct Layout {
-    static constexpr int NW = 4;                                   // warps per CTA
     static constexpr int UNIT_BYTES = U::R * U::D * (int)sizeof(typename U::T);
     static constexpr int STAGE_BYTES = 2 * UNIT_BYTES;
+    // warps per CTA: four, or two when a stage is 16 KiB (head_dim 256 on
+    // the tensor-core unit), so that three CTAs still fit an SM with a
+    // two-stage ring per warp (about 192 KiB of loads in flight per SM)
+    static constexpr int NW = STAGE_BYTES >= 16384 ? 2 : 4;
     static constexpr int DEPTH = cmin(8, cmax(2, 16384 / STAGE_BYTES));
     static constexpr int STAGE_REGION = NW * DEPTH * STAGE_BYTES;
     // warps merge in the drained ring: [NW][G] max, [NW][G] sum,
