@@ -114,6 +114,46 @@ __device__ __forceinline__ int shared_prefix_of(const DecodeArgs& a, int seq) {
     return __ldg(a.group_prefix + lo);
 }
 
+// Warp-wide selection: lane l holds values get(0..PL-1) of entries l, l+32,
+// ... (-1 for no entry, else >= 0).  Returns the entry at rank r of the list
+// sorted by (value descending, entry ascending), and its value in `value`:
+// a binary search for the value v at rank r (counts by warp reduction), then
+// the k-th entry equal to v in entry order by ballots.  r must be below the
+// number of entries.
+template <int PL, class Get>
+__device__ __forceinline__ int rank_select(Get&& get, int r, int lane, int& value) {
+    int top = 0;
+#pragma unroll
+    for (int j = 0; j < PL; ++j) top = max(top, get(j));
+    top = (int)__reduce_max_sync(FULL_MASK, (unsigned)top);
+    int lo = 0, hi = top + 1;            // count(v >= lo) > r >= count(v >= hi)
+    while (hi - lo > 1) {
+        const int mid = lo + (hi - lo) / 2;
+        int cnt = 0;
+#pragma unroll
+        for (int j = 0; j < PL; ++j) cnt += get(j) >= mid;
+        if ((int)__reduce_add_sync(FULL_MASK, (unsigned)cnt) > r)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int j = 0; j < PL; ++j) gt += get(j) > lo;
+    const int k = r - (int)__reduce_add_sync(FULL_MASK, (unsigned)gt);
+    int base = 0, found = -1;
+#pragma unroll
+    for (int j = 0; j < PL; ++j) {
+        const bool eq = get(j) == lo;
+        const unsigned ball = __ballot_sync(FULL_MASK, eq);
+        const int before = __popc(ball & ((1u << lane) - 1u));
+        if (eq && base + before == k) found = lane + 32 * j;
+        base += __popc(ball);
+    }
+    value = lo;
+    return (int)__reduce_max_sync(FULL_MASK, (unsigned)(found + 1)) - 1;
+}
+
 // Fused append: the CTA of (seq, kvh) writes kv head kvh's part of the new
 // token's key and value rows into the cache, then makes the writes visible
 // to its own TMA loads.  Only this sequence reads the new token's block (a
@@ -536,7 +576,10 @@ struct Layout {
     // the tensor-core unit), so that three CTAs still fit an SM with a
     // two-stage ring per warp (about 192 KiB of loads in flight per SM)
     static constexpr int NW = STAGE_BYTES >= 16384 ? 2 : 4;
-    static constexpr int DEPTH = cmin(8, cmax(2, 16384 / STAGE_BYTES));
+    // stages per warp: about 12 KiB of ring per warp, at least two; with
+    // 4 KiB stages (head_dim 64) the smaller CTA lets four CTAs share an SM,
+    // which hides the per-CTA prologue and merge of these short items better
+    static constexpr int DEPTH = cmin(8, cmax(2, 12288 / STAGE_BYTES));
     static constexpr int STAGE_REGION = NW * DEPTH * STAGE_BYTES;
     // warps merge in the drained ring: [NW][G] max, [NW][G] sum,
     // [NW][G][D] output, then the cluster exchange [G], [G], [G][D]
@@ -819,69 +862,55 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
 
         if (a.sched == SCHED_LPT) {
             // Which sequence sits at rank r = blockIdx.x / Hk of the list sorted
-            // by (length descending, index ascending)?  Warp 0 binary-searches
-            // the length value v at rank r (counts by warp reduction), then
-            // picks the k-th sequence of length v in index order by ballots.
+            // by (tokens this pass reads descending, index ascending)?  Warp 0
+            // selects it (rank_select); up to 256 sequences it holds the
+            // lengths in registers and the other warps go straight to the
+            // barrier, above that the CTA stages them in shared memory.
             const int S = a.num_seqs, Hk = a.num_kv_heads;
             const int r = blockIdx.x / Hk;
-            int* pick = reinterpret_cast<int*>(smem + Ly::ORDER_OFFSET);
-            int* lens = pick + 1;                            // S lengths (S <= MAX_SORT)
-            if (S <= MAX_SORT)
-                for (int i = threadIdx.x; i < S; i += NT) {
-                    const int x = a.context_lens[i];
-                    if (x < 0 || x > a.max_tokens) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
-                    const int len = x < 0 ? 0 : (x > a.max_tokens ? a.max_tokens : x);
-                    // order by the tokens this pass reads (own tokens with a shared prefix)
-                    lens[i] = len - cmin(shared_prefix_of(a, i), len);
-                }
-            __syncthreads();
+            int* pick = reinterpret_cast<int*>(smem + Ly::ORDER_OFFSET);   // sequence, its tokens
+            int* lens = pick + 2;                                           // S <= MAX_SORT
+            auto own_tokens = [&](int i) {
+                const int x = a.context_lens[i];
+                if (x < 0 || x > a.max_tokens) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
+                const int len = x < 0 ? 0 : (x > a.max_tokens ? a.max_tokens : x);
+                // order by the tokens this pass reads (own tokens with a shared prefix)
+                return len - cmin(shared_prefix_of(a, i), len);
+            };
+            constexpr int REG_PER_LANE = 8;
+            const bool in_regs = S <= 32 * REG_PER_LANE;
+            if (!in_regs && S <= MAX_SORT) {
+                for (int i = threadIdx.x; i < S; i += NT) lens[i] = own_tokens(i);
+                __syncthreads();
+            }
             if (warp == 0) {
-                int found = r;                               // natural order beyond MAX_SORT
-                if (S <= MAX_SORT) {
-                    const int per_lane = (S + 31) / 32;
-                    int top = 0;
-                    for (int j = 0; j < per_lane; ++j) {
+                int found = r, tokens = -1;                  // natural order beyond MAX_SORT
+                if (in_regs) {
+                    int v[REG_PER_LANE];
+#pragma unroll
+                    for (int j = 0; j < REG_PER_LANE; ++j) {
                         const int i = lane + 32 * j;
-                        if (i < S) top = max(top, lens[i]);
+                        v[j] = i < S ? own_tokens(i) : -1;
                     }
-                    top = (int)__reduce_max_sync(FULL_MASK, (unsigned)top);
-                    int lo = 0, hi = top + 1;        // count(len >= lo) > r >= count(len >= hi)
-                    while (hi - lo > 1) {
-                        const int mid = lo + (hi - lo) / 2;
-                        int cnt = 0;
-                        for (int j = 0; j < per_lane; ++j) {
+                    found = rank_select<REG_PER_LANE>([&](int j) { return v[j]; }, r, lane,
+                                                      tokens);
+                } else if (S <= MAX_SORT) {
+                    found = rank_select<MAX_SORT / 32>(
+                        [&](int j) {
                             const int i = lane + 32 * j;
-                            cnt += i < S && lens[i] >= mid;
-                        }
-                        if ((int)__reduce_add_sync(FULL_MASK, (unsigned)cnt) > r)
-                            lo = mid;
-                        else
-                            hi = mid;
-                    }
-                    int gt = 0;
-                    for (int j = 0; j < per_lane; ++j) {
-                        const int i = lane + 32 * j;
-                        gt += i < S && lens[i] > lo;
-                    }
-                    const int k = r - (int)__reduce_add_sync(FULL_MASK, (unsigned)gt);
-                    int base = 0;
-                    found = -1;
-                    for (int j = 0; j < per_lane; ++j) {
-                        const int i = lane + 32 * j;
-                        const bool eq = i < S && lens[i] == lo;
-                        const unsigned ball = __ballot_sync(FULL_MASK, eq);
-                        const int before = __popc(ball & ((1u << lane) - 1u));
-                        if (eq && base + before == k) found = i;
-                        base += __popc(ball);
-                    }
-                    found = (int)__reduce_max_sync(FULL_MASK, (unsigned)(found + 1)) - 1;
+                            return i < S ? lens[i] : -1;
+                        },
+                        r, lane, tokens);
                 }
-                if (lane == 0) *pick = found;
+                if (lane == 0) {
+                    pick[0] = found;
+                    pick[1] = tokens;
+                }
             }
             __syncthreads();
-            seq = *pick;
+            seq = pick[0];
             kvh = blockIdx.x % Hk;
-            L = S <= MAX_SORT && !a.group_starts ? lens[seq] : clamp_len(seq);
+            L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
             const int tok0 = cmin(shared_prefix_of(a, seq), L);    // whole 16-token units
             if (a.new_slots) {
                 append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);

@@ -179,3 +179,18 @@ def test_longest_first_order_with_length_ties():
     data = pa_inputs.materialize(problem, "cuda")
     assert_close(run_decode(data, problem), oracle_decode(data, problem))
     device_clean()
+
+
+@pytest.mark.parametrize("num_seqs", [255, 256, 257, 600, 1024])
+def test_longest_first_order_around_the_register_and_shared_ranges(num_seqs):
+    """The rank search holds up to 256 lengths in registers and stages up to
+    1024 in shared memory: batches on both sides of each limit, with repeated
+    lengths, decode every sequence exactly once."""
+    fixed = {i: 41 for i in range(0, num_seqs, 5)}
+    problem = pa_inputs.random_small(900 + num_seqs, num_seqs=num_seqs, max_len=120,
+                                     num_heads=8, num_kv_heads=2, head_dim=64, block_size=16,
+                                     dtype="bf16", zero_len=True, fixed=fixed)
+    data = pa_inputs.materialize(problem, "cuda")
+    out = torch.full_like(data["q"], float("nan"))
+    assert_close(run_decode(data, problem, out=out), oracle_decode(data, problem))
+    device_clean()
