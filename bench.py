@@ -762,6 +762,7 @@ def workload_config(p, args):
                 -(-int(x) // p.block_size) * p.block_size for x in lens)), 5),
             "kernel": args.kernel + ("+append (fused)" if args.fused else ""),
             "partition": args.partition,
+            "pdl": not getattr(args, "no_pdl", False),
             "l2": "inputs larger than L2 (KV cache %.2f GB vs 126 MB L2), no flush" %
                   (decode_kv_bytes(lens, p) / 1e9)}
 
@@ -785,6 +786,8 @@ def main():
                     help="gqa workload: block size (default 16; the block-size study)")
     ap.add_argument("--head-dim", type=int, default=None,
                     help="gqa workload: head_dim (default 128)")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch (PA_OPT_PDL 0)")
     ap.add_argument("--compact", action="store_true",
                     help="after the timed loop: free half the batch, compact the pool, report")
     ap.add_argument("--ref-sample", type=int, default=64,
@@ -821,6 +824,8 @@ def main():
         raise SystemExit("bench.py needs a CUDA GPU (no CPU fallback)")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    import paged_kv_cache_359_b200 as pa
+    pa.pa_set_option("pdl", 0 if args.no_pdl else 1)
     dist_init(world, "nccl")
     try:
         extra = 2 * (args.steps + args.warmup) + 4

@@ -78,7 +78,12 @@ enum {
 
 typedef enum pa_option {
     PA_OPT_VALIDATE = 0,         /* 0/1: host-side index validation before launch */
-    PA_OPT_DECODE_SPLIT_CTAS = 1  /* pa_decode CTAs per (sequence, kv head): 0 = auto, 1, 2, 4, 8 */
+    PA_OPT_DECODE_SPLIT_CTAS = 1, /* pa_decode CTAs per (sequence, kv head): 0 = auto, 1, 2, 4, 8 */
+    PA_OPT_PDL = 2                /* 0/1 (default 1, or PA_PDL in the environment): launch with
+                                     programmatic dependent launch.  Every kernel still waits
+                                     for the grid before it on the stream to complete before
+                                     touching memory; only the launch and the CTA placement
+                                     overlap that grid's tail */
 } pa_option;
 
 const char* pa_last_error(void);

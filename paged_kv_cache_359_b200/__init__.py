@@ -29,7 +29,7 @@ import numpy as np
 import torch
 
 from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SPLIT_CTAS,
-                      PA_OPT_VALIDATE, PagedAttnError, check, lib)
+                      PA_OPT_PDL, PA_OPT_VALIDATE, PagedAttnError, check, lib)
 
 __all__ = [
     "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_split", "pa_decode_split_workspace_bytes",
@@ -40,7 +40,8 @@ __all__ = [
 ]
 
 _DTYPES = {torch.float32: PA_DTYPE_F32, torch.bfloat16: PA_DTYPE_BF16}
-_OPTIONS = {"validate": PA_OPT_VALIDATE, "decode_split_ctas": PA_OPT_DECODE_SPLIT_CTAS}
+_OPTIONS = {"validate": PA_OPT_VALIDATE, "decode_split_ctas": PA_OPT_DECODE_SPLIT_CTAS,
+            "pdl": PA_OPT_PDL}
 
 
 class OutOfBlocks(PagedAttnError):

@@ -17,7 +17,7 @@ STATUS_NAMES = {
     4: "PA_ERR_BAD_BLOCK_ID", 5: "PA_ERR_CUDA", 6: "PA_ERR_DEVICE_CHECK",
 }
 PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
-PA_OPT_VALIDATE, PA_OPT_DECODE_SPLIT_CTAS = 0, 1
+PA_OPT_VALIDATE, PA_OPT_DECODE_SPLIT_CTAS, PA_OPT_PDL = 0, 1, 2
 
 DEVERR_BITS = {
     1: "PA_DEVERR_BLOCK_ID", 2: "PA_DEVERR_CONTEXT_LEN", 4: "PA_DEVERR_WAIT_TIMEOUT",

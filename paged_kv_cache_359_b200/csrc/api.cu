@@ -21,6 +21,7 @@ namespace {
 thread_local std::string g_last_error;
 int g_validate = -1;                 // -1: read PA_VALIDATE on first use
 int g_decode_ctas = 0;               // 0: automatic
+int g_pdl = -1;                      // -1: read PA_PDL on first use (default on)
 
 bool validate_enabled() {
     if (g_validate < 0) {
@@ -145,6 +146,21 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
 
+bool pdl_enabled() {
+    if (g_pdl < 0) {
+        const char* v = std::getenv("PA_PDL");
+        g_pdl = (v && v[0] == '0') ? 0 : 1;
+    }
+    return g_pdl == 1;
+}
+
+void add_pdl_attr(cudaLaunchAttribute* attrs, unsigned* n) {
+    if (!pdl_enabled()) return;
+    attrs[*n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[*n].val.programmaticStreamSerializationAllowed = 1;
+    ++*n;
+}
+
 pa_status fail(pa_status status, const char* fmt, ...) {
     char buf[512];
     va_list ap;
@@ -204,6 +220,7 @@ int pa_version(void) { return 1; }
 pa_status pa_set_option(pa_option option, int value) {
     switch (option) {
         case PA_OPT_VALIDATE: g_validate = value ? 1 : 0; return PA_OK;
+        case PA_OPT_PDL: g_pdl = value ? 1 : 0; return PA_OK;
         case PA_OPT_DECODE_SPLIT_CTAS:
             if (value != 0 && value != 1 && value != 2 && value != 4 && value != 8)
                 return fail(PA_ERR_INVALID_ARG, "CTAs per (sequence, kv head) must be 0,1,2,4,8");
@@ -217,6 +234,7 @@ int pa_get_option(pa_option option) {
     switch (option) {
         case PA_OPT_VALIDATE: return validate_enabled() ? 1 : 0;
         case PA_OPT_DECODE_SPLIT_CTAS: return g_decode_ctas;
+        case PA_OPT_PDL: return pdl_enabled() ? 1 : 0;
     }
     return -1;
 }

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(128)
                              uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                              const int64_t* __restrict__ slots, int num_tokens, int row_vecs,
                              int64_t num_slots, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     for (int t = blockIdx.x; t < num_tokens; t += gridDim.x) {
         const int64_t s = slots[t];
         if (s < 0) continue;
@@ -52,6 +54,8 @@ __global__ void __launch_bounds__(256)
                        const uint4* __restrict__ src_k, const uint4* __restrict__ src_v,
                        const int64_t* __restrict__ mapping, int64_t block_vecs, int src_blocks,
                        int dst_blocks, unsigned err_bits, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int pair = blockIdx.x;
     const int64_t src = mapping[2 * pair], dst = mapping[2 * pair + 1];
     if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
@@ -102,11 +106,17 @@ pa_status launch_reshape_and_cache(const void* key, const void* value, void* k_c
     unsigned* err = device_error_word();
     if (!err) return fail(PA_ERR_CUDA, "device error word unavailable");
     const int grid = num_tokens < 8 * num_sms() ? num_tokens : 8 * num_sms();
-    reshape_and_cache_kernel<<<grid, 128, 0, stream>>>(
-        static_cast<const uint4*>(key), static_cast<const uint4*>(value),
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slots, num_tokens,
-        (int)(row_bytes / 16), num_slots, err);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(128);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    add_pdl_attr(attr, &cfg.numAttrs);
+    cudaError_t e = cudaLaunchKernelEx(
+        &cfg, reshape_and_cache_kernel, static_cast<const uint4*>(key),
+        static_cast<const uint4*>(value), static_cast<uint4*>(k_cache),
+        static_cast<uint4*>(v_cache), slots, num_tokens, (int)(row_bytes / 16), num_slots, err);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reshape_and_cache launch: %s", cudaGetErrorString(e));
     return PA_OK;
 }
@@ -121,10 +131,17 @@ pa_status launch_move_blocks(void* dst_k, void* dst_v, const void* src_k, const 
     const int64_t vecs = block_bytes / 16;
     int chunks = (int)(vecs / 1024);
     chunks = chunks < 1 ? 1 : (chunks > 32 ? 32 : chunks);
-    move_blocks_kernel<<<dim3(num_pairs, chunks), 256, 0, stream>>>(
-        static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), static_cast<const uint4*>(src_k),
-        static_cast<const uint4*>(src_v), mapping, vecs, src_blocks, dst_blocks, err_bits, err);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_pairs, chunks);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    add_pdl_attr(attr, &cfg.numAttrs);
+    cudaError_t e = cudaLaunchKernelEx(
+        &cfg, move_blocks_kernel, static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v),
+        static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v), mapping, vecs,
+        src_blocks, dst_blocks, err_bits, err);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "block move launch: %s", cudaGetErrorString(e));
     return PA_OK;
 }

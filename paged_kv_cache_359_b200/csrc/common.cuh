@@ -180,6 +180,18 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Programmatic dependent launch.  Every kernel of the library starts with
+// pdl_wait(): it returns once the grid launched before it on the stream has
+// completed and its writes are visible (at once when the kernel was launched
+// without the attribute), so the stream's order is kept exactly; what
+// overlaps is only the launch and CTA placement of this grid with the tail
+// of the previous one.  pdl_launch_dependents() then lets the next grid be
+// launched, whose CTAs take SM slots as this grid's CTAs retire.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (TMA) accesses to the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {

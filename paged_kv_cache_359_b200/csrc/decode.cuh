@@ -736,6 +736,8 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
     using Ly = Layout<U>;
     constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
     constexpr int NT = NW * 32;
+    pdl_wait();
+    pdl_launch_dependents();
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -1001,6 +1003,8 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
 // w, w+8, ...; lane = one of 32 dimensions.
 template <typename T, int D>
 __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int sh = blockIdx.x;
     const int seq = sh / a.num_heads;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;

@@ -35,6 +35,11 @@ unsigned* device_error_word();
 // SM count of the current device.
 int num_sms();
 
+// PA_OPT_PDL: launch with programmatic stream serialisation.  Appends the
+// attribute to attrs[*n] when enabled.
+bool pdl_enabled();
+void add_pdl_attr(cudaLaunchAttribute* attrs, unsigned* n);
+
 // Everything a decode launch needs besides the template parameters.
 struct DecodeLaunch;
 

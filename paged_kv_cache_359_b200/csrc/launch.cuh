@@ -61,7 +61,9 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
         return fail(PA_ERR_INVALID_ARG, "partition must be a multiple of %d tokens", U::R);
 
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    cfg.attrs = attr;
+    add_pdl_attr(attr, &cfg.numAttrs);
     cfg.blockDim = dim3(Ly::NW * 32);
     cfg.dynamicSmemBytes = Ly::SMEM_BYTES;
     cfg.stream = l.stream;
@@ -87,6 +89,9 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
                 pc.blockDim = dim3((l.consumers + 1) * 32);
                 pc.dynamicSmemBytes = C::SMEM_BYTES;
                 pc.stream = l.stream;
+                cudaLaunchAttribute pattr[1];
+                pc.attrs = pattr;
+                add_pdl_attr(pattr, &pc.numAttrs);
                 e = cudaLaunchKernelEx(&pc, pk, sk, sv, l.args, l.row_blocks);
                 if (e != cudaSuccess)
                     return fail(PA_ERR_CUDA, "shared-prefix launch: %s", cudaGetErrorString(e));
@@ -102,9 +107,14 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
         cfg.gridDim = dim3(l.args.max_parts, l.num_kv_heads, l.num_seqs);
         e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
         if (e == cudaSuccess) {
-            lse_reduce_kernel<T, D><<<dim3(l.num_seqs * l.args.num_heads, D / 32), 256, 0,
-                                      l.stream>>>(l.args);
-            e = cudaGetLastError();
+            cudaLaunchConfig_t rc = {};
+            rc.gridDim = dim3(l.num_seqs * l.args.num_heads, D / 32);
+            rc.blockDim = dim3(256);
+            rc.stream = l.stream;
+            cudaLaunchAttribute rattr[1];
+            rc.attrs = rattr;
+            add_pdl_attr(rattr, &rc.numAttrs);
+            e = cudaLaunchKernelEx(&rc, lse_reduce_kernel<T, D>, l.args);
         }
     } else {
         static std::atomic<unsigned long long> done{0};
@@ -115,12 +125,11 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
         } else {
             cfg.gridDim = dim3(l.ctas, l.num_kv_heads, l.num_seqs);
             if (l.ctas > 1) {
-                attr[0].id = cudaLaunchAttributeClusterDimension;
-                attr[0].val.clusterDim.x = l.ctas;
-                attr[0].val.clusterDim.y = 1;
-                attr[0].val.clusterDim.z = 1;
-                cfg.attrs = attr;
-                cfg.numAttrs = 1;
+                cudaLaunchAttribute& c = attr[cfg.numAttrs++];
+                c.id = cudaLaunchAttributeClusterDimension;
+                c.val.clusterDim.x = l.ctas;
+                c.val.clusterDim.y = 1;
+                c.val.clusterDim.z = 1;
             }
         }
         e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);

@@ -57,6 +57,8 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS)
     shared_prefix_kernel(const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a,
                          int row_blocks) {
+    pdl_wait();
+    pdl_launch_dependents();
     using C = PrefixCfg<D, BS, G>;
     constexpr int R = C::R, STAGES = C::STAGES, KS = C::KS, NT = C::NT;
     const int chunk = blockIdx.x, kvh = blockIdx.y;
