@@ -262,12 +262,16 @@ def decode_kv_bytes(lens: np.ndarray, problem) -> int:
         problem.elem_bytes
 
 
-def decode_alg_bytes(lens: np.ndarray, problem) -> int:
-    """K/V rows read + q read + out written + block-table entries + lengths."""
+def decode_alg_bytes(lens: np.ndarray, problem, fused: bool = False) -> int:
+    """K/V rows read + q read + out written + block-table entries + lengths;
+    fused: + the new key/value rows read and written into the cache + slots."""
     s = len(lens)
     qo = 2 * s * problem.num_heads * problem.head_dim * problem.elem_bytes
     tab = 4 * int(sum(-(-int(x) // problem.block_size) for x in lens)) + 4 * s
-    return decode_kv_bytes(lens, problem) + qo + tab
+    extra = 0
+    if fused:
+        extra = 2 * 2 * s * problem.num_kv_heads * problem.head_dim * problem.elem_bytes + 8 * s
+    return decode_kv_bytes(lens, problem) + qo + tab + extra
 
 
 def kernel_hash() -> str:
@@ -439,7 +443,7 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
     timed_lens = lens[warmup:]
     kv = sum(decode_kv_bytes(x, p) for x in timed_lens)
-    alg = [decode_alg_bytes(x, p) for x in timed_lens]
+    alg = [decode_alg_bytes(x, p, loop.fused) for x in timed_lens]
     launches = sum(loop.launches_per_step(len(c)) for c in cows[warmup:])
     uniq = (sum(unique_kv_bytes(t, l, p) for t, l in zip(tabs[warmup:], timed_lens))
             if unique else None)
@@ -778,8 +782,9 @@ def main():
     ap.add_argument("--workload", choices=["gqa", "mha", "long", "prefix"], default="gqa")
     ap.add_argument("--kernel", choices=["decode", "split", "cascade"], default=None)
     ap.add_argument("--partition", type=int, default=512)
-    ap.add_argument("--fused", action="store_true",
-                    help="pa_decode_append: the cache write fused into the decode launch")
+    ap.add_argument("--unfused", action="store_true",
+                    help="decode kernel: pa_reshape_and_cache then pa_decode (two launches) "
+                         "instead of pa_decode_append (the cache write fused into the decode)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block-size", type=int, default=None,
@@ -797,8 +802,10 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.kernel is None:
         args.kernel = "split" if args.workload == "long" else "decode"
-    if args.fused and args.kernel != "decode":
-        ap.error("--fused fuses the cache write into pa_decode (not the split kernel)")
+    if args.unfused and args.kernel != "decode":
+        ap.error("--unfused applies to the decode kernel (split and cascade write separately)")
+    # the decode kernel's step is the fused append + decode unless asked otherwise
+    args.fused = args.kernel == "decode" and not args.unfused
     if args.compact and args.workload not in ("gqa", "mha"):
         ap.error("--compact runs on the gqa and mha workloads")
     if (args.block_size or args.head_dim) and args.workload != "gqa":
@@ -850,7 +857,7 @@ def main():
         achieved = dec_alg / (dec_mean_ms / 1e3) / 1e9
         peak, peak_src = hbm_peak()
         # the committed capture is of the default gqa decode launch
-        default_shape = (args.workload == "gqa" and args.kernel == "decode" and not args.fused
+        default_shape = (args.workload == "gqa" and args.kernel == "decode" and args.fused
                          and args.block_size in (None, 16) and args.head_dim in (None, 128))
         cap = measured_traffic() if default_shape else None
         # scaled from the captured launch to this run's mean launch by
