@@ -206,6 +206,7 @@ struct CoreUnit {
     static constexpr int DUP = LPR >> RS;
     static constexpr int BOX_INNER = D;
     static constexpr int BOXES = 1;
+    static constexpr int BOX_ROWS = R;            // a unit lies in one block
     static constexpr bool SWIZZLE128 = false;
     static constexpr int PBUF_FLOATS = R * G;           // per warp
     static_assert(D % VEC == 0 && VPR % LPR == 0, "head_dim must be a multiple of 16 bytes");
@@ -432,12 +433,16 @@ struct MmaUnit {
     static constexpr int R = 16;
     static constexpr int BOX_INNER = 64;
     static constexpr int BOXES = D / 64;
+    // 8-token blocks: a unit's rows 0..7 and 8..15 come from two consecutive
+    // blocks of the table, as two 8-row boxes; the second lands 1 KiB further,
+    // a whole swizzle atom, so the tile's layout is that of one 16-row box
+    static constexpr int BOX_ROWS = BS < R ? BS : R;
     static constexpr bool SWIZZLE128 = true;
     static constexpr int KS = D / 16;            // QK k-steps
     static constexpr int NT = D / 8;             // PV n-tiles
     static constexpr int PBUF_FLOATS = 0;
     static constexpr int BOX_BYTES = R * 128;
-    static_assert(G >= 1 && G <= 8 && BS % R == 0 && D % 64 == 0, "MmaUnit shape");
+    static_assert(G >= 1 && G <= 8 && (BS % R == 0 || BS == 8) && D % 64 == 0, "MmaUnit shape");
 
     uint32_t qa[KS][2];     // A fragments of Q: row g, k-low and k-high halves
     float o[NT][2];         // PV accumulators of row g (rows 8..15 are zero padding)
@@ -560,11 +565,11 @@ struct MmaUnit {
     }
 };
 
-// Policy choice: tensor cores for bf16 whose blocks hold whole 16-token
-// units; fp32 FMAs otherwise (fp32 caches, 8-token blocks).
+// Policy choice: tensor cores for bf16 (a 16-token unit spans two 8-token
+// blocks); fp32 FMAs for fp32 caches.
 template <typename T, int D, int BS, int G>
 using UnitFor = typename std::conditional<(std::is_same<T, __nv_bfloat16>::value &&
-                                           BS % 16 == 0),
+                                           (BS % 16 == 0 || BS == 8)),
                                           MmaUnit<D, BS, G>, CoreUnit<T, D, BS, G>>::type;
 
 // ---------------------------------------------------- kernel geometry ----
@@ -623,33 +628,50 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
     const int nk = first < u_end ? (u_end - first + ustride - 1) / ustride : 0;
 
     const int32_t* table = a.block_tables + (size_t)seq * a.max_blocks;
-    int win = 0;
+    // a unit spans two 8-token blocks on the tensor-core unit with bs 8
+    constexpr int HALVES = R / U::BOX_ROWS;
+    static_assert(HALVES == 1 || HALVES == 2, "a unit is one box of rows or two");
+    auto checked = [&](int id) {
+        if (id < 0 || id >= a.num_blocks) {
+            raise_error(a.err, PA_DEVERR_BLOCK_ID);
+            return a.num_blocks;         // outside the tensor map: TMA fills zeros
+        }
+        return id;
+    };
+    int win = 0, win1 = -1;
     auto load_window = [&](int k0) {
         const int k = k0 + lane;
-        int id = 0;
+        int id = 0, id1 = -1;
         if (k < nk) {
-            const int uu = first + ustride * k;
-            id = __ldg(table + (uu * R) / U::BS);
-            if (id < 0 || id >= a.num_blocks) {
-                raise_error(a.err, PA_DEVERR_BLOCK_ID);
-                id = a.num_blocks;       // outside the tensor map: TMA fills zeros
+            const int t0 = (first + ustride * k) * R;
+            id = checked(__ldg(table + t0 / U::BS));
+            if constexpr (HALVES == 2) {
+                if (t0 + U::BOX_ROWS < L) id1 = checked(__ldg(table + t0 / U::BS + 1));
             }
         }
         win = id;
+        win1 = id1;
     };
     auto slot = [&](int k) { return (cx.ring + k) % DEPTH; };
-    auto issue = [&](int k, int id) {     // lane 0 only
+    auto issue = [&](int k, int id, int id1) {     // lane 0 only
         const int s = slot(k);
         T* kdst = cx.stages + (size_t)s * (2 * R * D);
         const int uu = first + ustride * k;
-        const int row0 = (uu * R) % U::BS;
-        mbar_arrive_expect_tx(&cx.bars[s], Ly::STAGE_BYTES);
+        const int row0 = HALVES == 2 ? 0 : (uu * R) % U::BS;
+        const bool second = HALVES == 2 && id1 >= 0;
+        mbar_arrive_expect_tx(&cx.bars[s], HALVES == 1 || second ? Ly::STAGE_BYTES
+                                                                 : Ly::STAGE_BYTES / 2);
 #pragma unroll
         for (int b = 0; b < U::BOXES; ++b) {
-            tma_load_4d(kdst + b * R * U::BOX_INNER, tm_k, &cx.bars[s], b * U::BOX_INNER, kvh,
-                        row0, id);
-            tma_load_4d(kdst + R * D + b * R * U::BOX_INNER, tm_v, &cx.bars[s],
-                        b * U::BOX_INNER, kvh, row0, id);
+            T* kb = kdst + b * R * U::BOX_INNER;
+            T* vb = kdst + R * D + b * R * U::BOX_INNER;
+            tma_load_4d(kb, tm_k, &cx.bars[s], b * U::BOX_INNER, kvh, row0, id);
+            tma_load_4d(vb, tm_v, &cx.bars[s], b * U::BOX_INNER, kvh, row0, id);
+            if (second) {
+                constexpr int OFF = U::BOX_ROWS * U::BOX_INNER;
+                tma_load_4d(kb + OFF, tm_k, &cx.bars[s], b * U::BOX_INNER, kvh, 0, id1);
+                tma_load_4d(vb + OFF, tm_v, &cx.bars[s], b * U::BOX_INNER, kvh, 0, id1);
+            }
         }
     };
 
@@ -657,7 +679,8 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
     const int pro = cmin(DEPTH, nk);
     for (int k = 0; k < pro; ++k) {
         const int id = __shfl_sync(FULL_MASK, win, k);
-        if (lane == 0) issue(k, id);
+        const int id1 = __shfl_sync(FULL_MASK, win1, k);
+        if (lane == 0) issue(k, id, id1);
     }
     // the queries load while the first tiles are in flight
     U u;
@@ -685,7 +708,8 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
         if (kn < nk) {
             if (kn % 32 == 0) load_window(kn);
             const int id = __shfl_sync(FULL_MASK, win, kn % 32);
-            if (lane == 0) issue(kn, id);
+            const int id1 = __shfl_sync(FULL_MASK, win1, kn % 32);
+            if (lane == 0) issue(kn, id, id1);
         }
     }
     if (failed) {

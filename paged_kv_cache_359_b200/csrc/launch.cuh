@@ -52,10 +52,12 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
     constexpr pa_dtype DT = std::is_same<T, float>::value ? PA_DTYPE_F32 : PA_DTYPE_BF16;
     CUtensorMap mk, mv;
     if (pa_status s = encode_cache_map(&mk, l.k_cache, DT, D, l.num_kv_heads, BS,
-                                       l.args.num_blocks, U::BOX_INNER, U::R, U::SWIZZLE128))
+                                       l.args.num_blocks, U::BOX_INNER, U::BOX_ROWS,
+                                       U::SWIZZLE128))
         return s;
     if (pa_status s = encode_cache_map(&mv, l.v_cache, DT, D, l.num_kv_heads, BS,
-                                       l.args.num_blocks, U::BOX_INNER, U::R, U::SWIZZLE128))
+                                       l.args.num_blocks, U::BOX_INNER, U::BOX_ROWS,
+                                       U::SWIZZLE128))
         return s;
     if (l.split && l.args.part_tokens % U::R != 0)
         return fail(PA_ERR_INVALID_ARG, "partition must be a multiple of %d tokens", U::R);
