@@ -56,7 +56,8 @@ def test_tiny_fp32_append():
 
 
 @pytest.mark.parametrize("d,bs,hq,hk", [(128, 16, 32, 8), (64, 8, 8, 8), (256, 32, 16, 2),
-                                        (128, 16, 32, 32)])
+                                        (128, 16, 32, 32), (128, 8, 32, 8), (128, 64, 32, 8),
+                                        (64, 128, 8, 2)])
 def test_append_block_boundaries_and_skips(d, bs, hq, hk):
     # lengths ending on, just past and inside a block; two sequences skip
     fixed = {0: bs, 1: bs - 1, 2: 1, 3: 3 * bs + 5, 4: 0}

@@ -19,7 +19,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("bs,hq,hk,d,dt", [(16, 32, 8, 128, "bf16"), (8, 8, 8, 64, "f32"),
-                                           (32, 16, 2, 256, "bf16")])
+                                           (32, 16, 2, 256, "bf16"), (8, 32, 8, 128, "bf16"),
+                                           (64, 32, 8, 128, "bf16")])
 def test_compaction_preserves_decode_bits(bs, hq, hk, d, dt):
     rng = np.random.default_rng(bs * 7 + d)
     nb, cap = 900, 64

@@ -1,7 +1,7 @@
 """GPU parity for prefix sharing and copy-on-write: 64 sequences forked from
 one prefix (the last shared block half full, so the first write of each
 sharer but the last copies it), divergent tails, one copy_blocks, one
-reshape_and_cache, then decode -- for block_size {8,16,32} x head_dim
+reshape_and_cache, then decode -- for block_size {8,16,32,64,128} x head_dim
 {64,128,256}, 32 q / 8 kv heads, bf16."""
 
 import numpy as np
@@ -51,7 +51,7 @@ def build(problem):
 
 @pytest.mark.parametrize("aligned", [False, True])
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("bs", [8, 16, 32, 64, 128])
 def test_prefix_sharing_copy_on_write(bs, d, aligned):
     problem = pa_inputs.prefix(bs, d, aligned=aligned)
     tables, lens, slots, cows, prefix_table = build(problem)

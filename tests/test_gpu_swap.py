@@ -27,7 +27,8 @@ def _pools(nb_dev, nb_host, bs=16, hk=8, d=128, dtype=torch.bfloat16, seed=0):
 
 
 @pytest.mark.parametrize("bs,d,dt", [(16, 128, torch.bfloat16), (8, 64, torch.float32),
-                                     (32, 256, torch.bfloat16)])
+                                     (32, 256, torch.bfloat16), (64, 128, torch.bfloat16),
+                                     (128, 64, torch.bfloat16)])
 @pytest.mark.parametrize("mapping_on_device", [True, False])
 def test_swap_out_and_in_bitwise(bs, d, dt, mapping_on_device):
     rng = np.random.default_rng(bs + d)
