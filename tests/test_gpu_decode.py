@@ -194,3 +194,23 @@ def test_longest_first_order_around_the_register_and_shared_ranges(num_seqs):
     out = torch.full_like(data["q"], float("nan"))
     assert_close(run_decode(data, problem, out=out), oracle_decode(data, problem))
     device_clean()
+
+
+@pytest.mark.parametrize("hk,g,bs", [(1, 4, 16), (3, 2, 16), (1, 8, 8), (3, 1, 32), (4, 4, 16)])
+def test_head_dim_64_with_odd_and_even_kv_heads(hk, g, bs):
+    """bf16 head_dim 64 with odd and even kv head counts, through the
+    longest-first, split and cluster launches."""
+    problem = pa_inputs.random_small(700 + 10 * hk + g, num_seqs=7, max_len=400,
+                                     num_heads=hk * g, num_kv_heads=hk, head_dim=64,
+                                     block_size=bs, dtype="bf16", zero_len=True,
+                                     fixed={0: 1, 1: 0, 2: bs})
+    data = pa_inputs.materialize(problem, "cuda")
+    ref = oracle_decode(data, problem)
+    assert_close(run_decode(data, problem), ref)
+    assert_close(run_decode(data, problem, split=True, partition=64), ref)
+    pa.pa_set_option("decode_split_ctas", 2)
+    try:
+        assert_close(run_decode(data, problem), ref)
+    finally:
+        pa.pa_set_option("decode_split_ctas", 0)
+    device_clean()
