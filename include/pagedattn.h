@@ -171,6 +171,10 @@ pa_status pa_decode_append(void* out_d, const void* q_d, const void* key_d,
  * the unnormalised output into `workspace_d`; a second kernel merges them:
  *   out = sum_p exp(m_p - M) o_p / sum_p exp(m_p - M) l_p,  M = max_p m_p.
  * Sequences with a single partition are written directly by the first kernel.
+ * When few (sequence, head) pairs have many partitions, the merge splits each
+ * pair's partitions into chunks over several CTAs, which leave their sums in
+ * the workspace; the last chunk adds them in chunk order, so the result does
+ * not depend on timing.
  *   max_context_len  >= every context_lens[s]; sizes the workspace
  *   workspace_d      caller-owned device memory of at least
  *                    pa_decode_split_workspace_bytes(...) bytes, 16-byte aligned

@@ -144,6 +144,17 @@ pa_status dispatch_decode(const DecodeLaunch& l, pa_dtype dt, int head_dim) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Chunks of partitions per (sequence, head) in the log-sum-exp reduce: enough
+// CTAs to fill the GPU a few times over (a fixed target, so the workspace
+// size does not depend on the device), at least 16 partitions per chunk.
+int reduce_chunks(size_t heads, size_t parts) {
+    constexpr size_t TARGET_CTAS = 600;
+    size_t c = (TARGET_CTAS + heads - 1) / heads;
+    const size_t most = (parts + 15) / 16;
+    if (c > most) c = most;
+    return c < 1 ? 1 : (int)c;
+}
+
 }  // namespace
 
 bool pdl_enabled() {
@@ -405,8 +416,14 @@ size_t pa_decode_split_workspace_bytes(int num_seqs, int num_heads, int head_dim
                              ? 1
                              : (size_t)((max_context_len + (int64_t)partition_size - 1) /
                                         partition_size);
-    const size_t rows = (size_t)num_seqs * num_heads * parts;
-    return 2 * align256(rows * sizeof(float)) + rows * head_dim * sizeof(float);
+    const size_t heads = (size_t)num_seqs * num_heads;
+    const size_t rows = heads * parts;
+    size_t bytes = 2 * align256(rows * sizeof(float)) + align256(rows * head_dim * sizeof(float));
+    const int chunks = reduce_chunks(heads, parts);
+    if (chunks > 1)      // the reduce's per-chunk sums and arrival counts
+        bytes += align256(heads * chunks * (head_dim + 4) * sizeof(float)) +
+                 align256(heads * sizeof(unsigned));
+    return bytes;
 }
 
 pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -449,6 +466,15 @@ pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const v
     l.args.ws_m = reinterpret_cast<float*>(ws);
     l.args.ws_l = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
     l.args.ws_o = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
+    const size_t heads = (size_t)num_seqs * num_heads;
+    l.args.reduce_chunks = reduce_chunks(heads, (size_t)parts64);
+    if (l.args.reduce_chunks > 1) {
+        char* p = ws + 2 * align256(rows * sizeof(float)) +
+                  align256(rows * head_dim * sizeof(float));
+        l.args.ws_part = reinterpret_cast<float*>(p);
+        l.args.ws_cnt = reinterpret_cast<unsigned*>(
+            p + align256(heads * l.args.reduce_chunks * (head_dim + 4) * sizeof(float)));
+    }
     l.args.err = device_error_word();
     if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
     l.args.scale_log2 = scale * 1.4426950408889634f;

@@ -69,6 +69,12 @@ struct DecodeArgs {
     float* ws_m;                  // split: [S, Hq, max_parts] running max (log2 units)
     float* ws_l;                  // split: [S, Hq, max_parts] sum of exponentials
     float* ws_o;                  // split: [S, Hq, max_parts, D] unnormalised output
+    // split reduce over reduce_chunks chunks of partitions per (sequence,
+    // head): per chunk (sum of weighted outputs [D], sum of weights), then the
+    // last chunk to arrive combines them (arrival counts zeroed by partition 0)
+    float* ws_part;               // [S * Hq, reduce_chunks, D + 4]: sums [D], weight sum
+    unsigned* ws_cnt;             // [S * Hq]
+    int reduce_chunks;
     unsigned* err;                // device error word
     float scale_log2;             // scale * log2(e)
     int num_seqs;
@@ -790,6 +796,9 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             if (part > 0) return;
             nparts = 1;                       // degrade: partition 0 covers everything
         }
+        // partition 0 zeroes the reduce's arrival counts of this kv head's group
+        if (part == 0 && nparts > 1 && a.ws_cnt && threadIdx.x < G)
+            a.ws_cnt[(size_t)seq * a.num_heads + (size_t)kvh * G + threadIdx.x] = 0u;
     }
 
     Ctx<U> cx;
@@ -1023,15 +1032,21 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
 }
 
 // ---- log-sum-exp merge of split partitions ----
-// grid (num_seqs * num_heads, D / 32), 256 threads: warp w folds partitions
-// w, w+8, ...; lane = one of 32 dimensions.
+// grid (num_seqs * num_heads, reduce_chunks), 256 threads.  With the maximum
+// M of all the head's partition maxima, chunk c sums w_p = 2^(m_p - M) times
+// l_p and times o_p over its partitions: D/4 threads take the float4 columns
+// of a partition's row, 256/(D/4) rows at a time (several loads in flight
+// per thread), and the rows' sums fold in shared memory in a fixed order.
+// With one chunk it writes the output; otherwise it leaves its sums and the
+// last chunk to arrive adds them in chunk order (the result does not depend
+// on the arrival order).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
     pdl_wait();
     pdl_launch_dependents();
-    const int sh = blockIdx.x;
+    constexpr int NT = 256, TPR = D / 4, RP = NT / TPR;
+    const int sh = blockIdx.x, chunk = blockIdx.y, C = gridDim.y;
     const int seq = sh / a.num_heads;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     int L = a.context_lens[seq];
     L = L < 0 ? 0 : cmin(L, a.max_tokens);
     const int nparts = (L + a.part_tokens - 1) / a.part_tokens;
@@ -1040,38 +1055,93 @@ __global__ void __launch_bounds__(256) lse_reduce_kernel(const DecodeArgs a) {
     const float* m = a.ws_m + base;
     const float* l = a.ws_l + base;
     const float* o = a.ws_o + base * D;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
 
-    __shared__ float red[8];
-    __shared__ float part_num[8][32];
+    __shared__ float red[NT / 32];
+    __shared__ float4 rows[RP][TPR];
+    __shared__ int last;
     float big = -INFINITY;
-    for (int p = threadIdx.x; p < nparts; p += 256) big = fmaxf(big, m[p]);
+    for (int p = tid; p < nparts; p += NT) big = fmaxf(big, m[p]);
     for (int off = 16; off >= 1; off >>= 1) big = fmaxf(big, __shfl_xor_sync(FULL_MASK, big, off));
     if (lane == 0) red[warp] = big;
     __syncthreads();
     big = red[0];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) big = fmaxf(big, red[w]);
+    for (int w = 1; w < NT / 32; ++w) big = fmaxf(big, red[w]);
     __syncthreads();
+
+    const int per = (nparts + C - 1) / C;
+    const int p0 = chunk * per, p1 = cmin(nparts, p0 + per);
     float den = 0.f;
-    for (int p = threadIdx.x; p < nparts; p += 256) den += exp2_approx(m[p] - big) * l[p];
+    for (int p = p0 + tid; p < p1; p += NT) den += exp2_approx(m[p] - big) * l[p];
     for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(FULL_MASK, den, off);
     if (lane == 0) red[warp] = den;
     __syncthreads();
     den = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) den += red[w];
+    for (int w = 0; w < NT / 32; ++w) den += red[w];
 
-    const int d = blockIdx.y * 32 + lane;
-    float num = 0.f;
-    for (int p = warp; p < nparts; p += 8) num = fmaf(exp2_approx(m[p] - big), o[(size_t)p * D + d], num);
-    part_num[warp][lane] = num;
-    __syncthreads();
-    if (warp == 0) {
-        float t = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) t += part_num[w][lane];
-        store_out(reinterpret_cast<T*>(a.out) + (size_t)sh * D + d, den > 0.f ? t / den : 0.f);
+    const int r = tid / TPR, c4 = tid % TPR;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int p = p0 + r; p < p1; p += RP) {
+        const float w = exp2_approx(m[p] - big);
+        const float4 v = reinterpret_cast<const float4*>(o + (size_t)p * D)[c4];
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
     }
+    rows[r][c4] = acc;
+    __syncthreads();
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid < TPR) {
+#pragma unroll
+        for (int rr = 0; rr < RP; ++rr) {
+            num.x += rows[rr][tid].x;
+            num.y += rows[rr][tid].y;
+            num.z += rows[rr][tid].z;
+            num.w += rows[rr][tid].w;
+        }
+    }
+    T* out = reinterpret_cast<T*>(a.out) + (size_t)sh * D;
+    auto write = [&](float4 n, float dd) {
+        const float inv = dd > 0.f ? 1.f / dd : 0.f;
+        store_out(out + 4 * tid + 0, dd > 0.f ? n.x * inv : 0.f);
+        store_out(out + 4 * tid + 1, dd > 0.f ? n.y * inv : 0.f);
+        store_out(out + 4 * tid + 2, dd > 0.f ? n.z * inv : 0.f);
+        store_out(out + 4 * tid + 3, dd > 0.f ? n.w * inv : 0.f);
+    };
+    if (C == 1) {
+        if (tid < TPR) write(num, den);
+        return;
+    }
+    float* part = a.ws_part + ((size_t)sh * C + chunk) * (D + 4);
+    if (tid < TPR) reinterpret_cast<float4*>(part)[tid] = num;
+    if (tid == 0) part[D] = den;
+    __threadfence();                                 // the sums, device-wide
+    __syncthreads();
+    if (tid == 0) {
+        last = atomicAdd(a.ws_cnt + sh, 1u) == (unsigned)(C - 1);
+        __threadfence();
+    }
+    __syncthreads();
+    if (!last) return;
+    if (tid < TPR) {
+        float4 n = make_float4(0.f, 0.f, 0.f, 0.f);
+        float dd = 0.f;
+        for (int k = 0; k < C; ++k) {
+            const float* pk = a.ws_part + ((size_t)sh * C + k) * (D + 4);
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(pk) + tid);
+            n.x += v.x;
+            n.y += v.y;
+            n.z += v.z;
+            n.w += v.w;
+            dd += __ldcg(pk + D);
+        }
+        write(n, dd);
+    }
+    if (tid == 0) a.ws_cnt[sh] = 0;                  // ready for the next launch
 }
 
 }  // namespace pa

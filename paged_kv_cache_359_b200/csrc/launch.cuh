@@ -110,7 +110,7 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
         e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
         if (e == cudaSuccess) {
             cudaLaunchConfig_t rc = {};
-            rc.gridDim = dim3(l.num_seqs * l.args.num_heads, D / 32);
+            rc.gridDim = dim3(l.num_seqs * l.args.num_heads, l.args.reduce_chunks);
             rc.blockDim = dim3(256);
             rc.stream = l.stream;
             cudaLaunchAttribute rattr[1];

@@ -71,10 +71,17 @@ def test_decode_argument_checks(over, status):
 
 def test_split_workspace_size():
     lib = _native.lib()
-    # 2 sequences x 32 heads x ceil(1048576 / 512) partitions
+    def a256(x):
+        return (x + 255) // 256 * 256
+    # 2 sequences x 32 heads x ceil(1048576 / 512) partitions: m, l, o, then
+    # the reduce's 10 chunks per head (ceil(600 / 64)) of D + 4 floats and counts
     rows = 2 * 32 * 2048
     n = lib.pa_decode_split_workspace_bytes(2, 32, 128, 1048576, 512)
-    assert n == 2 * (((rows * 4) + 255) // 256 * 256) + rows * 128 * 4
+    assert n == 2 * a256(rows * 4) + a256(rows * 128 * 4) + a256(64 * 10 * 132 * 4) + a256(64 * 4)
+    # a large batch: one chunk per head, no extra
+    rows = 256 * 32 * 2
+    n = lib.pa_decode_split_workspace_bytes(256, 32, 128, 1024, 512)
+    assert n == 2 * a256(rows * 4) + a256(rows * 128 * 4)
     assert lib.pa_decode_split_workspace_bytes(0, 32, 128, 10, 512) == 0
 
 
