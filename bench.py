@@ -195,14 +195,15 @@ def make_problem(name: str, extra_tokens: int, rank: int, block_size=None, head_
     raise ValueError(f"unknown workload {name}")
 
 
-def build_prefix_loop(device, extra_tokens: int, kernel: str, partition: int):
-    """64 sequences forked from one 2040-token prefix (block 16, head_dim 128,
-    32 q / 8 kv heads, bf16), tails U[0, 512]: the parent's prefix is
-    written, the children fork it, every sequence appends its tail through
-    the allocator (the shared half-full last block is copied on first write),
-    then one pa_copy_blocks and one pa_reshape_and_cache fill the cache."""
+def build_prefix_loop(device, extra_tokens: int, kernel: str, partition: int,
+                      block_size: int = 16, head_dim: int = 128):
+    """64 sequences forked from one (2048 - block_size/2)-token prefix (32 q /
+    8 kv heads, bf16), tails U[0, 512]: the parent's prefix is written, the
+    children fork it, every sequence appends its tail through the allocator
+    (the shared half-full last block is copied on first write), then one
+    pa_copy_blocks and one pa_reshape_and_cache fill the cache."""
     import paged_kv_cache_359_b200 as pa
-    pp = pa_inputs.prefix(16, 128, extra_tokens=extra_tokens)
+    pp = pa_inputs.prefix(block_size, head_dim, extra_tokens=extra_tokens)
     bs, hk, d, s = pp.block_size, pp.num_kv_heads, pp.head_dim, pp.num_seqs
     cap = pp.max_blocks_per_seq
     alloc = pa.BlockAllocator(pp.num_blocks, bs, pp.free_order)
@@ -790,9 +791,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--block-size", type=int, default=None,
-                    help="gqa workload: block size (default 16; the block-size study)")
+                    help="gqa / prefix workloads: block size (default 16)")
     ap.add_argument("--head-dim", type=int, default=None,
-                    help="gqa workload: head_dim (default 128)")
+                    help="gqa / prefix workloads: head_dim (default 128)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (PA_OPT_PDL 0)")
     ap.add_argument("--compact", action="store_true",
@@ -810,8 +811,8 @@ def main():
     args.fused = args.kernel == "decode" and not args.unfused
     if args.compact and args.workload not in ("gqa", "mha"):
         ap.error("--compact runs on the gqa and mha workloads")
-    if (args.block_size or args.head_dim) and args.workload != "gqa":
-        ap.error("--block-size / --head-dim apply to the gqa workload")
+    if (args.block_size or args.head_dim) and args.workload not in ("gqa", "prefix"):
+        ap.error("--block-size / --head-dim apply to the gqa and prefix workloads")
     if args.kernel == "cascade" and args.workload != "prefix":
         ap.error("--kernel cascade needs the prefix workload (its sequences share a prefix)")
     rank, world, local = dist_env()
@@ -839,7 +840,8 @@ def main():
     try:
         extra = 2 * (args.steps + args.warmup) + 4
         if args.workload == "prefix":
-            loop = build_prefix_loop(dev, extra, args.kernel, args.partition)
+            loop = build_prefix_loop(dev, extra, args.kernel, args.partition,
+                                     args.block_size or 16, args.head_dim or 128)
             p = loop.p
         else:
             p = make_problem(args.workload, extra, rank, args.block_size, args.head_dim)
