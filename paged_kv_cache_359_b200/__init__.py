@@ -63,6 +63,43 @@ def _dev(*tensors):
             raise ValueError("tensors must be contiguous")
 
 
+def _need(cond: bool, what: str):
+    if not cond:
+        raise ValueError(what)
+
+
+def _cache_pair(k_cache, v_cache):
+    """[NB, bs, Hk, D] each, same shape and dtype.  Returns (NB, bs, Hk, D)."""
+    _need(k_cache.dim() == 4, "caches must be [num_blocks, block_size, kv_heads, head_dim]")
+    _need(v_cache.shape == k_cache.shape and v_cache.dtype == k_cache.dtype,
+          "k_cache and v_cache must have the same shape and dtype")
+    return tuple(k_cache.shape)
+
+
+def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens):
+    """Shapes and dtypes of a decode call.  Returns (S, Hq, D, NB, bs, Hk)."""
+    _dev(out, q, k_cache, v_cache, block_tables, context_lens)
+    nb, bs, hk, d = _cache_pair(k_cache, v_cache)
+    _need(q.dim() == 3 and q.shape[2] == d, "q must be [num_seqs, num_heads, head_dim]")
+    _need(out.shape == q.shape, "out must have q's shape")
+    _need(q.dtype == k_cache.dtype and out.dtype == q.dtype, "q, out and caches share one dtype")
+    s, hq, _ = q.shape
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2 and
+          block_tables.shape[0] == s, "block_tables must be int32 [num_seqs, max_blocks]")
+    _need(context_lens.dtype == torch.int32 and tuple(context_lens.shape) == (s,),
+          "context_lens must be int32 [num_seqs]")
+    return s, hq, d, nb, bs, hk
+
+
+def _new_rows(key, value, num_tokens, hk, d, cache_dtype, slot_mapping):
+    _need(key.shape == value.shape and tuple(key.shape) == (num_tokens, hk, d),
+          "key and value must be [num_tokens, kv_heads, head_dim]")
+    _need(key.dtype == cache_dtype and value.dtype == cache_dtype,
+          "key and value must have the caches' dtype")
+    _need(slot_mapping.dtype == torch.int64 and tuple(slot_mapping.shape) == (num_tokens,),
+          "slot_mapping must be int64 [num_tokens]")
+
+
 def _ptr(t: torch.Tensor):
     return ctypes.c_void_p(t.data_ptr())
 
@@ -76,9 +113,8 @@ def _stream(stream):
 def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
     """key/value [T, Hk, D]; caches [NB, bs, Hk, D]; slot_mapping int64 [T]."""
     _dev(key, value, k_cache, v_cache, slot_mapping)
-    nb, bs, hk, d = k_cache.shape
-    if slot_mapping.dtype != torch.int64:
-        raise ValueError("slot_mapping must be int64")
+    nb, bs, hk, d = _cache_pair(k_cache, v_cache)
+    _new_rows(key, value, key.shape[0], hk, d, k_cache.dtype, slot_mapping)
     check(lib().pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
                                      _ptr(slot_mapping), key.shape[0], hk, d, bs, nb,
                                      _dtype(k_cache), _stream(stream)))
@@ -87,9 +123,7 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, stream=None):
     """out/q [S, Hq, D]; caches [NB, bs, Hk, D]; block_tables int32 [S, maxB];
     context_lens int32 [S].  Writes ``out`` and returns it."""
-    _dev(out, q, k_cache, v_cache, block_tables, context_lens)
-    s, hq, d = q.shape
-    nb, bs, hk, _ = k_cache.shape
+    s, hq, d, nb, bs, hk = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens)
     check(lib().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                           block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb,
                           float(scale), _dtype(q), _stream(stream)))
@@ -100,11 +134,9 @@ def pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, block_t
                      context_lens, scale, stream=None):
     """pa_reshape_and_cache of one new row per sequence (key/value [S, Hk, D],
     slot_mapping int64 [S], -1 = none) then pa_decode, in one launch."""
-    _dev(out, q, key, value, k_cache, v_cache, slot_mapping, block_tables, context_lens)
-    s, hq, d = q.shape
-    nb, bs, hk, _ = k_cache.shape
-    if slot_mapping.dtype != torch.int64:
-        raise ValueError("slot_mapping must be int64")
+    s, hq, d, nb, bs, hk = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens)
+    _dev(key, value, slot_mapping)
+    _new_rows(key, value, s, hk, d, k_cache.dtype, slot_mapping)
     check(lib().pa_decode_append(_ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_cache),
                                  _ptr(v_cache), _ptr(slot_mapping), _ptr(block_tables),
                                  block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb,
@@ -122,9 +154,7 @@ def pa_decode_split(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                     max_context_len, partition_size=512, workspace=None, stream=None):
     """Split-K decode; ``workspace`` is a CUDA byte tensor of at least
     ``pa_decode_split_workspace_bytes(...)`` bytes (allocated here if None)."""
-    _dev(out, q, k_cache, v_cache, block_tables, context_lens)
-    s, hq, d = q.shape
-    nb, bs, hk, _ = k_cache.shape
+    s, hq, d, nb, bs, hk = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens)
     need = pa_decode_split_workspace_bytes(s, hq, d, max_context_len, partition_size)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -142,9 +172,7 @@ def pa_decode_split_noalloc(out, q, k_cache, v_cache, block_tables, context_lens
     """pa_decode_split for callers that cannot allocate device memory: the
     library's built-in 16 MiB scratch replaces the caller workspace.  Calls
     share that scratch, so calls that overlap on the GPU must not be issued."""
-    _dev(out, q, k_cache, v_cache, block_tables, context_lens)
-    s, hq, d = q.shape
-    nb, bs, hk, _ = k_cache.shape
+    s, hq, d, nb, bs, hk = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens)
     check(lib().pa_decode_split_noalloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                         _ptr(block_tables), block_tables.shape[1],
                                         _ptr(context_lens), s, hq, hk, d, bs, nb, float(scale),
@@ -165,9 +193,12 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens
     """Decode of a batch whose sequences come in groups sharing a prefix:
     group_starts int32 [G+1] (device), prefix_lens int32 [G] (device, whole
     blocks, multiples of 16).  Same result as pa_decode."""
-    _dev(out, q, k_cache, v_cache, block_tables, context_lens, group_starts, prefix_lens)
-    s, hq, d = q.shape
-    nb, bs, hk, _ = k_cache.shape
+    s, hq, d, nb, bs, hk = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens)
+    _dev(group_starts, prefix_lens)
+    _need(group_starts.dtype == torch.int32 and prefix_lens.dtype == torch.int32 and
+          group_starts.dim() == 1 and prefix_lens.dim() == 1 and
+          group_starts.shape[0] == prefix_lens.shape[0] + 1,
+          "group_starts must be int32 [groups + 1] and prefix_lens int32 [groups]")
     need = pa_decode_shared_prefix_workspace_bytes(s, hq, d, max_prefix_len)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
@@ -184,9 +215,9 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
     """block_mapping int64 [P, 2] of (src, dst) on the device."""
     _dev(k_cache, v_cache, block_mapping)
-    nb, bs, hk, d = k_cache.shape
-    if block_mapping.dtype != torch.int64:
-        raise ValueError("block_mapping must be int64")
+    nb, bs, hk, d = _cache_pair(k_cache, v_cache)
+    _need(block_mapping.dtype == torch.int64 and block_mapping.dim() == 2 and
+          block_mapping.shape[1] == 2, "block_mapping must be int64 [pairs, 2]")
     check(lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping),
                                block_mapping.shape[0], hk, d, bs, nb, _dtype(k_cache),
                                _stream(stream)))
@@ -200,10 +231,12 @@ def pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping, stream=None):
             raise ValueError("tensors must be contiguous")
         if not (t.is_cuda or t.is_pinned()):
             raise ValueError("pools and mapping must be on a CUDA device or in pinned memory")
-    if block_mapping.dtype != torch.int64:
-        raise ValueError("block_mapping must be int64")
-    nb_dst, bs, hk, d = dst_k.shape
-    nb_src = src_k.shape[0]
+    _need(block_mapping.dtype == torch.int64 and block_mapping.dim() == 2 and
+          block_mapping.shape[1] == 2, "block_mapping must be int64 [pairs, 2]")
+    nb_dst, bs, hk, d = _cache_pair(dst_k, dst_v)
+    nb_src = _cache_pair(src_k, src_v)[0]
+    _need(tuple(src_k.shape[1:]) == (bs, hk, d) and src_k.dtype == dst_k.dtype,
+          "both pools must have the same block shape and dtype")
     check(lib().pa_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v),
                                _ptr(block_mapping), block_mapping.shape[0], hk, d, bs, nb_src,
                                nb_dst, _dtype(dst_k), _stream(stream)))

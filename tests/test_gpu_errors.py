@@ -63,3 +63,26 @@ def test_split_workspace_too_small_is_rejected():
         pa.pa_decode_split(out, data["q"], data["k_cache"], data["v_cache"],
                            data["block_tables"], data["context_lens"], problem.scale,
                            max_context_len=60, partition_size=16, workspace=ws)
+
+
+def test_binding_rejects_wrong_dtypes_and_shapes_before_the_library():
+    problem, data = _small()
+    out = torch.empty_like(data["q"])
+    args = [out, data["q"], data["k_cache"], data["v_cache"], data["block_tables"],
+            data["context_lens"], problem.scale]
+    bad = [
+        (4, data["block_tables"].long()),                        # int64 tables
+        (5, data["context_lens"].long()),                        # int64 lengths
+        (3, data["v_cache"][:-1].contiguous()),                  # pools of different sizes
+        (0, out.float()),                                        # out in another dtype
+        (1, data["q"][:, :4].contiguous()),                      # q and out shapes differ
+    ]
+    for i, t in bad:
+        call = list(args)
+        call[i] = t
+        with pytest.raises(ValueError):
+            pa.pa_decode(*call)
+    with pytest.raises(ValueError):
+        pa.pa_copy_blocks(data["k_cache"], data["v_cache"],
+                          torch.tensor([0, 1], dtype=torch.int64, device="cuda"))
+    device_clean()
