@@ -1,7 +1,8 @@
 """Plant plausible mistakes in the oracle (CPU only, via monkeypatch) and
 check that at least one pin catches each: a wrong index, a dropped term, a
 wrong sign, a transposed operand, a wrong merge weight, a wrong free-pool
-order and a missed reference-count update."""
+order, a missed reference-count update, and compaction that drops counts,
+reuses a destination, overwrites a live block or remaps backwards."""
 
 import importlib
 import math
@@ -104,3 +105,43 @@ def test_copy_on_write_without_decref_is_caught(monkeypatch):
         orig_decref(self, block)
     monkeypatch.setattr(alloc_mod.BlockAllocator, "decref", skip_first_decref)
     assert _fails(alloc_pins.test_copy_on_write_of_a_shared_partial_block)
+
+
+def _compaction_variant(carry_counts=True, drop_taken=True, only_free=True):
+    """oracle.compact with one step of it changed."""
+    def compact(alloc, target):
+        live_high = [b for b in range(target, alloc.num_blocks) if alloc.ref[b] > 0]
+        low = sorted(b for b in alloc.free if b < target) if only_free else list(range(target))
+        if len(live_high) > len(low):
+            raise oracle.OutOfBlocks()
+        moves = list(zip(live_high, low[:len(live_high)]))
+        taken = {d for _, d in moves} if drop_taken else set()
+        for s, d in moves:
+            alloc.ref[d] = alloc.ref[s] if carry_counts else 1
+            alloc.ref[s] = 0
+        alloc.free = [b for b in alloc.free if b < target and b not in taken]
+        alloc.ref = alloc.ref[:target]
+        alloc.num_blocks = target
+        return moves
+    return compact
+
+
+@pytest.mark.parametrize("mutation", [dict(carry_counts=False), dict(drop_taken=False),
+                                      dict(only_free=False)])
+def test_compaction_mistakes_are_caught(monkeypatch, mutation):
+    monkeypatch.setattr(oracle, "compact", _compaction_variant(**mutation))
+    assert any(_fails(lambda s=s: alloc_pins.test_compaction_packs_live_blocks_below_the_target(s))
+               for s in range(5))
+
+
+def test_reversed_remap_is_caught(monkeypatch):
+    monkeypatch.setattr(oracle, "remap", lambda table, moves: [
+        {d: s for s, d in moves}.get(b, b) for b in table])
+    assert _fails(lambda: alloc_pins.test_compaction_packs_live_blocks_below_the_target(0))
+
+
+def test_unmutated_compaction_variant_passes(monkeypatch):
+    """The variant builder with nothing changed is the oracle's compaction."""
+    monkeypatch.setattr(oracle, "compact", _compaction_variant())
+    for s in range(5):
+        alloc_pins.test_compaction_packs_live_blocks_below_the_target(s)
