@@ -245,8 +245,9 @@ pa_status pa_decode_split_noalloc(void* out_d, const void* q_d,
  *                    prefix_lens[g] / block_size table entries
  *   max_group_size   >= every group's size
  *   workspace_d      >= pa_decode_shared_prefix_workspace_bytes(...) bytes
- * bf16 and block_size a multiple of 16 only (else PA_ERR_UNSUPPORTED).
- * Validate mode checks every precondition above.
+ * bf16 only (else PA_ERR_UNSUPPORTED); any built block_size (with 8-token
+ * blocks a 16-token unit spans two blocks).  Validate mode checks every
+ * precondition above.
  */
 size_t pa_decode_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                                int max_prefix_len);

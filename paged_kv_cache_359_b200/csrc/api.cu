@@ -520,8 +520,8 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
                                         num_kv_heads, head_dim, block_size, num_blocks, dtype,
                                         scale))
         return s;
-    if (dtype != PA_DTYPE_BF16 || block_size % 16 != 0)
-        return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs bf16 and a block_size multiple of 16");
+    if (dtype != PA_DTYPE_BF16)
+        return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs bf16");
     if (num_groups <= 0 || max_group_size <= 0 || max_prefix_len < 0 ||
         (int64_t)max_prefix_len > (int64_t)max_blocks_per_seq * block_size)
         return fail(PA_ERR_INVALID_ARG, "bad group or prefix bounds");

@@ -71,19 +71,19 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
     cfg.stream = l.stream;
     cudaError_t e;
     if (l.cascade) {
-        if constexpr (std::is_same<T, __nv_bfloat16>::value && BS % 16 == 0) {
+        if constexpr (std::is_same<T, __nv_bfloat16>::value && (BS % 16 == 0 || BS == 8)) {
             using C = PrefixCfg<D, BS, G>;
             static std::atomic<unsigned long long> done_p{0};
             auto pk = shared_prefix_kernel<D, BS, G>;
             if (pa_status s = allow_smem(pk, C::SMEM_BYTES, done_p)) return s;
             // all of L1 as shared memory, so two CTAs fit an SM
             cudaFuncSetAttribute(pk, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-            CUtensorMap sk, sv;        // 128B-swizzled {64, 1, 16, 1} boxes
+            CUtensorMap sk, sv;        // 128B-swizzled {64, 1, 16 or 8, 1} boxes
             if (pa_status s = encode_cache_map(&sk, l.k_cache, DT, D, l.num_kv_heads, BS,
-                                               l.args.num_blocks, 64, 16, true))
+                                               l.args.num_blocks, 64, C::BOX_ROWS, true))
                 return s;
             if (pa_status s = encode_cache_map(&sv, l.v_cache, DT, D, l.num_kv_heads, BS,
-                                               l.args.num_blocks, 64, 16, true))
+                                               l.args.num_blocks, 64, C::BOX_ROWS, true))
                 return s;
             if (l.max_chunks > 0) {
                 cudaLaunchConfig_t pc = {};
@@ -99,7 +99,7 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
                     return fail(PA_ERR_CUDA, "shared-prefix launch: %s", cudaGetErrorString(e));
             }
         } else {
-            return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs bf16 and 16 | block_size");
+            return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs bf16");
         }
     }
     if (l.split) {

@@ -29,6 +29,9 @@ template <int D_, int BS_, int G_>
 struct PrefixCfg {
     static constexpr int D = D_, BS = BS_, G = G_;
     static constexpr int R = 16;                 // tokens per unit
+    // 8-token blocks: a unit's rows 0..7 and 8..15 are two 8-row boxes from
+    // consecutive table entries, the second one swizzle atom further on
+    static constexpr int BOX_ROWS = BS < R ? BS : R;
     static constexpr int BOXES = D / 64;         // 128-byte swizzled boxes per tile
     static constexpr int BOX_BYTES = R * 128;
     static constexpr int KS = D / 16, NT = D / 8;
@@ -37,7 +40,7 @@ struct PrefixCfg {
     static constexpr int MAX_CONSUMERS = 4;      // 64 query rows per CTA: two CTAs per SM
     static constexpr int THREADS = (MAX_CONSUMERS + 1) * 32;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * STAGES * 8 + 1024;
-    static_assert(BS % R == 0 && D % 64 == 0, "shared-prefix shape");
+    static_assert((BS % R == 0 || BS == 8) && D % 64 == 0, "shared-prefix shape");
 };
 
 constexpr int PREFIX_CHUNK_TOKENS = 256;
@@ -102,19 +105,30 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS)
                     break;                  // consumers time out on `full` and finish
                 }
                 const int u = u_begin + k;
-                int id = __ldg(table + (u * R) / BS);
-                if (id < 0 || id >= a.num_blocks) {
-                    raise_error(a.err, PA_DEVERR_BLOCK_ID);
-                    id = a.num_blocks;
-                }
-                const int rr = (u * R) % BS;
+                auto checked = [&](int id) {
+                    if (id < 0 || id >= a.num_blocks) {
+                        raise_error(a.err, PA_DEVERR_BLOCK_ID);
+                        return a.num_blocks;
+                    }
+                    return id;
+                };
+                // the prefix is whole 16-token units, so both halves of a unit exist
+                const int id = checked(__ldg(table + (u * R) / BS));
+                const int id1 = C::BOX_ROWS < R ? checked(__ldg(table + (u * R) / BS + 1)) : id;
+                const int rr = C::BOX_ROWS < R ? 0 : (u * R) % BS;
                 unsigned char* kdst = smem + s * C::STAGE_BYTES;
                 mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
 #pragma unroll
                 for (int b = 0; b < C::BOXES; ++b) {
-                    tma_load_4d(kdst + b * C::BOX_BYTES, &tm_k, &full[s], b * 64, kvh, rr, id);
-                    tma_load_4d(kdst + C::STAGE_BYTES / 2 + b * C::BOX_BYTES, &tm_v, &full[s],
-                                b * 64, kvh, rr, id);
+                    unsigned char* kb = kdst + b * C::BOX_BYTES;
+                    unsigned char* vb = kb + C::STAGE_BYTES / 2;
+                    tma_load_4d(kb, &tm_k, &full[s], b * 64, kvh, rr, id);
+                    tma_load_4d(vb, &tm_v, &full[s], b * 64, kvh, rr, id);
+                    if (C::BOX_ROWS < R) {
+                        constexpr int OFF = C::BOX_ROWS * 128;     // bytes
+                        tma_load_4d(kb + OFF, &tm_k, &full[s], b * 64, kvh, 0, id1);
+                        tma_load_4d(vb + OFF, &tm_v, &full[s], b * 64, kvh, 0, id1);
+                    }
                 }
             }
         }

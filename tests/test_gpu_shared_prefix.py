@@ -40,7 +40,7 @@ def _prefix_batch(bs, d, aligned):
 
 @pytest.mark.parametrize("aligned", [False, True])
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("bs", [16, 32, 64, 128])
+@pytest.mark.parametrize("bs", [8, 16, 32, 64, 128])
 def test_shared_prefix_workload(bs, d, aligned):
     problem, tables, lens, kc, vc, q, k_ref, v_ref = _prefix_batch(bs, d, aligned)
     # the shared part is the prefix's whole blocks before any copy-on-write
