@@ -214,3 +214,30 @@ def test_head_dim_64_with_odd_and_even_kv_heads(hk, g, bs):
     finally:
         pa.pa_set_option("decode_split_ctas", 0)
     device_clean()
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 256)])
+def test_split_merge_in_chunks_with_a_reused_workspace(dtype, d):
+    """Few (sequence, head) pairs with many partitions: the merge splits each
+    pair's partitions into chunks over several CTAs (some chunks empty for
+    short sequences) and the last to arrive adds them.  Three calls reuse one
+    workspace, so stale arrival counts would show; every call matches the
+    oracle and the calls agree bit for bit."""
+    problem = pa_inputs.random_small(4040 + d, num_seqs=5, max_len=4096, num_heads=8,
+                                     num_kv_heads=2, head_dim=d, block_size=16, dtype=dtype,
+                                     fixed={0: 64, 1: 65, 2: 1100, 3: 4096, 4: 3000})
+    data = pa_inputs.materialize(problem, "cuda")
+    ref = oracle_decode(data, problem)
+    need = pa.pa_decode_split_workspace_bytes(5, 8, d, 4096, 64)
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device="cuda")   # garbage counts
+    outs = []
+    for _ in range(3):
+        out = torch.empty_like(data["q"])
+        pa.pa_decode_split(out, data["q"], data["k_cache"], data["v_cache"],
+                           data["block_tables"], data["context_lens"], problem.scale,
+                           max_context_len=4096, partition_size=64, workspace=ws)
+        torch.cuda.synchronize()
+        assert_close(out, ref)
+        outs.append(out)
+    assert same_bits(outs[0], outs[1]) and same_bits(outs[1], outs[2])
+    device_clean()
