@@ -161,10 +161,10 @@ __device__ __forceinline__ int rank_select(Get&& get, int r, int lane, int& valu
 }
 
 // Fused append: the CTA of (seq, kvh) writes kv head kvh's part of the new
-// token's key and value rows into the cache for later steps.  No load of
-// this launch reads that row (the new token's contribution comes from the
-// input rows, see fold_new_token; the boxes that cover the row mask it), so
-// neither a proxy fence nor a barrier follows.
+// token's key and value rows into the cache, then makes the writes visible
+// to its own TMA loads.  Only this sequence reads the new token's block (a
+// shared block is copied before it is written), so no other CTA can race
+// with the write.  The caller follows with a CTA (or cluster) barrier.
 template <typename T, int D, int BS>
 __device__ __forceinline__ void append_row(const DecodeArgs& a, int seq, int kvh, void* k_cache,
                                            void* v_cache) {
@@ -183,46 +183,7 @@ __device__ __forceinline__ void append_row(const DecodeArgs& a, int seq, int kvh
         const uint4 x = reinterpret_cast<const uint4*>(val ? a.new_v : a.new_k)[src + j];
         reinterpret_cast<uint4*>(val ? v_cache : k_cache)[dst + j] = x;
     }
-}
-
-template <typename T>
-__device__ __forceinline__ float as_float(T x) {
-    if constexpr (std::is_same<T, float>::value)
-        return x;
-    else
-        return __bfloat162float(x);
-}
-
-// The new token's scores s_g = scale * q_g . k_new (log2 units) for the G
-// query heads of kv head kvh, one warp per head, into snew[G].
-template <typename T, int D, int G>
-__device__ __forceinline__ void new_token_scores(const DecodeArgs& a, int seq, int kvh,
-                                                 float* snew, int warp, int nwarps, int lane) {
-    const T* kn = reinterpret_cast<const T*>(a.new_k) + ((size_t)seq * a.num_kv_heads + kvh) * D;
-    for (int g = warp; g < G; g += nwarps) {
-        const T* q = reinterpret_cast<const T*>(a.q) +
-                     ((size_t)seq * a.num_heads + (size_t)kvh * G + g) * D;
-        float acc = 0.f;
-#pragma unroll
-        for (int i = lane; i < D; i += 32) acc = fmaf(as_float(q[i]), as_float(kn[i]), acc);
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(FULL_MASK, acc, off);
-        if (lane == 0) snew[g] = acc * a.scale_log2;
-    }
-}
-
-// Fold the new token (score s in log2 units, value v_new[d]) into a merged
-// (max, numerator, denominator) of the cached tokens.
-template <typename T, int D>
-__device__ __forceinline__ void fold_new_token(const DecodeArgs& a, int seq, int kvh, int d,
-                                               float s, float& big, float& num, float& den) {
-    const T* vn = reinterpret_cast<const T*>(a.new_v) + ((size_t)seq * a.num_kv_heads + kvh) * D;
-    const float mx = fmaxf(big, s);
-    const float e = big == -INFINITY ? 0.f : exp2_approx(big - mx);
-    const float en = exp2_approx(s - mx);
-    num = fmaf(en, as_float(vn[d]), num * e);
-    den = fmaf(en, 1.f, den * e);
-    big = mx;
+    fence_proxy_async_global();
 }
 
 enum class Mode { Decode, Split };
@@ -887,16 +848,15 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             kvh = blockIdx.y;
             L = clamp_len(seq);
             const int ctas = gridDim.x;
-            // the new token (fused append) comes from the input rows, not the cache
-            const bool has_new = a.new_slots && a.new_slots[seq] >= 0 && L > 0;
-            float* snew = reinterpret_cast<float*>(smem + Ly::ORDER_OFFSET);   // [G]
-            if (a.new_slots && blockIdx.x == 0)
-                append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
-            if (has_new && blockIdx.x == 0)
-                new_token_scores<T, D, G>(a, seq, kvh, snew, warp, NW, lane);
-            const int Lc = has_new ? L - 1 : L;
+            if (a.new_slots) {
+                if (blockIdx.x == 0) append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
+                if (ctas > 1)
+                    cg::this_cluster().sync();         // every rank loads after the write
+                else
+                    __syncthreads();
+            }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
-            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, Lc, 0, (Lc + R - 1) / R, ctas, blockIdx.x,
+            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, ctas, blockIdx.x,
                         [&](int g, int d, float big, float num, float den, float* x) {
                             // x: [G] max, [G] sum, [G][D] unnormalised output
                             if (ctas > 1) {
@@ -906,7 +866,6 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                                 }
                                 x[2 * G + g * D + d] = num;
                             } else {
-                                if (has_new) fold_new_token<T, D>(a, seq, kvh, d, snew[g], big, num, den);
                                 store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
                             }
                         });
@@ -928,7 +887,6 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                             num = fmaf(e, rx[2 * G + g * D + d], num);
                             den = fmaf(e, rx[G + g], den);
                         }
-                        if (has_new) fold_new_token<T, D>(a, seq, kvh, d, snew[g], big, num, den);
                         store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
                     }
                 }
@@ -988,20 +946,18 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             seq = pick[0];
             kvh = blockIdx.x % Hk;
             L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
-            // the new token (fused append) comes from the input rows, not the cache
-            const bool has_new = a.new_slots && a.new_slots[seq] >= 0 && L > 0;
-            float* snew = reinterpret_cast<float*>(pick + 2);       // [G]; lens is done with
-            if (a.new_slots) append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
-            if (has_new) new_token_scores<T, D, G>(a, seq, kvh, snew, warp, NW, lane);
-            const int Lc = has_new ? L - 1 : L;
-            const int tok0 = cmin(shared_prefix_of(a, seq), Lc);   // whole 16-token units
+            const int tok0 = cmin(shared_prefix_of(a, seq), L);    // whole 16-token units
+            if (a.new_slots) {
+                append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
+                __syncthreads();                       // the loads below see the new row
+            }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
             const int nchunks = a.group_starts ? (tok0 + a.chunk_tokens - 1) / a.chunk_tokens : 0;
             // chunk weights of the shared pass live after the exchange area
             constexpr int XCH_FLOATS = (NW + 1) * G * (D + 2);
             constexpr int MAX_STAGED_CHUNKS = (Ly::MAIN_REGION / 4 - XCH_FLOATS - G) / (2 * G);
             const bool staged = nchunks > 0 && nchunks <= MAX_STAGED_CHUNKS;
-            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, Lc, tok0 / R, (Lc + R - 1) / R, 1, 0,
+            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, tok0 / R, (L + R - 1) / R, 1, 0,
                         [&](int g, int d, float big, float num, float den, float* x) {
                             if (staged) {
                                 // keep this CTA's own part; merged below with the chunks
@@ -1026,7 +982,6 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                                     den = fmaf(ec, a.ws_l[b + c], den);
                                 }
                             }
-                            if (has_new) fold_new_token<T, D>(a, seq, kvh, d, snew[g], big, num, den);
                             store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
                         });
             if (staged) {
