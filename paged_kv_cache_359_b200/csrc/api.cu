@@ -1,6 +1,7 @@
 // C ABI of libpagedattn.so: argument checks, optional host-side index
 // validation, tensor-map encoding and dispatch to the kernel instances.
 // The public contract of every call is documented in include/pagedattn.h.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -19,16 +20,21 @@ namespace pa {
 namespace {
 
 thread_local std::string g_last_error;
-int g_validate = -1;                 // -1: read PA_VALIDATE on first use
-int g_decode_ctas = 0;               // 0: automatic
-int g_pdl = -1;                      // -1: read PA_PDL on first use (default on)
+// process-wide options, read and set from any host thread
+std::atomic<int> g_validate{-1};     // -1: read PA_VALIDATE on first use
+std::atomic<int> g_decode_ctas{0};   // 0: automatic
+std::atomic<int> g_pdl{-1};          // -1: read PA_PDL on first use (default on)
 
 bool validate_enabled() {
-    if (g_validate < 0) {
-        const char* v = std::getenv("PA_VALIDATE");
-        g_validate = (v && v[0] && v[0] != '0') ? 1 : 0;
+    int v = g_validate.load(std::memory_order_relaxed);
+    if (v < 0) {
+        const char* e = std::getenv("PA_VALIDATE");
+        int want = (e && e[0] && e[0] != '0') ? 1 : 0;
+        // an explicit pa_set_option set since then wins
+        g_validate.compare_exchange_strong(v, want);
+        v = g_validate.load(std::memory_order_relaxed);
     }
-    return g_validate == 1;
+    return v == 1;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -158,11 +164,14 @@ int reduce_chunks(size_t heads, size_t parts) {
 }  // namespace
 
 bool pdl_enabled() {
-    if (g_pdl < 0) {
-        const char* v = std::getenv("PA_PDL");
-        g_pdl = (v && v[0] == '0') ? 0 : 1;
+    int v = g_pdl.load(std::memory_order_relaxed);
+    if (v < 0) {
+        const char* e = std::getenv("PA_PDL");
+        int want = (e && e[0] == '0') ? 0 : 1;
+        g_pdl.compare_exchange_strong(v, want);
+        v = g_pdl.load(std::memory_order_relaxed);
     }
-    return g_pdl == 1;
+    return v == 1;
 }
 
 void add_pdl_attr(cudaLaunchAttribute* attrs, unsigned* n) {
@@ -244,7 +253,7 @@ pa_status pa_set_option(pa_option option, int value) {
 int pa_get_option(pa_option option) {
     switch (option) {
         case PA_OPT_VALIDATE: return validate_enabled() ? 1 : 0;
-        case PA_OPT_DECODE_SPLIT_CTAS: return g_decode_ctas;
+        case PA_OPT_DECODE_SPLIT_CTAS: return g_decode_ctas.load();
         case PA_OPT_PDL: return pdl_enabled() ? 1 : 0;
     }
     return -1;
@@ -370,7 +379,8 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     l.num_kv_heads = num_kv_heads;
     l.block_size = block_size;
     l.group = num_heads / num_kv_heads;
-    l.ctas = g_decode_ctas ? g_decode_ctas
+    const int ctas_opt = g_decode_ctas.load(std::memory_order_relaxed);
+    l.ctas = ctas_opt ? ctas_opt
                            : auto_decode_ctas(num_seqs, num_kv_heads, max_blocks_per_seq,
                                               block_size);
     // one CTA per item: a longest-first grid; several CTAs per item: one
