@@ -21,11 +21,15 @@ Reported line (rank 0):
              over ranks, whole job (all replicas).
   e2e        the same metric through the public API with host buffers: the
              live allocator on the host, pinned H2D copies of each step's
-             q / new K,V / slots / lengths / table, and a D2H read of the
-             step's output, all inside the timed region; uploads and
-             downloads run on their own streams, double-buffered,
-             overlapping the neighbouring steps' kernels as a serving loop
-             would.
+             q / new K,V / slots / lengths / copy-on-write pairs, the table
+             changes applied on the device (pa_update_block_tables), and a
+             D2H read of the step's output, all inside the timed region;
+             uploads and downloads run on their own streams through a ring
+             of three buffer sets, overlapping the neighbouring steps'
+             kernels as a serving loop would.
+  other_configs  (default gqa run, 1 GPU) short device-timed runs of the
+             mha, long-context split and prefix-sharing workloads, each with
+             its kernel's roofline fraction.
   roofline   the decode kernel: algorithmic bytes per launch / mean launch
              time (CUDA events on the launching stream) vs measured HBM GB/s.
   cpu_baseline  the fp64 oracle on the host's cores, bounded sample.
@@ -478,10 +482,9 @@ def run_compaction(loop: DecodeLoop, reps: int = 5):
     t0 = time.perf_counter()
     moves = loop.alloc.compact(target)
     host_ms = (time.perf_counter() - t0) * 1e3
+    n_blocks = (-(-lens // bs)).astype(np.int32)
     t0 = time.perf_counter()
-    n_blocks = -(-lens // bs)
-    for t, n in zip(tables, n_blocks):
-        pa.BlockAllocator.remap(t, int(n), moves)
+    pa.BlockAllocator.remap_batch(tables, n_blocks, moves)
     remap_ms = (time.perf_counter() - t0) * 1e3
     moves_d = torch.from_numpy(moves.astype(np.int64)).to(dev)
     stream = torch.cuda.current_stream()
@@ -505,9 +508,63 @@ def run_compaction(loop: DecodeLoop, reps: int = 5):
     return {"pool_blocks_before": before, "pool_blocks_after": target, "live_blocks": live,
             "moves": len(moves), "released_gb": round((before - target) * blk / 1e9, 3),
             "host_compact_ms": round(host_ms, 3), "host_remap_ms": round(remap_ms, 3),
+            "remapped_tables": int(len(tables)),
             "copy_ms": round(copy_ms, 4),
             "copy_gbs_read_plus_write": round(2 * moved / (copy_ms / 1e3) / 1e9, 1),
             "decode_bits_identical": same}
+
+
+def _config_entry(loop, res, steps, peak, label, kernel):
+    """Kernel and step figures of one short device-timed run."""
+    dec_mean_ms = statistics.fmean(res["dec_ms"])
+    dec_alg = statistics.fmean(res["dec_alg_bytes"])
+    achieved = dec_alg / (dec_mean_ms / 1e3) / 1e9
+    step_ms = res["ms"] / steps
+    e = {"workload": label, "kernel": kernel, "steps": steps,
+         "mean_launch_ms": round(dec_mean_ms, 5), "alg_bytes_per_launch": int(dec_alg),
+         "achieved_gbs": round(achieved, 1), "frac": round(achieved / peak, 4),
+         "ms_per_step": round(step_ms, 5),
+         "value_gbs": round(res["kv_bytes"] / (res["ms"] / 1e3) / 1e9, 1),
+         "clocks_sm_mhz": res["clocks"]["sm_mhz"], "clock_reasons": res["clocks"]["reasons"]}
+    if res["unique"] is not None:
+        # shared prefix blocks are read by every sharer; unique bytes count
+        # each physical block once and are the HBM-bound figure
+        uniq = res["unique"] / steps
+        e["unique_kv_bytes_per_step"] = int(uniq)
+        e["unique_gbs"] = round(uniq / (step_ms / 1e3) / 1e9, 1)
+        e["frac_unique"] = round(e["unique_gbs"] / peak, 4)
+    return e
+
+
+def run_other_configs(dev, local, peak, steps=10, warmup=3):
+    """The other decode workloads, measured briefly after the headline run:
+    MHA batch 64 (fused append + decode), the long-context split at the
+    config's 512-token partitions, and the prefix-sharing batch (block 16,
+    head_dim 128) with plain decode and with the cascade.  Each builds its
+    own pool, runs ``warmup`` + ``steps`` device-timed steps and is freed."""
+    out = []
+    extra = 2 * (steps + warmup) + 4
+
+    def run(build, label, kernel, fused=False, unique=False):
+        loop = build()
+        loop.fused = fused
+        res = run_device_timed(loop, steps, warmup, 1, local, unique=unique)
+        out.append(_config_entry(loop, res, steps, peak, label, kernel))
+        del loop
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        return out[-1]
+
+    run(lambda: DecodeLoop(make_problem("mha", extra, 0), dev, "decode", 512),
+        "mha_decode_b64", "pa_decode_append", fused=True)
+    run(lambda: DecodeLoop(make_problem("long", extra, 0), dev, "split", 512),
+        "long_context_split_p512", "pa_decode_split")
+    plain = run(lambda: build_prefix_loop(dev, extra, "decode", 512, 16, 128),
+                "prefix_sharing_b64_bs16_d128", "pa_decode", unique=True)
+    casc = run(lambda: build_prefix_loop(dev, extra, "cascade", 512, 16, 128),
+               "prefix_sharing_b64_bs16_d128", "pa_decode_shared_prefix", unique=True)
+    casc["speedup_vs_pa_decode"] = round(plain["ms_per_step"] / casc["ms_per_step"], 3)
+    return out
 
 
 def _segments(spec):
@@ -524,29 +581,36 @@ def _view(buf, seg, dtype, shape):
     return buf[off:off + nbytes].view(dtype).view(shape)
 
 
-def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int):
+def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3):
     """Through the public API from host buffers, as a serving loop runs it.
 
     Every step: the host allocator appends a token to every sequence, writing
-    the block table, lengths, slots and copy-on-write pairs straight into a
-    pinned metadata buffer; the step's inputs go host->device from pinned
-    memory (one copy for q and the new K/V rows, one for the metadata); the
-    kernels run; the step's output comes back device->host and is read on the
-    host.  Copies run on a second stream with double-buffered device inputs,
-    so step i+1's upload and step i-1's download overlap step i's kernels; the
-    timed region spans every copy of every timed step."""
+    the lengths, slots and copy-on-write pairs straight into a pinned
+    metadata buffer; the step's inputs go host->device from pinned memory
+    (one copy for q and the new K/V rows, one for the metadata); on the
+    device pa_copy_blocks runs the copy-on-write pairs, pa_update_block_tables
+    applies the step's table changes to the device-resident block tables
+    (one entry per sequence at most, derived from the lengths and slots
+    already uploaded, so the table itself never crosses the link), and the
+    decode runs; the step's output comes back device->host and the host
+    reads it.  A ring of ``ring`` buffer sets lets the host run up to
+    ring - 1 steps ahead of the last completed download: step i's uploads
+    go out as soon as step i - ring has been read back, on their own stream,
+    and downloads have a third stream, so copies overlap the neighbouring
+    steps' kernels.  The timed region spans every copy of every timed step."""
     pa, p, dev = loop.pa, loop.p, loop.device
     total = steps + warmup
     s, cap = loop.tables.shape
     dt = loop.q0.dtype
     esz = loop.q0.element_size()
+    bs = p.block_size
     qshape = (s, p.num_heads, p.head_dim)
     kshape = (s, p.num_kv_heads, p.head_dim)
     in_seg, in_bytes = _segments([("q", s * p.num_heads * p.head_dim * esz),
                                   ("k", s * p.num_kv_heads * p.head_dim * esz),
                                   ("v", s * p.num_kv_heads * p.head_dim * esz)])
-    meta_seg, meta_bytes = _segments([("tables", s * cap * 4), ("lens", s * 4), ("slots", s * 8),
-                                      ("cows", s * 2 * 8)])
+    meta_seg, meta_bytes = _segments([("lens", s * 4), ("slots", s * 8), ("cows", s * 2 * 8)])
+    cow_off = meta_seg["cows"][0]
     host = []
     for st in range(total):
         t = pa_inputs.step_tokens(p.num_seqs, p.num_heads, p.num_kv_heads, p.head_dim, p.dtype,
@@ -556,92 +620,93 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int):
         _view(hb, in_seg["k"], dt, kshape).copy_(t["key"])
         _view(hb, in_seg["v"], dt, kshape).copy_(t["value"])
         host.append(hb)
-    meta_h = torch.zeros(meta_bytes, dtype=torch.uint8).pin_memory()
-    tables_np = _view(meta_h, meta_seg["tables"], torch.int32, (s, cap)).numpy()
-    lens_np = _view(meta_h, meta_seg["lens"], torch.int32, (s,)).numpy()
-    slots_np = _view(meta_h, meta_seg["slots"], torch.int64, (s,)).numpy()
-    cows_np = _view(meta_h, meta_seg["cows"], torch.int64, (s, 2)).numpy()
-    tables_np[:] = loop.tables             # the allocator continues from here, in place
-    lens_np[:] = loop.lens
+    # the allocator works on host tables; the device copy is uploaded once
+    # and from then on only updated on the device
+    tables_np = loop.tables
+    lens_np = loop.lens.copy()
+    tables_d = torch.from_numpy(tables_np).to(dev)
     comp = torch.cuda.current_stream()
     up = torch.cuda.Stream(device=dev)      # host -> device
     down = torch.cuda.Stream(device=dev)    # device -> host, so uploads never queue behind it
-    meta_up = torch.cuda.Event()
 
     class Buf:
         def __init__(self):
             self.inp = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
             self.meta = torch.empty(meta_bytes, dtype=torch.uint8, device=dev)
+            self.meta_h = torch.zeros(meta_bytes, dtype=torch.uint8).pin_memory()
             self.q = _view(self.inp, in_seg["q"], dt, qshape)
             self.k = _view(self.inp, in_seg["k"], dt, kshape)
             self.v = _view(self.inp, in_seg["v"], dt, kshape)
-            self.tables = _view(self.meta, meta_seg["tables"], torch.int32, (s, cap))
             self.lens = _view(self.meta, meta_seg["lens"], torch.int32, (s,))
             self.slots = _view(self.meta, meta_seg["slots"], torch.int64, (s,))
             self.cows = _view(self.meta, meta_seg["cows"], torch.int64, (s, 2))
+            self.lens_h = _view(self.meta_h, meta_seg["lens"], torch.int32, (s,)).numpy()
+            self.slots_h = _view(self.meta_h, meta_seg["slots"], torch.int64, (s,)).numpy()
+            self.cows_h = _view(self.meta_h, meta_seg["cows"], torch.int64, (s, 2)).numpy()
             self.out = torch.empty_like(loop.out)
             self.out_h = torch.empty(tuple(loop.out.shape), dtype=loop.out.dtype).pin_memory()
             self.h2d, self.done, self.d2h = (torch.cuda.Event(), torch.cuda.Event(),
                                              torch.cuda.Event())
             self.used = False
 
-    bufs = [Buf(), Buf()]
+    bufs = [Buf() for _ in range(ring)]
     counts = {"h2d": 0, "d2h": 0, "kv": 0}
-    pending = []
 
-    def read_back(upto_all=False):
-        while pending and (upto_all or len(pending) > 1):
-            b = pending.pop(0)
-            b.d2h.synchronize()
-            float(b.out_h.view(-1)[0])                 # the host reads the result
+    def read_back(b):
+        b.d2h.synchronize()
+        float(b.out_h.view(-1)[0])                     # the host reads the result
+        b.used = False
 
     def step(i, count):
-        b = bufs[i % 2]
-        meta_up.synchronize()                          # last step's metadata upload is done
+        b = bufs[i % ring]
+        if b.used:
+            read_back(b)                               # step i - ring is done with b
         sl, cw = loop.alloc.append_slots(tables_np, lens_np)
-        slots_np[:] = sl
+        b.lens_h[:] = lens_np
+        b.slots_h[:] = sl
         n = len(cw)
         if n:
-            cows_np[:n] = cw
+            b.cows_h[:n] = cw
+        meta_used = cow_off + 16 * n                   # lengths, slots, this step's pairs
         with torch.cuda.stream(up):
-            if b.used:
-                up.wait_event(b.done)                  # step i-2 is done with buffer b
             b.inp.copy_(host[i], non_blocking=True)
-            b.meta.copy_(meta_h, non_blocking=True)
-            meta_up.record(up)
+            b.meta[:meta_used].copy_(b.meta_h[:meta_used], non_blocking=True)
             b.h2d.record(up)
         comp.wait_event(b.h2d)
         if n:
             pa.pa_copy_blocks(loop.k_cache, loop.v_cache, b.cows[:n], stream=comp)
+        pa.pa_update_block_tables(tables_d, b.lens, b.slots, bs, p.num_blocks, stream=comp)
         if loop.fused:
             pa.pa_decode_append(b.out, b.q, b.k, b.v, loop.k_cache, loop.v_cache, b.slots,
-                                b.tables, b.lens, p.scale, stream=comp)
-        elif loop.kernel in ("split", "cascade"):
+                                tables_d, b.lens, p.scale, stream=comp)
+        else:
             pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
             saved_out, loop.out = loop.out, b.out
             with torch.cuda.stream(comp):
-                loop.decode(b.q, b.tables, b.lens, int(lens_np.max()))
+                loop.decode(b.q, tables_d, b.lens, int(lens_np.max()))
             loop.out = saved_out
-        else:
-            pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
-            pa.pa_decode(b.out, b.q, loop.k_cache, loop.v_cache, b.tables, b.lens, p.scale,
-                         stream=comp)
         b.done.record(comp)
         with torch.cuda.stream(down):
             down.wait_event(b.done)
             b.out_h.copy_(b.out, non_blocking=True)
             b.d2h.record(down)
         b.used = True
-        pending.append(b)
-        read_back()
         if count:
-            counts["h2d"] += in_bytes + meta_bytes
+            counts["h2d"] += in_bytes + meta_used
             counts["d2h"] += b.out_h.numel() * b.out_h.element_size()
             counts["kv"] += decode_kv_bytes(lens_np, p)
 
+    def drain():
+        for k in range(ring):                          # oldest first
+            b = bufs[(next_step[0] + k) % ring]
+            if b.used:
+                read_back(b)
+
+    next_step = [0]
     for i in range(warmup):
         step(i, False)
-    read_back(True)
+        next_step[0] = i + 1
+    drain()
     torch.cuda.synchronize()
     barrier(world)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -650,13 +715,20 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int):
     down.wait_event(t0)
     for j in range(steps):
         step(warmup + j, True)
-    for b in pending:
-        comp.wait_event(b.d2h)
+        next_step[0] = warmup + j + 1
+    for b in bufs:
+        if b.used:
+            comp.wait_event(b.d2h)
     t1.record(comp)
-    read_back(True)
+    drain()
     torch.cuda.synchronize()
     barrier(world)
-    loop.tables[:] = tables_np
+    # the device tables must have followed the host allocator exactly
+    n_live = -(-lens_np // bs)
+    got = tables_d.cpu().numpy()
+    for i in range(s):
+        if not (got[i, :n_live[i]] == tables_np[i, :n_live[i]]).all():
+            raise RuntimeError(f"device block table of sequence {i} diverged from the host's")
     loop.lens[:] = lens_np
     return {"ms": t0.elapsed_time(t1), "kv_bytes": counts["kv"], "h2d": counts["h2d"] / steps,
             "d2h": counts["d2h"] / steps}
@@ -703,8 +775,7 @@ def run_reference(args, rank, world):
     import oracle
     if world > 1 and rank != 0:
         return
-    extra = args.steps + args.warmup + 2
-    p = make_problem(args.workload, extra, 0, args.block_size, args.head_dim)
+    p = make_problem(args.workload, pool_headroom_tokens(args), 0, args.block_size, args.head_dim)
     data = pa_inputs.materialize(p, "cpu")
     kc, vc = data["k_cache"], data["v_cache"]
     alloc = oracle.BlockAllocator(p.num_blocks, p.block_size, p.free_order)
@@ -753,6 +824,13 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def pool_headroom_tokens(args) -> int:
+    """Tokens each sequence may grow by during a run: the device-timed loop
+    and the end-to-end loop each append one per step.  Both bench arms size
+    their pool from this, so they run the same configuration."""
+    return 2 * (args.steps + args.warmup) + 4
+
+
 def workload_config(p, args):
     lens = p.context_lens
     return {"workload": {"gqa": "gqa_decode_b256", "mha": "mha_decode_b64",
@@ -790,6 +868,9 @@ def main():
                          "instead of pa_decode_append (the cache write fused into the decode)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the short runs of the mha, long and prefix workloads that the "
+                         "default gqa run appends as other_configs")
     ap.add_argument("--block-size", type=int, default=None,
                     help="gqa / prefix workloads: block size (default 16)")
     ap.add_argument("--head-dim", type=int, default=None,
@@ -838,7 +919,7 @@ def main():
     pa.pa_set_option("pdl", 0 if args.no_pdl else 1)
     dist_init(world, "nccl")
     try:
-        extra = 2 * (args.steps + args.warmup) + 4
+        extra = pool_headroom_tokens(args)
         if args.workload == "prefix":
             loop = build_prefix_loop(dev, extra, args.kernel, args.partition,
                                      args.block_size or 16, args.head_dim or 128)
@@ -904,6 +985,11 @@ def main():
                            "ms_per_step": round(e2e_ms / args.steps, 4)}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(loop)
+        if world == 1 and not args.no_other_configs and default_shape and not args.compact:
+            del loop
+            torch.cuda.empty_cache()
+            line["other_configs"] = run_other_configs(dev, local, peak)
+            loop = None
         if args.compact:                     # last: it frees half the batch
             line["compaction"] = run_compaction(loop)
         if rank == 0:

@@ -79,11 +79,22 @@ enum {
 typedef enum pa_option {
     PA_OPT_VALIDATE = 0,         /* 0/1: host-side index validation before launch */
     PA_OPT_DECODE_SPLIT_CTAS = 1, /* pa_decode CTAs per (sequence, kv head): 0 = auto, 1, 2, 4, 8 */
-    PA_OPT_PDL = 2                /* 0/1 (default 1, or PA_PDL in the environment): launch with
+    PA_OPT_PDL = 2,               /* 0/1 (default 1, or PA_PDL in the environment): launch with
                                      programmatic dependent launch.  Every kernel still waits
                                      for the grid before it on the stream to complete before
                                      touching memory; only the launch and the CTA placement
                                      overlap that grid's tail */
+    PA_OPT_WAIT_LIMIT_US = 3,     /* upper bound, in microseconds, on every pipeline wait inside
+                                     the decode kernels (default 2000000 = 2 s; 100 .. 10000000).
+                                     A wait that runs out sets PA_DEVERR_WAIT_TIMEOUT; the warp
+                                     stops issuing, waits (bounded) for its own loads in flight
+                                     and contributes nothing, so the kernel still ends */
+    PA_OPT_TEST_UNDERFED_STAGES = 4 /* TEST ONLY, 0/1 (default 0): arm every pipeline stage's
+                                     barrier for 16 bytes more than its loads deliver.  Every
+                                     load still lands in the CTA's own shared memory, but no
+                                     stage ever completes, so every wait runs out: this drives
+                                     the timeout path above without a lost load.  Outputs are
+                                     then meaningless (zeros where nothing was merged) */
 } pa_option;
 
 const char* pa_last_error(void);
@@ -160,6 +171,33 @@ pa_status pa_decode_append(void* out_d, const void* q_d, const void* key_d,
                            int max_blocks_per_seq, const int32_t* context_lens_d, int num_seqs,
                            int num_heads, int num_kv_heads, int head_dim, int block_size,
                            int num_blocks, float scale, pa_dtype dtype, pa_stream_t stream);
+
+/*
+ * pa_update_block_tables -- the "update the mapping" step of a decode step
+ * ([csdn-QA] 四 flow: allocate a free page, update the mapping, run the
+ * attention kernel; [course] 2.4.2: a new block only when the last one is
+ * full).  After the host allocator has appended one token to each sequence,
+ * the device copy of the block tables needs at most one new entry per
+ * sequence: the block holding the new token, which is a newly allocated
+ * block, the copy-on-write replacement of a shared last block, or the entry
+ * already there.  This call writes
+ *   block_tables[s, (context_lens[s] - 1) / block_size] = slot_mapping[s] / block_size
+ * for every s with slot_mapping[s] >= 0, so a serving loop keeps the tables
+ * resident on the device and uploads only the lengths and slots it already
+ * sends for the cache write, instead of the whole table.
+ *   block_tables_d   int32 [num_seqs, max_blocks_per_seq] (updated in place)
+ *   context_lens_d   int32 [num_seqs], counting the new token
+ *   slot_mapping_d   int64 [num_seqs], the new token's slot (-1: no token)
+ * Entries a kernel earlier on the stream reads may change (copy-on-write),
+ * so the call belongs on the stream of the decode that follows.  A slot
+ * outside the pool, or a position outside the table, is skipped and sets
+ * PA_DEVERR_SLOT; validate mode also checks that the slot's row is the new
+ * token's row in its block.
+ */
+pa_status pa_update_block_tables(int32_t* block_tables_d, int max_blocks_per_seq,
+                                 const int32_t* context_lens_d, const int64_t* slot_mapping_d,
+                                 int num_seqs, int block_size, int num_blocks,
+                                 pa_stream_t stream);
 
 /*
  * pa_decode_split -- long-context decode in fixed token partitions merged by
@@ -370,6 +408,16 @@ pa_status pa_alloc_compact(pa_allocator* alloc, int target_num_blocks, int32_t* 
 
 /* Replace every entry of a host table that is a move's src by its dst. */
 pa_status pa_seq_remap(int32_t* table, int num_table_blocks, const int32_t* moves, int num_moves);
+
+/* pa_seq_remap for a whole batch in one call ([tech] 2.1: defragmentation
+ * rewrites the block pointers; 4.2 item 2).  tables: host int32
+ * [num_seqs][stride], row s holding lengths_in_blocks[s] live entries (the
+ * rest is left untouched); moves: the (src, dst) pairs pa_alloc_compact
+ * returned.  Every live entry equal to a move's src becomes its dst.
+ * INVALID_ARG (nothing changes) for null arrays, a negative count, a row
+ * longer than stride or a negative block in moves. */
+pa_status pa_seq_remap_batch(int32_t* tables, int stride, const int* lengths_in_blocks,
+                             int num_seqs, const int32_t* moves, int num_moves);
 
 #ifdef __cplusplus
 }

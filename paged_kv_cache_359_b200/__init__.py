@@ -29,11 +29,12 @@ import numpy as np
 import torch
 
 from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SPLIT_CTAS,
-                      PA_OPT_PDL, PA_OPT_VALIDATE, PagedAttnError, check, lib)
+                      PA_OPT_PDL, PA_OPT_TEST_UNDERFED_STAGES, PA_OPT_VALIDATE,
+                      PA_OPT_WAIT_LIMIT_US, PagedAttnError, check, lib)
 
 __all__ = [
     "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_split", "pa_decode_split_workspace_bytes",
-    "pa_decode_split_noalloc", "pa_decode_shared_prefix",
+    "pa_decode_split_noalloc", "pa_decode_shared_prefix", "pa_update_block_tables",
     "pa_decode_shared_prefix_workspace_bytes", "pa_copy_blocks", "pa_swap_blocks",
     "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
     "PagedAttnError", "OutOfBlocks", "DEVERR_BITS",
@@ -41,7 +42,8 @@ __all__ = [
 
 _DTYPES = {torch.float32: PA_DTYPE_F32, torch.bfloat16: PA_DTYPE_BF16}
 _OPTIONS = {"validate": PA_OPT_VALIDATE, "decode_split_ctas": PA_OPT_DECODE_SPLIT_CTAS,
-            "pdl": PA_OPT_PDL}
+            "pdl": PA_OPT_PDL, "wait_limit_us": PA_OPT_WAIT_LIMIT_US,
+            "test_underfed_stages": PA_OPT_TEST_UNDERFED_STAGES}
 
 
 class OutOfBlocks(PagedAttnError):
@@ -210,6 +212,24 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens
         int(max_prefix_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
     return out
+
+
+def pa_update_block_tables(block_tables, context_lens, slot_mapping, block_size, num_blocks,
+                           stream=None):
+    """Device tables int32 [S, max_blocks] updated in place after one append
+    per sequence: entry (context_lens[s] - 1) // block_size becomes
+    slot_mapping[s] // block_size (slot -1: unchanged)."""
+    _dev(block_tables, context_lens, slot_mapping)
+    _need(block_tables.dtype == torch.int32 and block_tables.dim() == 2,
+          "block_tables must be int32 [num_seqs, max_blocks_per_seq]")
+    s = block_tables.shape[0]
+    _need(context_lens.dtype == torch.int32 and context_lens.shape == (s,),
+          "context_lens must be int32 [num_seqs]")
+    _need(slot_mapping.dtype == torch.int64 and slot_mapping.shape == (s,),
+          "slot_mapping must be int64 [num_seqs]")
+    check(lib().pa_update_block_tables(_ptr(block_tables), block_tables.shape[1],
+                                       _ptr(context_lens), _ptr(slot_mapping), s,
+                                       int(block_size), int(num_blocks), _stream(stream)))
 
 
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
@@ -381,3 +401,17 @@ class BlockAllocator:
         """Rewrite a host table in place after a compaction."""
         moves = np.ascontiguousarray(moves, dtype=np.int32)
         check(lib().pa_seq_remap(_i32(table), num_table_blocks, _i32(moves), moves.shape[0]))
+
+    @staticmethod
+    def remap_batch(tables: np.ndarray, lengths_in_blocks: np.ndarray, moves: np.ndarray) -> None:
+        """Rewrite every host table of a batch in place after a compaction:
+        tables int32 [S, stride] (C-contiguous), lengths_in_blocks [S]."""
+        if tables.dtype != np.int32 or tables.ndim != 2 or not tables.flags.c_contiguous:
+            raise ValueError("tables must be a C-contiguous int32 [num_seqs, stride] array")
+        n = np.ascontiguousarray(lengths_in_blocks, dtype=np.intc)
+        if n.shape != (tables.shape[0],):
+            raise ValueError("lengths_in_blocks must hold one count per table row")
+        moves = np.ascontiguousarray(moves, dtype=np.int32)
+        check(lib().pa_seq_remap_batch(_i32(tables), tables.shape[1],
+                                       n.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                       tables.shape[0], _i32(moves), moves.shape[0]))

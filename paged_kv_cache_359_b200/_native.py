@@ -18,6 +18,7 @@ STATUS_NAMES = {
 }
 PA_DTYPE_F32, PA_DTYPE_BF16 = 0, 1
 PA_OPT_VALIDATE, PA_OPT_DECODE_SPLIT_CTAS, PA_OPT_PDL = 0, 1, 2
+PA_OPT_WAIT_LIMIT_US, PA_OPT_TEST_UNDERFED_STAGES = 3, 4
 
 DEVERR_BITS = {
     1: "PA_DEVERR_BLOCK_ID", 2: "PA_DEVERR_CONTEXT_LEN", 4: "PA_DEVERR_WAIT_TIMEOUT",
@@ -55,6 +56,7 @@ SIGNATURES = {
     "pa_decode_shared_prefix": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
                                          _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp,
                                          _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "pa_update_block_tables": (_c_int, [_vp, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp]),
     "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _vp]),
     "pa_swap_blocks": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -76,6 +78,7 @@ SIGNATURES = {
     "pa_seq_free": (_c_int, [_vp, _i32p, _c_int]),
     "pa_alloc_compact": (_c_int, [_vp, _c_int, _i32p, _c_int, _intp]),
     "pa_seq_remap": (_c_int, [_i32p, _c_int, _i32p, _c_int]),
+    "pa_seq_remap_batch": (_c_int, [_i32p, _c_int, _intp, _c_int, _i32p, _c_int]),
 }
 
 

@@ -308,6 +308,35 @@ pa_status pa_seq_remap(int32_t* table, int n, const int32_t* moves, int num_move
     return PA_OK;
 }
 
+pa_status pa_seq_remap_batch(int32_t* tables, int stride, const int* lengths_in_blocks,
+                             int num_seqs, const int32_t* moves, int num_moves) {
+    if (num_seqs < 0 || num_moves < 0 || stride < 0 || (num_seqs > 0 && (!tables || !lengths_in_blocks)) ||
+        (num_moves > 0 && !moves))
+        return pa::fail(PA_ERR_INVALID_ARG, "null argument");
+    for (int s = 0; s < num_seqs; ++s)
+        if (lengths_in_blocks[s] < 0 || lengths_in_blocks[s] > stride)
+            return pa::fail(PA_ERR_INVALID_ARG, "sequence %d: %d table entries, stride %d", s,
+                            lengths_in_blocks[s], stride);
+    // a dense map from every moved block to its new id (moves name blocks of
+    // the pool before compaction, so the largest source bounds its size)
+    int32_t top = -1;
+    for (int i = 0; i < num_moves; ++i) {
+        if (moves[2 * i] < 0 || moves[2 * i + 1] < 0)
+            return pa::fail(PA_ERR_INVALID_ARG, "move %d names a negative block", i);
+        if (moves[2 * i] > top) top = moves[2 * i];
+    }
+    std::vector<int32_t> where((size_t)top + 1, -1);
+    for (int i = 0; i < num_moves; ++i) where[moves[2 * i]] = moves[2 * i + 1];
+    for (int s = 0; s < num_seqs; ++s) {
+        int32_t* t = tables + (size_t)s * stride;
+        for (int j = 0; j < lengths_in_blocks[s]; ++j) {
+            const int32_t b = t[j];
+            if (b >= 0 && b <= top && where[b] >= 0) t[j] = where[b];
+        }
+    }
+    return PA_OK;
+}
+
 pa_status pa_seq_free(pa_allocator* a, const int32_t* table, int n) {
     if (!a || n < 0 || (n > 0 && !table)) return pa::fail(PA_ERR_INVALID_ARG, "null argument");
     // a table may name one block more than once only through misuse; check

@@ -24,6 +24,8 @@ thread_local std::string g_last_error;
 std::atomic<int> g_validate{-1};     // -1: read PA_VALIDATE on first use
 std::atomic<int> g_decode_ctas{0};   // 0: automatic
 std::atomic<int> g_pdl{-1};          // -1: read PA_PDL on first use (default on)
+std::atomic<int> g_wait_us{(int)(WAIT_LIMIT_NS / 1000)};   // limit of every pipeline wait
+std::atomic<int> g_underfed{0};      // test only: stage barriers armed above their loads
 
 bool validate_enabled() {
     int v = g_validate.load(std::memory_order_relaxed);
@@ -150,6 +152,15 @@ pa_status dispatch_decode(const DecodeLaunch& l, pa_dtype dt, int head_dim) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// The device error word and the pipeline-wait settings every decode launch carries.
+pa_status set_error_and_waits(DecodeArgs& args) {
+    args.err = device_error_word();
+    if (!args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    args.wait_ns = 1000ull * (unsigned long long)g_wait_us.load(std::memory_order_relaxed);
+    args.tx_extra = g_underfed.load(std::memory_order_relaxed) ? 16u : 0u;
+    return PA_OK;
+}
+
 // Chunks of partitions per (sequence, head) in the log-sum-exp reduce: enough
 // CTAs to fill the GPU a few times over (a fixed target, so the workspace
 // size does not depend on the device), at least 16 partitions per chunk.
@@ -246,6 +257,12 @@ pa_status pa_set_option(pa_option option, int value) {
                 return fail(PA_ERR_INVALID_ARG, "CTAs per (sequence, kv head) must be 0,1,2,4,8");
             g_decode_ctas = value;
             return PA_OK;
+        case PA_OPT_WAIT_LIMIT_US:
+            if (value < 100 || value > 10000000)
+                return fail(PA_ERR_INVALID_ARG, "wait limit must be 100 .. 10000000 us");
+            g_wait_us = value;
+            return PA_OK;
+        case PA_OPT_TEST_UNDERFED_STAGES: g_underfed = value ? 1 : 0; return PA_OK;
     }
     return fail(PA_ERR_INVALID_ARG, "unknown option %d", (int)option);
 }
@@ -255,6 +272,8 @@ int pa_get_option(pa_option option) {
         case PA_OPT_VALIDATE: return validate_enabled() ? 1 : 0;
         case PA_OPT_DECODE_SPLIT_CTAS: return g_decode_ctas.load();
         case PA_OPT_PDL: return pdl_enabled() ? 1 : 0;
+        case PA_OPT_WAIT_LIMIT_US: return g_wait_us.load();
+        case PA_OPT_TEST_UNDERFED_STAGES: return g_underfed.load();
     }
     return -1;
 }
@@ -359,8 +378,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     l.args.q = q;
     l.args.block_tables = block_tables;
     l.args.context_lens = context_lens;
-    l.args.err = device_error_word();
-    if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    if (pa_status s = set_error_and_waits(l.args)) return s;
     l.args.scale_log2 = scale * 1.4426950408889634f;
     l.args.num_seqs = num_seqs;
     l.args.max_blocks = max_blocks_per_seq;
@@ -485,8 +503,7 @@ pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const v
         l.args.ws_cnt = reinterpret_cast<unsigned*>(
             p + align256(heads * l.args.reduce_chunks * (head_dim + 4) * sizeof(float)));
     }
-    l.args.err = device_error_word();
-    if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    if (pa_status s = set_error_and_waits(l.args)) return s;
     l.args.scale_log2 = scale * 1.4426950408889634f;
     l.args.num_seqs = num_seqs;
     l.args.max_blocks = max_blocks_per_seq;
@@ -588,8 +605,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
     l.args.ws_m = reinterpret_cast<float*>(ws);
     l.args.ws_l = reinterpret_cast<float*>(ws + align256(rows * sizeof(float)));
     l.args.ws_o = reinterpret_cast<float*>(ws + 2 * align256(rows * sizeof(float)));
-    l.args.err = device_error_word();
-    if (!l.args.err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    if (pa_status s = set_error_and_waits(l.args)) return s;
     l.args.scale_log2 = scale * 1.4426950408889634f;
     l.args.num_seqs = num_seqs;
     l.args.max_blocks = max_blocks_per_seq;
@@ -619,6 +635,38 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
     l.consumers = cmin(PrefixCfg<64, 16, 1>::MAX_CONSUMERS, (max_rows + 15) / 16);
     l.stream = st;
     return dispatch_decode(l, dtype, head_dim);
+}
+
+pa_status pa_update_block_tables(int32_t* block_tables, int max_blocks_per_seq,
+                                 const int32_t* context_lens, const int64_t* slot_mapping,
+                                 int num_seqs, int block_size, int num_blocks,
+                                 pa_stream_t stream) {
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || num_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "sizes must be positive (num_seqs >= 0)");
+    if (num_seqs == 0) return PA_OK;
+    if (!block_tables || !context_lens || !slot_mapping)
+        return fail(PA_ERR_INVALID_ARG, "null pointer");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (validate_enabled()) {
+        std::vector<int32_t> l;
+        std::vector<int64_t> sl;
+        if (!copy_to_host(l, context_lens, (size_t)num_seqs, st) ||
+            !copy_to_host(sl, slot_mapping, (size_t)num_seqs, st))
+            return fail(PA_ERR_CUDA, "validation copy failed");
+        for (int s = 0; s < num_seqs; ++s) {
+            if (sl[s] < 0) continue;
+            if (sl[s] >= (int64_t)num_blocks * block_size || l[s] <= 0 ||
+                (l[s] - 1) / block_size >= max_blocks_per_seq)
+                return fail(PA_ERR_BAD_BLOCK_ID, "sequence %d: slot %lld, length %d", s,
+                            (long long)sl[s], l[s]);
+            if (sl[s] % block_size != (l[s] - 1) % block_size)
+                return fail(PA_ERR_BAD_BLOCK_ID,
+                            "sequence %d: slot %lld is not at row %d of a block", s,
+                            (long long)sl[s], (l[s] - 1) % block_size);
+        }
+    }
+    return launch_update_tables(block_tables, max_blocks_per_seq, context_lens, slot_mapping,
+                                num_seqs, block_size, num_blocks, st);
 }
 
 pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,

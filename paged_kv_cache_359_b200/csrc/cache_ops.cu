@@ -73,7 +73,49 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// The mapping update of one decode step: sequence s's newest token (position
+// context_lens[s] - 1) sits in slot slot_mapping[s], so table entry
+// (context_lens[s] - 1) / block_size becomes slot / block_size -- a new
+// block, a copy-on-write replacement, or the entry it already holds.
+__global__ void __launch_bounds__(256)
+    update_tables_kernel(int32_t* __restrict__ tables, int stride,
+                         const int32_t* __restrict__ lens, const int64_t* __restrict__ slots,
+                         int num_seqs, int block_size, int num_blocks, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= num_seqs) return;
+    const int64_t slot = slots[s];
+    if (slot < 0) return;
+    const int pos = lens[s] - 1;
+    const int64_t blk = slot / block_size;
+    if (pos < 0 || pos / block_size >= stride || blk >= num_blocks) {
+        raise_error(err, PA_DEVERR_SLOT);
+        return;
+    }
+    tables[(size_t)s * stride + pos / block_size] = (int32_t)blk;
+}
+
 }  // namespace
+
+pa_status launch_update_tables(int32_t* tables, int stride, const int32_t* lens,
+                               const int64_t* slots, int num_seqs, int block_size,
+                               int num_blocks, cudaStream_t stream) {
+    if (num_seqs == 0) return PA_OK;
+    unsigned* err = device_error_word();
+    if (!err) return fail(PA_ERR_CUDA, "device error word unavailable");
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((num_seqs + 255) / 256);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    add_pdl_attr(attr, &cfg.numAttrs);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, update_tables_kernel, tables, stride, lens, slots,
+                                       num_seqs, block_size, num_blocks, err);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "table update launch: %s", cudaGetErrorString(e));
+    return PA_OK;
+}
 
 unsigned* device_error_word() {
     static unsigned* cached[64] = {};

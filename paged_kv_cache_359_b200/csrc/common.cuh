@@ -12,9 +12,10 @@ namespace pa {
 
 constexpr unsigned FULL_MASK = 0xffffffffu;
 
-// Upper bound on any single pipeline wait.  A TMA load that has not landed
-// after this long is treated as lost: the kernel records
-// PA_DEVERR_WAIT_TIMEOUT, stops issuing, and finishes with what it has.
+// Default upper bound on any single pipeline wait (PA_OPT_WAIT_LIMIT_US sets
+// another).  A TMA load that has not landed after this long is treated as
+// lost: the kernel records PA_DEVERR_WAIT_TIMEOUT, stops issuing, and
+// finishes with what it has.
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;   // 2 s
 
 // ---------------------------------------------------------------- dtypes --
@@ -99,16 +100,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for `parity` of `bar`, giving up after WAIT_LIMIT_NS.  Returns false
-// on timeout.  Every caller treats a timeout as an error and stops issuing.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+// Wait for `parity` of `bar`, giving up after `limit_ns`.  Returns false on
+// timeout.  Every caller treats a timeout as an error and stops issuing.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
 }
 

@@ -76,6 +76,11 @@ struct DecodeArgs {
     unsigned* ws_cnt;             // [S * Hq]
     int reduce_chunks;
     unsigned* err;                // device error word
+    unsigned long long wait_ns;   // limit of every pipeline wait
+    // test-only (PA_OPT_TEST_UNDERFED_STAGES): extra bytes armed on every
+    // stage barrier beyond what its loads deliver, so its phase never
+    // completes and each wait runs out; 0 in normal use
+    unsigned tx_extra;
     float scale_log2;             // scale * log2(e)
     int num_seqs;
     int max_blocks;
@@ -665,8 +670,9 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
         const int uu = first + ustride * k;
         const int row0 = HALVES == 2 ? 0 : (uu * R) % U::BS;
         const bool second = HALVES == 2 && id1 >= 0;
-        mbar_arrive_expect_tx(&cx.bars[s], HALVES == 1 || second ? Ly::STAGE_BYTES
-                                                                 : Ly::STAGE_BYTES / 2);
+        mbar_arrive_expect_tx(&cx.bars[s], (HALVES == 1 || second ? Ly::STAGE_BYTES
+                                                                  : Ly::STAGE_BYTES / 2) +
+                                               a.tx_extra);
 #pragma unroll
         for (int b = 0; b < U::BOXES; ++b) {
             T* kb = kdst + b * R * U::BOX_INNER;
@@ -698,7 +704,7 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
     for (; k < nk; ++k) {
         const int s = slot(k);
         const uint32_t parity = ((cx.ring + k) / DEPTH) & 1;
-        const bool landed = __all_sync(FULL_MASK, mbar_wait_bounded(&cx.bars[s], parity));
+        const bool landed = __all_sync(FULL_MASK, mbar_wait_bounded(&cx.bars[s], parity, a.wait_ns));
         if (!landed) {
             failed = true;
             break;
@@ -724,7 +730,7 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
         if (lane == 0) raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
         const int issued = cmin(nk, k + DEPTH);
         for (int kk = k + 1; kk < issued; ++kk)
-            (void)mbar_wait_bounded(&cx.bars[slot(kk)], ((cx.ring + kk) / DEPTH) & 1);
+            (void)mbar_wait_bounded(&cx.bars[slot(kk)], ((cx.ring + kk) / DEPTH) & 1, a.wait_ns);
         u.drop();
         // keep the ring's phase bookkeeping consistent with what was issued
         cx.ring += issued;

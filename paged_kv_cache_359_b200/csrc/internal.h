@@ -53,6 +53,9 @@ pa_status launch_decode_bf16_d256(const DecodeLaunch& l);
 pa_status launch_reshape_and_cache(const void* key, const void* value, void* k_cache,
                                    void* v_cache, const int64_t* slots, int num_tokens,
                                    int64_t row_bytes, int64_t num_slots, cudaStream_t stream);
+pa_status launch_update_tables(int32_t* tables, int stride, const int32_t* lens,
+                               const int64_t* slots, int num_seqs, int block_size,
+                               int num_blocks, cudaStream_t stream);
 pa_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping, int num_pairs,
                              int64_t block_bytes, int num_blocks, cudaStream_t stream);
 pa_status launch_move_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,

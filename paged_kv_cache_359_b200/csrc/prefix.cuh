@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS)
             for (int k = 0; k < nk; ++k) {
                 const int s = k % STAGES;
                 if (k >= STAGES &&
-                    !mbar_wait_bounded(&empty[s], ((k / STAGES) - 1) & 1)) {
+                    !mbar_wait_bounded(&empty[s], ((k / STAGES) - 1) & 1, a.wait_ns)) {
                     raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
                     break;                  // consumers time out on `full` and finish
                 }
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS)
                 const int id1 = C::BOX_ROWS < R ? checked(__ldg(table + (u * R) / BS + 1)) : id;
                 const int rr = C::BOX_ROWS < R ? 0 : (u * R) % BS;
                 unsigned char* kdst = smem + s * C::STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES + a.tx_extra);
 #pragma unroll
                 for (int b = 0; b < C::BOXES; ++b) {
                     unsigned char* kb = kdst + b * C::BOX_BYTES;
@@ -166,11 +166,11 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS)
     bool failed = false;
     for (int k = 0; k < nk; ++k) {
         const int s = k % STAGES;
-        if (!__all_sync(FULL_MASK, mbar_wait_bounded(&full[s], (k / STAGES) & 1))) {
+        if (!__all_sync(FULL_MASK, mbar_wait_bounded(&full[s], (k / STAGES) & 1, a.wait_ns))) {
             if (lane == 0) raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
             // later stages the producer may have issued: bounded waits
             for (int kk = k + 1; kk < cmin(nk, k + STAGES); ++kk)
-                (void)mbar_wait_bounded(&full[kk % STAGES], (kk / STAGES) & 1);
+                (void)mbar_wait_bounded(&full[kk % STAGES], (kk / STAGES) & 1, a.wait_ns);
             failed = true;
             break;
         }

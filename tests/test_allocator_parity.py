@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 
 import oracle
-from paged_kv_cache_359_b200 import BlockAllocator, OutOfBlocks
+from paged_kv_cache_359_b200 import BlockAllocator, OutOfBlocks, PagedAttnError
 
 
 def same_state(c, o):
@@ -173,6 +173,16 @@ def test_compaction_matches_the_oracle(seed):
     cm = c.compact(target)
     om = oracle.compact(o, target)
     assert [tuple(m) for m in cm.tolist()] == om
+    # the batch call on a copy of the kept tables (entries past each row's
+    # length stay untouched), then the per-table call
+    batch = np.stack([ctabs[i] for i in keep])
+    nblk = np.array([-(-lens[i] // bs) for i in keep], dtype=np.int32)
+    tail = [batch[r, n:].copy() for r, n in enumerate(nblk)]
+    BlockAllocator.remap_batch(batch, nblk, cm)
+    for r, i in enumerate(keep):
+        n = int(nblk[r])
+        assert list(batch[r, :n]) == oracle.remap(otabs[i], om)
+        assert (batch[r, n:] == tail[r]).all()
     for i in keep:
         n = -(-lens[i] // bs)
         BlockAllocator.remap(ctabs[i], n, cm)
@@ -188,3 +198,9 @@ def test_compaction_matches_the_oracle(seed):
     t = np.array([0, 5, 7], dtype=np.int32)
     BlockAllocator.remap(t, 3, np.array([[7, 2], [9, 1]], dtype=np.int32))
     assert list(t) == [0, 5, 2]
+    tb = np.array([[0, 5, 7], [9, 7, 9]], dtype=np.int32)
+    BlockAllocator.remap_batch(tb, np.array([3, 2]), np.array([[7, 2], [9, 1]], dtype=np.int32))
+    assert tb.tolist() == [[0, 5, 2], [1, 2, 9]]
+    with pytest.raises(PagedAttnError):        # a row longer than the stride changes nothing
+        BlockAllocator.remap_batch(tb, np.array([3, 4]), np.array([[0, 1]], dtype=np.int32))
+    assert tb.tolist() == [[0, 5, 2], [1, 2, 9]]

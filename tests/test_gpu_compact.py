@@ -68,9 +68,14 @@ def test_compaction_preserves_decode_bits(bs, hq, hk, d, dt):
     torch.cuda.synchronize()
     assert same_bits(kc[:target], ref_k[:target]) and same_bits(vc[:target], ref_v[:target])
 
-    for t, ln in zip(tables, lens):
+    # every table in one call; the per-table call must agree with it
+    batch = np.stack(tables)
+    nblk = np.array([-(-ln // bs) for ln in lens], dtype=np.int32)
+    BlockAllocator.remap_batch(batch, nblk, moves)
+    for r, (t, ln) in enumerate(zip(tables, lens)):
         BlockAllocator.remap(t, -(-ln // bs), moves)
         assert t[: -(-ln // bs)].max() < target
+        assert (t[: nblk[r]] == batch[r, : nblk[r]]).all()
     kc[target:] = float("nan")                        # the released tail
     vc[target:] = float("nan")
     out1 = torch.empty_like(q)

@@ -4,6 +4,15 @@ serving process with a fixed budget and no allocation after start-up).  It
 must give what pa_decode_split gives with a caller workspace, call after
 call, although every call reuses the library's one built-in scratch array.
 
+Each call is checked against the oracle at the attention tolerance and
+against pa_decode_split with a caller workspace bit for bit: both run the
+same kernels, and the merge adds partitions in a fixed order, so a stale or
+misplaced partial left in the shared scratch by an earlier call would show
+as a bit difference even where it stays inside the tolerance.  The calls
+change shape from one to the next, and two of them split the merge of each
+(sequence, head) into several chunks, whose arrival counts and per-chunk
+sums live in the scratch across calls.
+
 This file is collected last, so a stop-at-first-failure run has already run
 every other test; it also passes on its own in a fresh process."""
 
@@ -16,9 +25,11 @@ import torch
 import pa_inputs
 import paged_kv_cache_359_b200 as pa
 from paged_kv_cache_359_b200 import _native
-from gpu_common import assert_close, device_clean
+from gpu_common import assert_close, device_clean, oracle_decode, same_bits
 
 pytestmark = pytest.mark.gpu
+
+SCRATCH = 16 * 1024 * 1024
 
 
 def _noalloc(out, data, problem, max_len, partition):
@@ -35,26 +46,44 @@ def _noalloc(out, data, problem, max_len, partition):
     _native.check(status)
 
 
-@pytest.mark.parametrize("seeds", [(41, 42)])
-def test_noalloc_matches_caller_workspace_two_calls_in_a_row(seeds):
-    for call, seed in enumerate(seeds):
-        problem = pa_inputs.random_small(seed, num_seqs=5, max_len=2500 + 700 * call,
+def _merge_chunks(num_seqs, num_heads, parts):
+    """Chunks per (sequence, head) of the split merge: the library's rule
+    (about 600 merge CTAs, at least 16 partitions per chunk), restated so
+    the test can say which calls take the chunked path."""
+    heads = num_seqs * num_heads
+    return max(1, min(-(-600 // heads), -(-parts // 16)))
+
+
+# (seed, sequences, longest length, partition): the first call merges in one
+# chunk per head, the second in four (64 partitions of 256 tokens), the
+# third in one again at another shape, the fourth in several again with
+# other lengths, so each call inherits the scratch in another layout.
+CALLS = [(41, 5, 2500, 256), (43, 2, 16384, 256), (42, 5, 3200, 512), (44, 3, 12000, 256)]
+
+
+def test_noalloc_matches_oracle_and_caller_workspace_call_after_call():
+    chunked = 0
+    for seed, num_seqs, max_len, partition in CALLS:
+        problem = pa_inputs.random_small(seed, num_seqs=num_seqs, max_len=max_len,
                                          num_heads=32, num_kv_heads=8, head_dim=128,
-                                         block_size=16, dtype="bf16", fixed={0: 1})
+                                         block_size=16, dtype="bf16",
+                                         fixed={0: 1, 1: max_len})
         data = pa_inputs.materialize(problem, "cuda")
-        max_len = int(problem.context_lens.max())
-        partition = 256
-        need = pa.pa_decode_split_workspace_bytes(5, 32, 128, max_len, partition)
-        assert need <= 16 * 1024 * 1024            # fits the built-in scratch
+        longest = int(problem.context_lens.max())
+        need = pa.pa_decode_split_workspace_bytes(num_seqs, 32, 128, longest, partition)
+        assert need <= SCRATCH                     # fits the built-in scratch
+        chunked += _merge_chunks(num_seqs, 32, -(-longest // partition)) > 1
         expect = torch.empty_like(data["q"])
         pa.pa_decode_split(expect, data["q"], data["k_cache"], data["v_cache"],
                            data["block_tables"], data["context_lens"], problem.scale,
-                           max_len, partition)
+                           longest, partition)
         got = torch.full_like(data["q"], float("nan"))
-        _noalloc(got, data, problem, max_len, partition)
+        _noalloc(got, data, problem, longest, partition)
         torch.cuda.synchronize()
-        assert_close(got, expect.double().cpu())
         device_clean()
+        assert same_bits(got, expect), (seed, num_seqs, max_len, partition)
+        assert_close(got, oracle_decode(data, problem))
+    assert chunked >= 2                            # the chunked merge ran through the scratch
 
 
 def test_noalloc_rejects_batches_beyond_the_scratch():
