@@ -225,6 +225,23 @@ pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, i
     return PA_OK;
 }
 
+pa_status encode_query_map(CUtensorMap* map, const void* q, int head_dim, int num_heads,
+                           int num_seqs, int heads, int seqs) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_heads, (cuuint64_t)num_seqs};
+    cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)num_heads * head_dim * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)heads, (cuuint32_t)seqs};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", (int)r);
+    return PA_OK;
+}
+
 }  // namespace pa
 
 using namespace pa;
@@ -529,7 +546,8 @@ pa_status pa_decode_split(void* out, const void* q, const void* k_cache, const v
 size_t pa_decode_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                                int max_prefix_len) {
     if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_prefix_len < 0) return 0;
-    const size_t chunks = (size_t)((max_prefix_len + PREFIX_CHUNK_TOKENS - 1) / PREFIX_CHUNK_TOKENS);
+    const int ct = prefix_chunk_tokens(head_dim);
+    const size_t chunks = (size_t)((max_prefix_len + ct - 1) / ct);
     const size_t rows = (size_t)num_seqs * num_heads * (chunks ? chunks : 1);
     return 2 * align256(rows * sizeof(float)) + rows * head_dim * sizeof(float);
 }
@@ -593,7 +611,8 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
             }
         }
     }
-    const int chunks = (max_prefix_len + PREFIX_CHUNK_TOKENS - 1) / PREFIX_CHUNK_TOKENS;
+    const int chunk_tokens = prefix_chunk_tokens(head_dim);
+    const int chunks = (max_prefix_len + chunk_tokens - 1) / chunk_tokens;
     const int group = num_heads / num_kv_heads;
     const size_t rows = (size_t)num_seqs * num_heads * (size_t)(chunks ? chunks : 1);
     char* ws = static_cast<char*>(workspace);
@@ -616,7 +635,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
     l.args.group_starts = group_starts;
     l.args.group_prefix = prefix_lens;
     l.args.num_groups = num_groups;
-    l.args.chunk_tokens = PREFIX_CHUNK_TOKENS;
+    l.args.chunk_tokens = chunk_tokens;
     l.args.prefix_slot0 = 0;
     l.args.slot_stride = chunks ? chunks : 1;
     l.args.sched = SCHED_LPT;
@@ -632,7 +651,6 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
     l.max_chunks = chunks;
     const int max_rows = max_group_size * group;
     l.row_blocks = (max_rows + PREFIX_ROWS_PER_CTA - 1) / PREFIX_ROWS_PER_CTA;
-    l.consumers = cmin(PrefixCfg<64, 16, 1>::MAX_CONSUMERS, (max_rows + 15) / 16);
     l.stream = st;
     return dispatch_decode(l, dtype, head_dim);
 }

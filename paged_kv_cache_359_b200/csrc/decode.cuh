@@ -772,7 +772,15 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
     using Ly = Layout<U>;
     constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
     constexpr int NT = NW * 32;
-    pdl_wait();
+    // The own-token pass of the shared-prefix decode reads nothing the
+    // shared pass (the grid just before it) writes until its final merge:
+    // its inputs come from grids that completed before the shared pass got
+    // past its own wait.  It therefore streams its tokens first and waits for
+    // the shared pass only before the merge, so the two overlap where SMs
+    // are free; every CTA still waits before it leaves, which keeps the
+    // stream's completion order.  Every other launch waits here.
+    const bool late_wait = MODE == Mode::Decode && a.sched == SCHED_LPT && a.group_starts;
+    if (!late_wait) pdl_wait();
     pdl_launch_dependents();
 
     extern __shared__ unsigned char smem_raw[];
@@ -976,6 +984,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                             }
                             if (nchunks) {
                                 // merge with the shared pass's chunks of this head
+                                pdl_wait();
                                 const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0;
                                 float mm = big;
                                 for (int c = 0; c < nchunks; ++c) mm = fmaxf(mm, a.ws_m[b + c]);
@@ -990,6 +999,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                             }
                             store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
                         });
+            pdl_wait();                                // the shared pass is complete
             if (staged) {
                 // merge this CTA's part with the shared pass's chunks: chunk
                 // maxima and sums staged once, weights once per head, then

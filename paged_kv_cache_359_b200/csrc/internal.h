@@ -29,6 +29,13 @@ pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, i
                            int num_kv_heads, int block_size, int num_blocks, int box_inner,
                            int rows, bool swizzle128);
 
+// Encode a 3-D tensor map over bf16 queries [num_seqs][num_heads][head_dim]
+// with a {64, heads, seqs} box and the 128-byte swizzle: `heads` consecutive
+// query heads of `seqs` consecutive sequences, one 128-byte row per (sequence,
+// head), sequence-major.
+pa_status encode_query_map(CUtensorMap* map, const void* q, int head_dim, int num_heads,
+                           int num_seqs, int heads, int seqs);
+
 // Device error word of the current device (address from cudaGetSymbolAddress).
 unsigned* device_error_word();
 

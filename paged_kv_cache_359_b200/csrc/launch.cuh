@@ -22,11 +22,10 @@ struct DecodeLaunch {
     int ctas;          // pa_decode: CTAs (one cluster) per (sequence, kv head)
     bool split;
     // shared-prefix decode: the shared pass runs first (grid max_chunks x Hk x
-    // groups * row_blocks, `consumers` + 1 warps), then the split pass
+    // groups * row_blocks), then pa_decode's kernel over the own tokens
     bool cascade;
     int max_chunks;
     int row_blocks;
-    int consumers;
     cudaStream_t stream;
 };
 
@@ -76,9 +75,10 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
             static std::atomic<unsigned long long> done_p{0};
             auto pk = shared_prefix_kernel<D, BS, G>;
             if (pa_status s = allow_smem(pk, C::SMEM_BYTES, done_p)) return s;
-            // all of L1 as shared memory, so two CTAs fit an SM
-            cudaFuncSetAttribute(pk, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-            CUtensorMap sk, sv;        // 128B-swizzled {64, 1, 16 or 8, 1} boxes
+            CUtensorMap sq, sk, sv;    // 128B-swizzled boxes: q {64, G, 128 / G}, K/V {64, 1, 16 or 8, 1}
+            if (pa_status s = encode_query_map(&sq, l.args.q, D, l.args.num_heads, l.num_seqs,
+                                               G, C::M / G))
+                return s;
             if (pa_status s = encode_cache_map(&sk, l.k_cache, DT, D, l.num_kv_heads, BS,
                                                l.args.num_blocks, 64, C::BOX_ROWS, true))
                 return s;
@@ -88,13 +88,13 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
             if (l.max_chunks > 0) {
                 cudaLaunchConfig_t pc = {};
                 pc.gridDim = dim3(l.max_chunks, l.num_kv_heads, l.args.num_groups * l.row_blocks);
-                pc.blockDim = dim3((l.consumers + 1) * 32);
+                pc.blockDim = dim3(C::THREADS);
                 pc.dynamicSmemBytes = C::SMEM_BYTES;
                 pc.stream = l.stream;
                 cudaLaunchAttribute pattr[1];
                 pc.attrs = pattr;
                 add_pdl_attr(pattr, &pc.numAttrs);
-                e = cudaLaunchKernelEx(&pc, pk, sk, sv, l.args, l.row_blocks);
+                e = cudaLaunchKernelEx(&pc, pk, sq, sk, sv, l.args, l.row_blocks);
                 if (e != cudaSuccess)
                     return fail(PA_ERR_CUDA, "shared-prefix launch: %s", cudaGetErrorString(e));
             }

@@ -1,4 +1,5 @@
-// Shared-prefix pass of the cascade decode (sm_100a, bf16).
+// Shared-prefix pass of the cascade decode on the 5th-generation tensor
+// cores (sm_100a, bf16).
 //
 // Sequences forked from one prompt share its blocks ("vLLM内存管理与
 // PagedAttention精讲" ch.2 §2.4.3: several requests' block tables point at
@@ -6,19 +7,31 @@
 // item 8: shared prefix pages).  Plain decode re-reads those blocks once per
 // sharer.  Here the members of a group attend over the shared prefix
 // together: the query rows of all members (members x G heads of one kv
-// head) form the M side of a real dense contraction, so each prefix tile is
-// read from HBM once per kv head (the row blocks of one chunk run together
-// and share it through L2) instead of once per sequence.
+// head) form the M side of a dense contraction, so each prefix tile is read
+// from HBM once per kv head (once per 128 query rows from L2) instead of
+// once per sequence.
 //
-// CTA = (prefix chunk of 256 tokens, kv head, group x 64-row block).  One
-// producer warp streams the chunk's 16-token units with TMA into a ring of
-// STAGES shared-memory stages (full / empty mbarriers, bounded waits); up to
-// 4 consumer warps each own 16 query rows (two CTAs fit an SM) and run
-//   S[16 x 16] = Q K^T,  O[16 x D] += P V
-// with mma.sync m16n8k16 (bf16 in, fp32 accumulate), an online softmax with
-// a lazy running max, and write the chunk's (max, sum, unnormalised output)
-// per row to the workspace slot prefix_slot0 + chunk; pa_decode's CTAs for
-// each sequence's own tokens merge them into the output.
+// CTA = (prefix chunk of CH tokens, kv head, group x 128-row block); CH is
+// 256 (head_dim <= 128) or 128 (head_dim 256).  Roles:
+//  * producer warp: TMA loads of the CTA's 128 query rows (a 3-D box over
+//    q [S][Hq][D]: members x G heads, row = member * G + head), the chunk's K
+//    tiles in groups of 64 tokens, then its V tiles, all 128-byte swizzled;
+//    a unit past the prefix is loaded from outside the pool map, which TMA
+//    fills with zeros;
+//  * MMA warp (one elected thread): S = Q K^T into TMEM (M = 128 rows,
+//    N = 64 tokens per group as its K tiles land, K = head_dim), commit;
+//    then, once P is in shared memory, O = P V into TMEM (M = 128,
+//    N = head_dim, K = CH tokens, V read MN-major), commit;
+//  * four softmax warps, one TMEM lane (query row) per thread: the exact
+//    maximum of the row's scores over the chunk (masked past the prefix),
+//    p = 2^(s * scale * log2 e - max) rounded to bf16 into the swizzled P tile
+//    (which reuses the K tile's space), the fp32 sum of p; after the second
+//    MMA, the row's unnormalised output, maximum and sum go to the workspace
+//    slot prefix_slot0 + chunk, which pa_decode's CTAs for each sequence's
+//    own tokens merge into the output.
+// Every wait is bounded; a wait that runs out sets PA_DEVERR_WAIT_TIMEOUT,
+// the CTA skips what depends on it, waits (bounded) for its own loads and
+// MMAs, frees its TMEM and leaves without writing.
 #pragma once
 
 #include "decode.cuh"
@@ -28,250 +41,288 @@ namespace pa {
 template <int D_, int BS_, int G_>
 struct PrefixCfg {
     static constexpr int D = D_, BS = BS_, G = G_;
-    static constexpr int R = 16;                 // tokens per unit
-    // 8-token blocks: a unit's rows 0..7 and 8..15 are two 8-row boxes from
-    // consecutive table entries, the second one swizzle atom further on
-    static constexpr int BOX_ROWS = BS < R ? BS : R;
-    static constexpr int BOXES = D / 64;         // 128-byte swizzled boxes per tile
-    static constexpr int BOX_BYTES = R * 128;
-    static constexpr int KS = D / 16, NT = D / 8;
-    static constexpr int STAGE_BYTES = 2 * R * D * 2;
-    static constexpr int STAGES = D >= 256 ? 4 : 8;
-    static constexpr int MAX_CONSUMERS = 4;      // 64 query rows per CTA: two CTAs per SM
-    static constexpr int THREADS = (MAX_CONSUMERS + 1) * 32;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * STAGES * 8 + 1024;
+    static constexpr int R = 16;                       // tokens per unit (one or two TMA boxes)
+    static constexpr int BOX_ROWS = BS < R ? BS : R;   // 8-token blocks: two boxes per unit
+    static constexpr int CH = D <= 128 ? 256 : 128;    // chunk tokens
+    static constexpr int U = CH / R;                   // units per chunk
+    static constexpr int NG = CH / 64;                 // 64-token groups (S MMAs, K barriers)
+    static constexpr int KSL = D / 64;                 // 64-dim slabs of a 128-byte-swizzled tile
+    static constexpr int M = 128;                      // query rows per CTA
+    static constexpr int Q_BYTES = KSL * M * 128;
+    static constexpr int KV_BYTES = KSL * CH * 128;
+    static constexpr int P_BYTES = NG * M * 128;
+    static constexpr int KP_BYTES = KV_BYTES > P_BYTES ? KV_BYTES : P_BYTES;
+    static constexpr int Q_OFF = 0, K_OFF = Q_BYTES, V_OFF = Q_BYTES + KP_BYTES;
+    static constexpr int BAR_OFF = V_OFF + KV_BYTES;
+    // q_full, k_full[NG], v_full, s_full, p_full, o_full; then the TMEM address
+    static constexpr int NBARS = NG + 5;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;   // + alignment slack
+    static constexpr int TMEM_COLS = 512;             // S at column 0, O at column CH
+    static constexpr int THREADS = 6 * 32;            // 4 softmax warps, producer, MMA
     static_assert((BS % R == 0 || BS == 8) && D % 64 == 0, "shared-prefix shape");
+    static_assert(CH + D <= TMEM_COLS, "S and O must fit TMEM");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-constexpr int PREFIX_CHUNK_TOKENS = 256;
-constexpr int PREFIX_ROWS_PER_CTA = 64;
+constexpr int PREFIX_ROWS_PER_CTA = 128;
+
+// Tokens per prefix chunk (one CTA's share of the shared prefix).
+__host__ __device__ constexpr int prefix_chunk_tokens(int head_dim) {
+    return head_dim <= 128 ? 256 : 128;
+}
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// byte offset of 16-byte chunk `chunk` (of D/8) in row `row` of a swizzled tile
-__device__ __forceinline__ uint32_t swz128(int row, int chunk) {
-    return (uint32_t)((chunk >> 3) * (16 * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
-}
-
 template <int D, int BS, int G>
-__global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS)
-    shared_prefix_kernel(const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
+    shared_prefix_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a,
                          int row_blocks) {
+    using C = PrefixCfg<D, BS, G>;
+    constexpr int R = C::R, CH = C::CH, NG = C::NG, KSL = C::KSL, M = C::M;
     pdl_wait();
     pdl_launch_dependents();
-    using C = PrefixCfg<D, BS, G>;
-    constexpr int R = C::R, STAGES = C::STAGES, KS = C::KS, NT = C::NT;
     const int chunk = blockIdx.x, kvh = blockIdx.y;
     const int grp = blockIdx.z / row_blocks, rblk = blockIdx.z % row_blocks;
     const int gs = __ldg(a.group_starts + grp), ge = __ldg(a.group_starts + grp + 1);
     const int prefix = __ldg(a.group_prefix + grp);
     const int rows = (ge - gs) * G;
-    const int row0 = rblk * PREFIX_ROWS_PER_CTA;
+    const int row0 = rblk * M;
     const int nunits = prefix / R;
-    const int u_begin = chunk * (a.chunk_tokens / R);
-    const int u_end = cmin(u_begin + a.chunk_tokens / R, nunits);
-    if (u_begin >= u_end || row0 >= rows) return;     // whole CTA, before any barrier
-    const int nk = u_end - u_begin;
-    const int consumers = (blockDim.x / 32) - 1;
+    const int u_begin = chunk * C::U;
+    const int u_end = cmin(u_begin + C::U, nunits);
+    if (u_begin >= u_end || row0 >= rows) return;       // whole CTA, before any barrier
+    const int valid = (u_end - u_begin) * R;             // tokens of this chunk in the prefix
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-    uint64_t* empty = full + STAGES;
+    unsigned char* qs = smem + C::Q_OFF;
+    unsigned char* ks = smem + C::K_OFF;                  // K tiles, then P
+    unsigned char* vs = smem + C::V_OFF;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;                          // [NG]
+    uint64_t* v_full = bars + 1 + NG;
+    uint64_t* s_full = v_full + 1;
+    uint64_t* p_full = v_full + 2;
+    uint64_t* o_full = v_full + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+    // set by a role that gave up, read by the others after the final barrier
+    __shared__ int failed;
+
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], consumers);
-        }
+        failed = 0;
+        for (int i = 0; i < C::NBARS; ++i) mbar_init(&bars[i], i == NG + 3 ? 128 : 1);
         fence_mbar_init();
     }
+    if (warp == 5) {                                      // the MMA warp owns TMEM
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
     __syncthreads();
-    // the members share their first prefix / BS table entries: read the first member's
-    const int32_t* table = a.block_tables + (size_t)gs * a.max_blocks;
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t s_tmem = tmem, o_tmem = tmem + CH;
 
-    if (warp == consumers) {
-        // ---------------- producer warp: lane 0 streams the chunk's units ----------------
+    if (warp == 4) {
+        // ------------------------------------------------ producer (lane 0) --
         if (lane == 0) {
-            for (int k = 0; k < nk; ++k) {
-                const int s = k % STAGES;
-                if (k >= STAGES &&
-                    !mbar_wait_bounded(&empty[s], ((k / STAGES) - 1) & 1, a.wait_ns)) {
-                    raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
-                    break;                  // consumers time out on `full` and finish
+            prefetch_tensormap(&tm_q);
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            // the members share their first prefix / BS table entries: read the first member's
+            const int32_t* table = a.block_tables + (size_t)gs * a.max_blocks;
+            auto checked = [&](int id) {
+                if (id < 0 || id >= a.num_blocks) {
+                    raise_error(a.err, PA_DEVERR_BLOCK_ID);
+                    return a.num_blocks;          // outside the map: TMA fills zeros
                 }
-                const int u = u_begin + k;
-                auto checked = [&](int id) {
-                    if (id < 0 || id >= a.num_blocks) {
-                        raise_error(a.err, PA_DEVERR_BLOCK_ID);
-                        return a.num_blocks;
-                    }
-                    return id;
-                };
-                // the prefix is whole 16-token units, so both halves of a unit exist
-                const int id = checked(__ldg(table + (u * R) / BS));
-                const int id1 = C::BOX_ROWS < R ? checked(__ldg(table + (u * R) / BS + 1)) : id;
-                const int rr = C::BOX_ROWS < R ? 0 : (u * R) % BS;
-                unsigned char* kdst = smem + s * C::STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES + a.tx_extra);
+                return id;
+            };
+            mbar_arrive_expect_tx(q_full, C::Q_BYTES + a.tx_extra);
 #pragma unroll
-                for (int b = 0; b < C::BOXES; ++b) {
-                    unsigned char* kb = kdst + b * C::BOX_BYTES;
-                    unsigned char* vb = kb + C::STAGE_BYTES / 2;
-                    tma_load_4d(kb, &tm_k, &full[s], b * 64, kvh, rr, id);
-                    tma_load_4d(vb, &tm_v, &full[s], b * 64, kvh, rr, id);
-                    if (C::BOX_ROWS < R) {
-                        constexpr int OFF = C::BOX_ROWS * 128;     // bytes
-                        tma_load_4d(kb + OFF, &tm_k, &full[s], b * 64, kvh, 0, id1);
-                        tma_load_4d(vb + OFF, &tm_v, &full[s], b * 64, kvh, 0, id1);
+            for (int b = 0; b < KSL; ++b)
+                tma_load_3d(qs + b * M * 128, &tm_q, q_full, 64 * b, kvh * G, gs + row0 / G);
+            // unit j of the chunk lands at row 16 j of every 64-dim slab
+            auto load_unit = [&](const CUtensorMap* map, unsigned char* base, uint64_t* bar,
+                                 int j) {
+                const int u = u_begin + j;
+                int id = a.num_blocks, id1 = a.num_blocks, rr = 0;
+                if (u < u_end) {                    // the prefix is whole 16-token units
+                    id = checked(__ldg(table + (u * R) / BS));
+                    if (C::BOX_ROWS < R) id1 = checked(__ldg(table + (u * R) / BS + 1));
+                    else rr = (u * R) % BS;
+                }
+#pragma unroll
+                for (int b = 0; b < KSL; ++b) {
+                    unsigned char* dst = base + b * CH * 128 + j * R * 128;
+                    tma_load_4d(dst, map, bar, 64 * b, kvh, rr, id);
+                    if (C::BOX_ROWS < R)
+                        tma_load_4d(dst + C::BOX_ROWS * 128, map, bar, 64 * b, kvh, 0, id1);
+                }
+            };
+            for (int g = 0; g < NG; ++g) {
+                mbar_arrive_expect_tx(&k_full[g], 4 * KSL * R * 128 + a.tx_extra);
+                for (int j = 4 * g; j < 4 * g + 4; ++j) load_unit(&tm_k, ks, &k_full[g], j);
+            }
+            mbar_arrive_expect_tx(v_full, C::KV_BYTES + a.tx_extra);
+            for (int j = 0; j < C::U; ++j) load_unit(&tm_v, vs, v_full, j);
+        }
+    } else if (warp == 5) {
+        // --------------------------------------------- MMA issuer (lane 0) --
+        if (lane == 0) {
+            const uint32_t q0 = smem_addr(qs), k0 = smem_addr(ks), v0 = smem_addr(vs);
+            bool ok = mbar_wait_bounded(q_full, 0, a.wait_ns);
+            bool s_issued = false;
+            if (ok) {
+                for (int g = 0; g < NG && ok; ++g) {
+                    ok = mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < 4 * KSL; ++kk) {
+                        const uint64_t ad = sw128_desc(q0 + (kk / 4) * M * 128 + (kk % 4) * 32,
+                                                       16, 1024);
+                        const uint64_t bd = sw128_desc(
+                            k0 + (kk / 4) * CH * 128 + g * 64 * 128 + (kk % 4) * 32, 16, 1024);
+                        umma_bf16(s_tmem + 64 * g, ad, bd, umma_idesc_bf16(M, 64, false),
+                                  kk > 0);
                     }
+                }
+                if (ok) {
+                    umma_commit(s_full);
+                    s_issued = true;
                 }
             }
+            bool o_issued = false;
+            if (ok) ok = mbar_wait_bounded(p_full, 0, a.wait_ns) &&
+                         mbar_wait_bounded(v_full, 0, a.wait_ns);
+            if (ok) {
+                tc_fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < CH / 16; ++kk) {
+                    const uint64_t ad =
+                        sw128_desc(k0 + (kk / 4) * M * 128 + (kk % 4) * 32, 16, 1024);
+                    // V as B, MN-major: 64-dim slabs CH * 128 bytes apart (leading
+                    // offset), 8-token atoms 1 KiB apart (stride offset)
+                    const uint64_t bd = sw128_desc(v0 + kk * 16 * 128, CH * 128, 1024);
+                    umma_bf16(o_tmem, ad, bd, umma_idesc_bf16(M, D, true), kk > 0);
+                }
+                umma_commit(o_full);
+                o_issued = true;
+            }
+            if (!ok) {
+                raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+                failed = 1;
+            }
+            // nothing this thread issued may still run when TMEM is freed
+            if (o_issued) (void)mbar_wait_bounded(o_full, 0, a.wait_ns);
+            else if (s_issued) (void)mbar_wait_bounded(s_full, 0, a.wait_ns);
         }
-        return;
+    } else {
+        // -------------------------------- softmax and epilogue: warps 0-3 --
+        const int r = 32 * warp + lane;                   // this thread's query row / TMEM lane
+        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+        float m = -INFINITY, l = 0.f;
+        bool ok = __all_sync(FULL_MASK, mbar_wait_bounded(s_full, 0, a.wait_ns));
+        if (ok) {
+            tc_fence_after_sync();
+            // pass 1: the row's maximum over the chunk's prefix tokens (log2 units)
+#pragma unroll 1
+            for (int c = 0; c < CH / 32; ++c) {
+                float v[32];
+                tmem_ld32(s_tmem + lane_off + 32 * c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (32 * c + j < valid) m = fmaxf(m, v[j] * a.scale_log2);
+            }
+            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum of p
+            const uint32_t prow = smem_addr(ks) + (uint32_t)r * 128;
+#pragma unroll 1
+            for (int c = 0; c < CH / 32; ++c) {
+                float v[32];
+                tmem_ld32(s_tmem + lane_off + 32 * c, v);
+                tmem_ld_wait();
+                uint32_t w[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int t = 32 * c + 2 * j;
+                    const float p0 = t < valid ? exp2_approx(v[2 * j] * a.scale_log2 - m) : 0.f;
+                    const float p1 =
+                        t + 1 < valid ? exp2_approx(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
+                    l += p0 + p1;
+                    w[j] = pack_bf16x2(p0, p1);
+                }
+                // tokens 32c .. 32c+31: slab c / 2, 16-byte chunks 4 (c % 2) .. + 3
+                const uint32_t base = prow + (uint32_t)(c / 2) * (M * 128);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int ch = 4 * (c % 2) + q;
+                    const uint32_t addr = base + (uint32_t)((ch ^ (r & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]),
+                                 "r"(w[4 * q + 3])
+                                 : "memory");
+                }
+            }
+            fence_proxy_async_smem();                   // P is read by the tensor cores
+            tc_fence_before_sync();
+            mbar_arrive(p_full);
+            ok = __all_sync(FULL_MASK, mbar_wait_bounded(o_full, 0, a.wait_ns));
+        }
+        if (!ok) {
+            if (lane == 0) {
+                raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+                failed = 1;
+            }
+        } else {
+            tc_fence_after_sync();
+            const int row = row0 + r;
+            const bool mine = row < rows;
+            const int seq = gs + row / G, h = kvh * G + row % G;
+            const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride +
+                                a.prefix_slot0 + chunk;
+            float* dst = a.ws_o + slot * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float v[32];
+                tmem_ld32(o_tmem + lane_off + 32 * c, v);
+                tmem_ld_wait();
+                if (mine) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        reinterpret_cast<float4*>(dst + 32 * c)[j] =
+                            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+            }
+            if (mine) {
+                a.ws_m[slot] = m;
+                a.ws_l[slot] = l;
+            }
+        }
     }
 
-    // ---------------- consumer warps: 16 query rows each ----------------
-    // rows r0 = lane/4 and r1 = r0 + 8 of this warp's tile; row r -> member r / G, head r % G
-    const int wrow = row0 + 16 * warp;
-    const int r0 = wrow + (lane >> 2), r1 = r0 + 8;
-    const int c2 = 2 * (lane & 3);
-    const bool v0 = r0 < rows, v1 = r1 < rows;
-    auto qrow = [&](int r) {
-        const int seq = gs + r / G, h = kvh * G + r % G;
-        return reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                                                 ((size_t)seq * a.num_heads + h) * D);
-    };
-    uint32_t qa[KS][4];
-    {
-        const uint32_t* q0 = v0 ? qrow(r0) : nullptr;
-        const uint32_t* q1 = v1 ? qrow(r1) : nullptr;
-#pragma unroll
-        for (int k = 0; k < KS; ++k) {
-            qa[k][0] = v0 ? __ldg(q0 + (16 * k + c2) / 2) : 0u;
-            qa[k][1] = v1 ? __ldg(q1 + (16 * k + c2) / 2) : 0u;
-            qa[k][2] = v0 ? __ldg(q0 + (16 * k + 8 + c2) / 2) : 0u;
-            qa[k][3] = v1 ? __ldg(q1 + (16 * k + 8 + c2) / 2) : 0u;
-        }
+    // ---------------- teardown: every role is done with TMEM and shared memory --
+    tc_fence_before_sync();
+    __syncthreads();
+    if (failed && warp == 4 && lane == 0) {
+        // loads may still be in flight after a role gave up: wait (bounded) for them
+        (void)mbar_wait_bounded(q_full, 0, a.wait_ns);
+        for (int g = 0; g < NG; ++g) (void)mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
+        (void)mbar_wait_bounded(v_full, 0, a.wait_ns);
     }
-    float o[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    const int mi = lane >> 3, rr = lane & 7;
-    bool failed = false;
-    for (int k = 0; k < nk; ++k) {
-        const int s = k % STAGES;
-        if (!__all_sync(FULL_MASK, mbar_wait_bounded(&full[s], (k / STAGES) & 1, a.wait_ns))) {
-            if (lane == 0) raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
-            // later stages the producer may have issued: bounded waits
-            for (int kk = k + 1; kk < cmin(nk, k + STAGES); ++kk)
-                (void)mbar_wait_bounded(&full[kk % STAGES], (kk / STAGES) & 1, a.wait_ns);
-            failed = true;
-            break;
-        }
-        const uint32_t kb = smem_addr(smem + s * C::STAGE_BYTES);
-        const uint32_t vb = kb + C::STAGE_BYTES / 2;
-        // S = Q K^T for 16 rows x 16 tokens
-        // two accumulators per n-tile (even / odd k-steps) halve the dependent chain
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-            float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
-            const int tok = 8 * (mi >> 1) + rr;
-#pragma unroll
-            for (int kk = 0; kk < KS; ++kk) {
-                uint32_t b[4];
-                ldmatrix_x4(b, kb + swz128(tok, 2 * kk + (mi & 1)));
-                float(&u0)[4] = (kk & 1) ? t0 : s0;
-                float(&u1)[4] = (kk & 1) ? t1 : s1;
-                mma_bf16_16816(u0, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b[0], b[1]);
-                mma_bf16_16816(u1, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b[2], b[3]);
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                s0[j] += t0[j];
-                s1[j] += t1[j];
-            }
-        }
-        // rows r0: s0[0..1], s1[0..1]; rows r1: s0[2..3], s1[2..3] (log2 units)
-        float x0[4] = {s0[0] * a.scale_log2, s0[1] * a.scale_log2, s1[0] * a.scale_log2,
-                       s1[1] * a.scale_log2};
-        float x1[4] = {s0[2] * a.scale_log2, s0[3] * a.scale_log2, s1[2] * a.scale_log2,
-                       s1[3] * a.scale_log2};
-        const float mx0 = fmaxf(fmaxf(x0[0], x0[1]), fmaxf(x0[2], x0[3]));
-        const float mx1 = fmaxf(fmaxf(x1[0], x1[1]), fmaxf(x1[2], x1[3]));
-        if (__any_sync(FULL_MASK, mx0 > m0 + RESCALE_THRESHOLD || mx1 > m1 + RESCALE_THRESHOLD)) {
-            float a0 = mx0, a1 = mx1;
-            a0 = fmaxf(a0, __shfl_xor_sync(FULL_MASK, a0, 1));
-            a0 = fmaxf(a0, __shfl_xor_sync(FULL_MASK, a0, 2));
-            a1 = fmaxf(a1, __shfl_xor_sync(FULL_MASK, a1, 1));
-            a1 = fmaxf(a1, __shfl_xor_sync(FULL_MASK, a1, 2));
-            const float n0 = fmaxf(m0, a0), n1 = fmaxf(m1, a1);
-            const float al0 = exp2_approx(m0 - n0), al1 = exp2_approx(m1 - n1);
-            m0 = n0;
-            m1 = n1;
-            l0 *= al0;
-            l1 *= al1;
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                o[n][0] *= al0;
-                o[n][1] *= al0;
-                o[n][2] *= al1;
-                o[n][3] *= al1;
-            }
-        }
-        float p0[4], p1[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            p0[j] = exp2_approx(x0[j] - m0);
-            p1[j] = exp2_approx(x1[j] - m1);
-            l0 += p0[j];
-            l1 += p1[j];
-        }
-        const uint32_t pa0 = pack_bf16x2(p0[0], p0[1]), pa1 = pack_bf16x2(p1[0], p1[1]);
-        const uint32_t pa2 = pack_bf16x2(p0[2], p0[3]), pa3 = pack_bf16x2(p1[2], p1[3]);
-        // O += P V
-        {
-            const int tok = 8 * (mi & 1) + rr;
-#pragma unroll
-            for (int j = 0; j < NT / 2; ++j) {
-                uint32_t b[4];
-                ldmatrix_x4_trans(b, vb + swz128(tok, 2 * j + (mi >> 1)));
-                mma_bf16_16816(o[2 * j], pa0, pa1, pa2, pa3, b[0], b[1]);
-                mma_bf16_16816(o[2 * j + 1], pa0, pa1, pa2, pa3, b[2], b[3]);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+    if (warp == 5) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, C::TMEM_COLS);
     }
-    if (failed) {
-        // the error word says so; wait (bounded) for stages the producer may
-        // still have in flight, then leave without writing anything
-        return;
-    }
-    l0 += __shfl_xor_sync(FULL_MASK, l0, 1);
-    l0 += __shfl_xor_sync(FULL_MASK, l0, 2);
-    l1 += __shfl_xor_sync(FULL_MASK, l1, 1);
-    l1 += __shfl_xor_sync(FULL_MASK, l1, 2);
-    const int slot_in = a.prefix_slot0 + chunk;
-    auto write_row = [&](int r, float mm, float ll, int half) {
-        const int seq = gs + r / G, h = kvh * G + r % G;
-        const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride + slot_in;
-        if ((lane & 3) == 0) {
-            a.ws_m[slot] = mm;
-            a.ws_l[slot] = ll;
-        }
-        float* dst = a.ws_o + slot * D + c2;
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-            *reinterpret_cast<float2*>(dst + 8 * n) = make_float2(o[n][2 * half], o[n][2 * half + 1]);
-    };
-    if (v0) write_row(r0, m0, l0, 0);
-    if (v1) write_row(r1, m1, l1, 1);
+    if (failed) __syncthreads();                          // keep shared memory until the drain
 }
 
 }  // namespace pa
