@@ -385,9 +385,12 @@ class DecodeLoop:
 
 
 def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_index: int,
-                     unique: bool = False):
+                     unique: bool = False, graph: bool = False):
     """Allocator outputs for every step are computed up front and uploaded;
-    the timed region holds only device work on inputs resident in HBM."""
+    the timed region holds only device work on inputs resident in HBM.
+    graph: the timed steps are captured once into a CUDA graph (after the
+    eager warm-up) and the graph is replayed once inside the timed region,
+    which runs exactly the same launches without the host's issue cost."""
     pa, p, dev = loop.pa, loop.p, loop.device
     total = steps + warmup
     slots, cows, tabs, lens = [], [], [], []
@@ -417,25 +420,39 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
         if not loop.fused:
             pa.pa_reshape_and_cache(keys[i], vals[i], loop.k_cache, loop.v_cache, slots_d[i])
         if timed_index is not None:
-            dec_ev[timed_index][0].record(stream)
+            dec_ev[timed_index][0].record()            # the current (or capturing) stream
         if loop.fused:
             pa.pa_decode_append(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
                                 slots_d[i], tabs_d[i], lens_d[i], p.scale)
         else:
             loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
         if timed_index is not None:
-            dec_ev[timed_index][1].record(stream)
+            dec_ev[timed_index][1].record()
 
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
+    g = None
+    if graph:
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap):
+                for j in range(steps):
+                    step(warmup + j, j)
+        stream.wait_stream(cap)
+        torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev_index) as clocks:
         t0.record(stream)
-        for j in range(steps):
-            step(warmup + j, j)
+        if g is not None:
+            g.replay()
+        else:
+            for j in range(steps):
+                step(warmup + j, j)
         t1.record(stream)
         clocks.sample()                # the host is ahead: the GPU is still in the region
         torch.cuda.synchronize()
@@ -846,6 +863,8 @@ def workload_config(p, args):
             "kernel": args.kernel + ("+append (fused)" if args.fused else ""),
             "partition": args.partition,
             "pdl": not getattr(args, "no_pdl", False),
+            "timed_steps": "one CUDA graph replay" if getattr(args, "graph", False)
+                           else "eager launches",
             "l2": "inputs larger than L2 (KV cache %.2f GB vs 126 MB L2), no flush" %
                   (decode_kv_bytes(lens, p) / 1e9)}
 
@@ -875,6 +894,9 @@ def main():
                     help="gqa / prefix workloads: block size (default 16)")
     ap.add_argument("--head-dim", type=int, default=None,
                     help="gqa / prefix workloads: head_dim (default 128)")
+    ap.add_argument("--graph", action="store_true",
+                    help="device-timed loop: capture the timed steps in one CUDA graph and "
+                         "replay it (same launches, no host issue cost between them)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (PA_OPT_PDL 0)")
     ap.add_argument("--compact", action="store_true",
@@ -929,7 +951,7 @@ def main():
             loop = DecodeLoop(p, dev, args.kernel, args.partition)
         loop.fused = args.fused
         res = run_device_timed(loop, args.steps, args.warmup, world, local,
-                               unique=args.workload == "prefix")
+                               unique=args.workload == "prefix", graph=args.graph)
         e2e = None if args.no_e2e else run_e2e(loop, args.steps, args.warmup, world)
 
         ms = reduce_scalar(res["ms"], "max", world, dev)

@@ -917,13 +917,17 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             // barrier, above that the CTA stages them in shared memory.
             const int S = a.num_seqs, Hk = a.num_kv_heads;
             const int r = blockIdx.x / Hk;
-            int* pick = reinterpret_cast<int*>(smem + Ly::ORDER_OFFSET);   // sequence, its tokens
-            int* lens = pick + 2;                                           // S <= MAX_SORT
-            auto own_tokens = [&](int i) {
+            // sequence, tokens this pass reads, context length, shared prefix
+            int* pick = reinterpret_cast<int*>(smem + Ly::ORDER_OFFSET);
+            int* lens = pick + 4;                                           // S <= MAX_SORT
+            auto clamped_len = [&](int i) {
                 const int x = a.context_lens[i];
                 if (x < 0 || x > a.max_tokens) raise_error(a.err, PA_DEVERR_CONTEXT_LEN);
-                const int len = x < 0 ? 0 : (x > a.max_tokens ? a.max_tokens : x);
-                // order by the tokens this pass reads (own tokens with a shared prefix)
+                return x < 0 ? 0 : (x > a.max_tokens ? a.max_tokens : x);
+            };
+            // order by the tokens this pass reads (own tokens with a shared prefix)
+            auto own_tokens = [&](int i) {
+                const int len = clamped_len(i);
                 return len - cmin(shared_prefix_of(a, i), len);
             };
             constexpr int REG_PER_LANE = 8;
@@ -934,15 +938,28 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             }
             if (warp == 0) {
                 int found = r, tokens = -1;                  // natural order beyond MAX_SORT
+                int len_of = 0, pre_of = 0;
                 if (in_regs) {
-                    int v[REG_PER_LANE];
+                    int v[REG_PER_LANE], ln[REG_PER_LANE], pr[REG_PER_LANE];
 #pragma unroll
                     for (int j = 0; j < REG_PER_LANE; ++j) {
                         const int i = lane + 32 * j;
-                        v[j] = i < S ? own_tokens(i) : -1;
+                        ln[j] = i < S ? clamped_len(i) : 0;
+                        pr[j] = i < S ? cmin(shared_prefix_of(a, i), ln[j]) : 0;
+                        v[j] = i < S ? ln[j] - pr[j] : -1;
                     }
                     found = rank_select<REG_PER_LANE>([&](int j) { return v[j]; }, r, lane,
                                                       tokens);
+                    // the lane holding the picked entry hands over its length and
+                    // prefix, which saves two dependent loads after the pick
+#pragma unroll
+                    for (int j = 0; j < REG_PER_LANE; ++j)
+                        if (j == (found >> 5)) {
+                            len_of = ln[j];
+                            pre_of = pr[j];
+                        }
+                    len_of = __shfl_sync(FULL_MASK, len_of, found & 31);
+                    pre_of = __shfl_sync(FULL_MASK, pre_of, found & 31);
                 } else if (S <= MAX_SORT) {
                     found = rank_select<MAX_SORT / 32>(
                         [&](int j) {
@@ -954,27 +971,33 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                 if (lane == 0) {
                     pick[0] = found;
                     pick[1] = tokens;
+                    pick[2] = len_of;
+                    pick[3] = pre_of;
                 }
             }
             __syncthreads();
             seq = pick[0];
             kvh = blockIdx.x % Hk;
-            L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
-            const int tok0 = cmin(shared_prefix_of(a, seq), L);    // whole 16-token units
+            int tok0;                                   // whole 16-token units
+            if (in_regs) {
+                L = pick[2];
+                tok0 = pick[3];
+            } else {
+                L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
+                tok0 = cmin(shared_prefix_of(a, seq), L);
+            }
             if (a.new_slots) {
                 append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
                 __syncthreads();                       // the loads below see the new row
             }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
             const int nchunks = a.group_starts ? (tok0 + a.chunk_tokens - 1) / a.chunk_tokens : 0;
-            // chunk weights of the shared pass live after the exchange area
-            constexpr int XCH_FLOATS = (NW + 1) * G * (D + 2);
-            constexpr int MAX_STAGED_CHUNKS = (Ly::MAIN_REGION / 4 - XCH_FLOATS - G) / (2 * G);
-            const bool staged = nchunks > 0 && nchunks <= MAX_STAGED_CHUNKS;
+            // x: this CTA's own part, [G] max, [G] sum, [G][D] unnormalised output,
+            // kept after the exchange area when it is merged with prefix chunks
+            float* x = reinterpret_cast<float*>(smem) + NW * G * (D + 2);
             run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, tok0 / R, (L + R - 1) / R, 1, 0,
-                        [&](int g, int d, float big, float num, float den, float* x) {
-                            if (staged) {
-                                // keep this CTA's own part; merged below with the chunks
+                        [&](int g, int d, float big, float num, float den, float*) {
+                            if (nchunks) {
                                 if (d == 0) {
                                     x[g] = big;
                                     x[G + g] = den;
@@ -982,63 +1005,30 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                                 x[2 * G + g * D + d] = num;
                                 return;
                             }
-                            if (nchunks) {
-                                // merge with the shared pass's chunks of this head
-                                pdl_wait();
-                                const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0;
-                                float mm = big;
-                                for (int c = 0; c < nchunks; ++c) mm = fmaxf(mm, a.ws_m[b + c]);
-                                const float e = big == -INFINITY ? 0.f : exp2_approx(big - mm);
-                                num *= e;
-                                den *= e;
-                                for (int c = 0; c < nchunks; ++c) {
-                                    const float ec = exp2_approx(a.ws_m[b + c] - mm);
-                                    num = fmaf(ec, a.ws_o[(b + c) * D + d], num);
-                                    den = fmaf(ec, a.ws_l[b + c], den);
-                                }
-                            }
                             store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
                         });
             pdl_wait();                                // the shared pass is complete
-            if (staged) {
-                // merge this CTA's part with the shared pass's chunks: chunk
-                // maxima and sums staged once, weights once per head, then
-                // every output's chunk loads issued independently
-                float* x = reinterpret_cast<float*>(smem) + NW * G * (D + 2);
-                float* cw = x + 2 * G + G * D;           // [G][nchunks] weights, then sums
-                float* cl = cw + G * nchunks;
-                float* tot = cl + G * nchunks;           // [G] own weight, then total sum
-                __syncthreads();
-                for (int i = threadIdx.x; i < G * nchunks; i += NT) {
-                    const int g = i / nchunks, c = i % nchunks;
-                    const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0 + c;
-                    cw[i] = a.ws_m[b];
-                    cl[i] = a.ws_l[b];
-                }
-                __syncthreads();
-                if (threadIdx.x < G) {
-                    const int g = threadIdx.x;
-                    float mm = x[g];
-                    for (int c = 0; c < nchunks; ++c) mm = fmaxf(mm, cw[g * nchunks + c]);
-                    const float e0 = x[g] == -INFINITY ? 0.f : exp2_approx(x[g] - mm);
-                    float den = e0 * x[G + g];
-                    for (int c = 0; c < nchunks; ++c) {
-                        const float ec = exp2_approx(cw[g * nchunks + c] - mm);
-                        cw[g * nchunks + c] = ec;
-                        den = fmaf(ec, cl[g * nchunks + c], den);
-                    }
-                    tot[g] = e0;
-                    x[G + g] = den;
-                }
-                __syncthreads();
+            if (nchunks) {
+                // merge with the shared pass's chunks of each head: every thread
+                // reads the chunk maxima and sums of the head it writes (one
+                // address across the warp's lanes of that head) and its own
+                // outputs' chunk values; no load depends on another's value
+                // beyond the maxima, so this costs about two L2 round trips
+                __syncthreads();                       // x is complete
                 for (int idx = threadIdx.x; idx < G * D; idx += NT) {
                     const int g = idx / D, d = idx % D;
                     const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0;
-                    float num = tot[g] * x[2 * G + g * D + d];
+                    float mm = x[g];
 #pragma unroll 8
-                    for (int c = 0; c < nchunks; ++c)
-                        num = fmaf(cw[g * nchunks + c], a.ws_o[(b + c) * D + d], num);
-                    const float den = x[G + g];
+                    for (int c = 0; c < nchunks; ++c) mm = fmaxf(mm, a.ws_m[b + c]);
+                    const float e0 = x[g] == -INFINITY ? 0.f : exp2_approx(x[g] - mm);
+                    float num = e0 * x[2 * G + g * D + d], den = e0 * x[G + g];
+#pragma unroll 8
+                    for (int c = 0; c < nchunks; ++c) {
+                        const float ec = exp2_approx(a.ws_m[b + c] - mm);
+                        num = fmaf(ec, a.ws_o[(b + c) * D + d], num);
+                        den = fmaf(ec, a.ws_l[b + c], den);
+                    }
                     store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
                 }
             }

@@ -22,13 +22,16 @@
 //    N = 64 tokens per group as its K tiles land, K = head_dim), commit;
 //    then, once P is in shared memory, O = P V into TMEM (M = 128,
 //    N = head_dim, K = CH tokens, V read MN-major), commit;
-//  * four softmax warps, one TMEM lane (query row) per thread: the exact
-//    maximum of the row's scores over the chunk (masked past the prefix),
-//    p = 2^(s * scale * log2 e - max) rounded to bf16 into the swizzled P tile
-//    (which reuses the K tile's space), the fp32 sum of p; after the second
-//    MMA, the row's unnormalised output, maximum and sum go to the workspace
-//    slot prefix_slot0 + chunk, which pa_decode's CTAs for each sequence's
-//    own tokens merge into the output.
+//  * eight softmax warps, two per TMEM lane quarter: a thread holds half of
+//    one query row's scores in registers (one TMEM read), the two halves
+//    exchange their maxima through shared memory, and each writes
+//    p = 2^(s * scale * log2 e - max), rounded to bf16, into its half of the
+//    swizzled P tile (which reuses the K tile's space) and sums p in fp32;
+//    after the second MMA each thread stages its half of the row's output in
+//    the (now free) shared memory, and the warps write whole 512-byte rows
+//    to the workspace slot prefix_slot0 + chunk with coalesced stores, with
+//    the row's maximum and sum; pa_decode's CTAs for each sequence's own
+//    tokens merge these into the output.
 // Every wait is bounded; a wait that runs out sets PA_DEVERR_WAIT_TIMEOUT,
 // the CTA skips what depends on it, waits (bounded) for its own loads and
 // MMAs, frees its TMEM and leaves without writing.
@@ -56,9 +59,16 @@ struct PrefixCfg {
     static constexpr int BAR_OFF = V_OFF + KV_BYTES;
     // q_full, k_full[NG], v_full, s_full, p_full, o_full; then the TMEM address
     static constexpr int NBARS = NG + 5;
-    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;   // + alignment slack
+    // barriers, the TMEM address, the softmax exchange (max and sum per half
+    // row, agreement flags), then alignment slack
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 4 * M * 4 + 2 * 8 * 4 + 1024;
     static constexpr int TMEM_COLS = 512;             // S at column 0, O at column CH
-    static constexpr int THREADS = 6 * 32;            // 4 softmax warps, producer, MMA
+    static constexpr int SOFT_WARPS = 8;              // two per TMEM lane quarter
+    static constexpr int PRODUCER = SOFT_WARPS, MMA_WARP = SOFT_WARPS + 1;
+    static constexpr int THREADS = (SOFT_WARPS + 2) * 32;
+    static constexpr int HALF = CH / 2;               // score columns per softmax thread
+    static constexpr int OSTRIDE = D + 4;             // staged output row (floats), padded
+    static_assert(M * OSTRIDE * 4 <= BAR_OFF, "staged output fits the freed tiles");
     static_assert((BS % R == 0 || BS == 8) && D % 64 == 0, "shared-prefix shape");
     static_assert(CH + D <= TMEM_COLS, "S and O must fit TMEM");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -117,10 +127,11 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
 
     if (threadIdx.x == 0) {
         failed = 0;
-        for (int i = 0; i < C::NBARS; ++i) mbar_init(&bars[i], i == NG + 3 ? 128 : 1);
+        for (int i = 0; i < C::NBARS; ++i)
+            mbar_init(&bars[i], i == NG + 3 ? 32 * C::SOFT_WARPS : 1);
         fence_mbar_init();
     }
-    if (warp == 5) {                                      // the MMA warp owns TMEM
+    if (warp == C::MMA_WARP) {                            // the MMA warp owns TMEM
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -130,7 +141,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t s_tmem = tmem, o_tmem = tmem + CH;
 
-    if (warp == 4) {
+    if (warp == C::PRODUCER) {
         // ------------------------------------------------ producer (lane 0) --
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
@@ -174,7 +185,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             mbar_arrive_expect_tx(v_full, C::KV_BYTES + a.tx_extra);
             for (int j = 0; j < C::U; ++j) load_unit(&tm_v, vs, v_full, j);
         }
-    } else if (warp == 5) {
+    } else if (warp == C::MMA_WARP) {
         // --------------------------------------------- MMA issuer (lane 0) --
         if (lane == 0) {
             const uint32_t q0 = smem_addr(qs), k0 = smem_addr(ks), v0 = smem_addr(vs);
@@ -226,45 +237,68 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             else if (s_issued) (void)mbar_wait_bounded(s_full, 0, a.wait_ns);
         }
     } else {
-        // -------------------------------- softmax and epilogue: warps 0-3 --
-        const int r = 32 * warp + lane;                   // this thread's query row / TMEM lane
-        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-        float m = -INFINITY, l = 0.f;
-        bool ok = __all_sync(FULL_MASK, mbar_wait_bounded(s_full, 0, a.wait_ns));
-        if (ok) {
-            tc_fence_after_sync();
-            // pass 1: the row's maximum over the chunk's prefix tokens (log2 units)
-#pragma unroll 1
-            for (int c = 0; c < CH / 32; ++c) {
-                float v[32];
-                tmem_ld32(s_tmem + lane_off + 32 * c, v);
-                tmem_ld_wait();
+        // ------------------------------- softmax and epilogue: warps 0-7 --
+        // thread = (row r of TMEM lane quarter warp % 4, column half hf)
+        const int r = 32 * (warp & 3) + lane, hf = warp >> 2;
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        float* xm = reinterpret_cast<float*>(smem + C::BAR_OFF + C::NBARS * 8 + 16);   // [2][M]
+        float* xl = xm + 2 * M;                                                        // [2][M]
+        int* okw = reinterpret_cast<int*>(xl + 2 * M);                                 // [2][8]
+        auto soft_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(32 * C::SOFT_WARPS) : "memory"); };
+        // every softmax warp must agree before it depends on the others
+        // (each agreement point has its own flags: a fast warp must not
+        // overwrite flags a slow one is still reading)
+        auto all_ok = [&](int point, bool mine) {
+            int* f = okw + point * C::SOFT_WARPS;
+            if (lane == 0) f[warp] = mine ? 1 : 0;
+            soft_sync();
+            int ok = 1;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (32 * c + j < valid) m = fmaxf(m, v[j] * a.scale_log2);
+            for (int w = 0; w < C::SOFT_WARPS; ++w) ok &= f[w];
+            return ok != 0;
+        };
+        float v[C::HALF];
+        float mloc = -INFINITY;
+        const bool s_ok = __all_sync(FULL_MASK, mbar_wait_bounded(s_full, 0, a.wait_ns));
+        if (s_ok) {
+            tc_fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < C::HALF / 32; ++c) {
+                float t[32];
+                tmem_ld32(s_tmem + lane_off + hf * C::HALF + 32 * c, t);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[32 * c + j] = t[j];
             }
-            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum of p
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < C::HALF; ++j) {
+                v[j] = hf * C::HALF + j < valid ? v[j] * a.scale_log2 : -INFINITY;
+                mloc = fmaxf(mloc, v[j]);
+            }
+            xm[hf * M + r] = mloc;
+        }
+        bool ok = all_ok(0, s_ok);
+        float m = -INFINITY, lsum = 0.f;
+        if (ok) {
+            m = fmaxf(xm[r], xm[M + r]);
+            // p = 2^(x - m) into this half of the P tile (bf16, 128-byte swizzle)
             const uint32_t prow = smem_addr(ks) + (uint32_t)r * 128;
-#pragma unroll 1
-            for (int c = 0; c < CH / 32; ++c) {
-                float v[32];
-                tmem_ld32(s_tmem + lane_off + 32 * c, v);
-                tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < C::HALF / 32; ++c) {
                 uint32_t w[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const int t = 32 * c + 2 * j;
-                    const float p0 = t < valid ? exp2_approx(v[2 * j] * a.scale_log2 - m) : 0.f;
-                    const float p1 =
-                        t + 1 < valid ? exp2_approx(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
-                    l += p0 + p1;
+                    const float p0 = exp2_approx(v[32 * c + 2 * j] - m);
+                    const float p1 = exp2_approx(v[32 * c + 2 * j + 1] - m);
+                    lsum += p0 + p1;
                     w[j] = pack_bf16x2(p0, p1);
                 }
-                // tokens 32c .. 32c+31: slab c / 2, 16-byte chunks 4 (c % 2) .. + 3
-                const uint32_t base = prow + (uint32_t)(c / 2) * (M * 128);
+                // tokens t0 .. t0+31 of the chunk: slab t0 / 64, 16-byte chunks 4 ((t0 / 32) % 2) ..
+                const int t0 = hf * C::HALF + 32 * c;
+                const uint32_t base = prow + (uint32_t)(t0 / 64) * (M * 128);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int ch = 4 * (c % 2) + q;
+                    const int ch = 4 * ((t0 / 32) % 2) + q;
                     const uint32_t addr = base + (uint32_t)((ch ^ (r & 7)) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
                                  "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]),
@@ -272,53 +306,71 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                                  : "memory");
                 }
             }
+            xl[hf * M + r] = lsum;
             fence_proxy_async_smem();                   // P is read by the tensor cores
             tc_fence_before_sync();
             mbar_arrive(p_full);
-            ok = __all_sync(FULL_MASK, mbar_wait_bounded(o_full, 0, a.wait_ns));
+            const bool o_ok = __all_sync(FULL_MASK, mbar_wait_bounded(o_full, 0, a.wait_ns));
+            ok = all_ok(1, o_ok);
         }
         if (!ok) {
-            if (lane == 0) {
+            if (lane == 0 && warp == 0) {
                 raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
                 failed = 1;
             }
         } else {
             tc_fence_after_sync();
-            const int row = row0 + r;
-            const bool mine = row < rows;
-            const int seq = gs + row / G, h = kvh * G + row % G;
-            const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride +
-                                a.prefix_slot0 + chunk;
-            float* dst = a.ws_o + slot * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                float v[32];
-                tmem_ld32(o_tmem + lane_off + 32 * c, v);
-                tmem_ld_wait();
-                if (mine) {
+            // this thread's half of the row's output, staged row-major (padded
+            // rows) over the tiles, which no MMA or load uses any more
+            float* os = reinterpret_cast<float*>(smem);
+            constexpr int OH = D / 2;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        reinterpret_cast<float4*>(dst + 32 * c)[j] =
-                            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            for (int c = 0; c < OH / 32; ++c) {
+                float t[32];
+                tmem_ld32(o_tmem + lane_off + hf * OH + 32 * c, t);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<float4*>(os + r * C::OSTRIDE + hf * OH + 32 * c + 4 * j) =
+                        make_float4(t[4 * j], t[4 * j + 1], t[4 * j + 2], t[4 * j + 3]);
+            }
+            soft_sync();
+            // whole rows to the workspace: D / 4 float4 per row, lanes split over rows
+            constexpr int LPR = D / 4 < 32 ? D / 4 : 32;           // lanes per row
+            constexpr int RPI = 32 / LPR;                          // rows per instruction
+            constexpr int VPL = D / 4 / LPR;                       // float4 per lane
+            const int tw = warp * 32 + lane;
+            for (int rr = tw / LPR; rr < M; rr += 32 * C::SOFT_WARPS / LPR) {
+                const int row = row0 + rr;
+                if (row >= rows) continue;
+                const int seq = gs + row / G, h = kvh * G + row % G;
+                const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride +
+                                    a.prefix_slot0 + chunk;
+                const int c4 = tw % LPR;
+#pragma unroll
+                for (int k = 0; k < VPL; ++k)
+                    reinterpret_cast<float4*>(a.ws_o + slot * D)[c4 + LPR * k] =
+                        *reinterpret_cast<const float4*>(os + rr * C::OSTRIDE + 4 * (c4 + LPR * k));
+                if (c4 == 0) {
+                    a.ws_m[slot] = fmaxf(xm[rr], xm[M + rr]);
+                    a.ws_l[slot] = xl[rr] + xl[M + rr];
                 }
             }
-            if (mine) {
-                a.ws_m[slot] = m;
-                a.ws_l[slot] = l;
-            }
+            (void)RPI;
         }
+        (void)m;
     }
 
     // ---------------- teardown: every role is done with TMEM and shared memory --
     tc_fence_before_sync();
     __syncthreads();
-    if (failed && warp == 4 && lane == 0) {
+    if (failed && warp == C::PRODUCER && lane == 0) {
         // loads may still be in flight after a role gave up: wait (bounded) for them
         (void)mbar_wait_bounded(q_full, 0, a.wait_ns);
         for (int g = 0; g < NG; ++g) (void)mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
         (void)mbar_wait_bounded(v_full, 0, a.wait_ns);
     }
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
