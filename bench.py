@@ -390,7 +390,12 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     the timed region holds only device work on inputs resident in HBM.
     graph: the timed steps are captured once into a CUDA graph (after the
     eager warm-up) and the graph is replayed once inside the timed region,
-    which runs exactly the same launches without the host's issue cost."""
+    which runs exactly the same launches without the host's issue cost.
+    Events cannot time launches inside a graph, so the decode launches of
+    the same steps go into a second graph, replayed after the timed region:
+    its time / K is the mean decode launch (back to back; the decode calls
+    are idempotent on the final state: the fused append rewrites the same
+    rows, the other decodes only read)."""
     pa, p, dev = loop.pa, loop.p, loop.device
     total = steps + warmup
     slots, cows, tabs, lens = [], [], [], []
@@ -414,6 +419,13 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
 
+    def decode_only(i):
+        if loop.fused:
+            pa.pa_decode_append(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
+                                slots_d[i], tabs_d[i], lens_d[i], p.scale)
+        else:
+            loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
+
     def step(i, timed_index=None):
         if cows_d[i] is not None:
             pa.pa_copy_blocks(loop.k_cache, loop.v_cache, cows_d[i])
@@ -432,15 +444,18 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
-    g = None
+    g = g_dec = None
     if graph:
         cap = torch.cuda.Stream(device=dev)
         cap.wait_stream(stream)
-        g = torch.cuda.CUDAGraph()
+        g, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.stream(cap):
             with torch.cuda.graph(g, stream=cap):
                 for j in range(steps):
-                    step(warmup + j, j)
+                    step(warmup + j)
+            with torch.cuda.graph(g_dec, stream=cap):
+                for j in range(steps):
+                    decode_only(warmup + j)
         stream.wait_stream(cap)
         torch.cuda.synchronize()
     barrier(world)
@@ -462,7 +477,16 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     if flags:
         raise RuntimeError(f"device error word 0x{flags:x} during the timed region")
     ms = t0.elapsed_time(t1)
-    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+    if g_dec is not None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g_dec.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dec_ms = [e0.elapsed_time(e1) / steps] * steps
+        del g, g_dec
+    else:
+        dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
     timed_lens = lens[warmup:]
     kv = sum(decode_kv_bytes(x, p) for x in timed_lens)
     alg = [decode_alg_bytes(x, p, loop.fused) for x in timed_lens]

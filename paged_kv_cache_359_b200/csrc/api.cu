@@ -55,6 +55,48 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Encoded tensor maps, keyed by everything the encoding depends on (base
+// address, data type, sizes, box, swizzle): a hit returns the same 128 bytes
+// a fresh cuTensorMapEncodeTiled would, and saves the encode on every launch
+// over the same cache or query buffer.  A small round-robin cache, shared by
+// all host threads under a mutex.
+struct MapKey {
+    const void* base;
+    int kind;                      // 0: cache tensor, 1: query tensor
+    int v[7];
+    bool operator==(const MapKey& o) const {
+        if (base != o.base || kind != o.kind) return false;
+        for (int i = 0; i < 7; ++i)
+            if (v[i] != o.v[i]) return false;
+        return true;
+    }
+};
+constexpr int MAP_CACHE = 32;
+std::mutex g_map_mutex;
+MapKey g_map_keys[MAP_CACHE];
+CUtensorMap g_maps[MAP_CACHE];
+int g_map_count = 0, g_map_next = 0;
+
+bool map_lookup(const MapKey& k, CUtensorMap* out) {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (int i = 0; i < g_map_count; ++i)
+        if (g_map_keys[i] == k) {
+            *out = g_maps[i];
+            return true;
+        }
+    return false;
+}
+
+void map_store(const MapKey& k, const CUtensorMap& m) {
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    for (int i = 0; i < g_map_count; ++i)
+        if (g_map_keys[i] == k) return;
+    const int i = g_map_count < MAP_CACHE ? g_map_count++ : g_map_next;
+    g_map_next = (i + 1) % MAP_CACHE;
+    g_map_keys[i] = k;
+    g_maps[i] = m;
+}
+
 int elem_size(pa_dtype dt) { return dt == PA_DTYPE_F32 ? 4 : 2; }
 
 pa_status check_geometry(pa_dtype dt, int head_dim, int block_size) {
@@ -205,6 +247,9 @@ pa_status fail(pa_status status, const char* fmt, ...) {
 pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, int head_dim,
                            int num_kv_heads, int block_size, int num_blocks, int box_inner,
                            int rows, bool swizzle128) {
+    const MapKey key{base, 0, {(int)dtype, head_dim, num_kv_heads, block_size, num_blocks,
+                               box_inner * 1024 + rows, swizzle128 ? 1 : 0}};
+    if (map_lookup(key, map)) return PA_OK;
     auto enc = tensor_map_encoder();
     if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     const cuuint64_t es = (cuuint64_t)elem_size(dtype);
@@ -222,11 +267,14 @@ pa_status encode_cache_map(CUtensorMap* map, const void* base, pa_dtype dtype, i
                      swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    map_store(key, *map);
     return PA_OK;
 }
 
 pa_status encode_query_map(CUtensorMap* map, const void* q, int head_dim, int num_heads,
                            int num_seqs, int heads, int seqs) {
+    const MapKey key{q, 1, {head_dim, num_heads, num_seqs, heads, seqs, 0, 0}};
+    if (map_lookup(key, map)) return PA_OK;
     auto enc = tensor_map_encoder();
     if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_heads, (cuuint64_t)num_seqs};
@@ -239,6 +287,7 @@ pa_status encode_query_map(CUtensorMap* map, const void* q, int head_dim, int nu
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", (int)r);
+    map_store(key, *map);
     return PA_OK;
 }
 

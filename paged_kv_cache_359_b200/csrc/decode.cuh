@@ -1009,28 +1009,55 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                         });
             pdl_wait();                                // the shared pass is complete
             if (nchunks) {
-                // merge with the shared pass's chunks of each head: every thread
-                // reads the chunk maxima and sums of the head it writes (one
-                // address across the warp's lanes of that head) and its own
-                // outputs' chunk values; no load depends on another's value
-                // beyond the maxima, so this costs about two L2 round trips
+                // merge with the shared pass's chunks of each head.  A thread
+                // writes OPT outputs (g, d); for each batch of up to 8 chunks it
+                // first loads the chunk maxima of all its outputs' heads, then
+                // their outputs and sums, every load of a phase in flight at
+                // once: two L2 round trips per 8 chunks
                 __syncthreads();                       // x is complete
-                for (int idx = threadIdx.x; idx < G * D; idx += NT) {
-                    const int g = idx / D, d = idx % D;
-                    const size_t b = (head0 + g) * a.slot_stride + a.prefix_slot0;
-                    float mm = x[g];
-#pragma unroll 8
-                    for (int c = 0; c < nchunks; ++c) mm = fmaxf(mm, a.ws_m[b + c]);
-                    const float e0 = x[g] == -INFINITY ? 0.f : exp2_approx(x[g] - mm);
-                    float num = e0 * x[2 * G + g * D + d], den = e0 * x[G + g];
-#pragma unroll 8
-                    for (int c = 0; c < nchunks; ++c) {
-                        const float ec = exp2_approx(a.ws_m[b + c] - mm);
-                        num = fmaf(ec, a.ws_o[(b + c) * D + d], num);
-                        den = fmaf(ec, a.ws_l[b + c], den);
-                    }
-                    store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                constexpr int OPT = (G * D + NT - 1) / NT;
+                float mm[OPT], num[OPT], den[OPT];
+                size_t bse[OPT];
+                int dd[OPT], gg[OPT];
+#pragma unroll
+                for (int k = 0; k < OPT; ++k) {
+                    const int idx = threadIdx.x + k * NT;
+                    gg[k] = idx < G * D ? idx / D : 0;
+                    dd[k] = idx % D;
+                    bse[k] = (head0 + gg[k]) * a.slot_stride + a.prefix_slot0;
+                    mm[k] = x[gg[k]];
                 }
+                for (int c0 = 0; c0 < nchunks; c0 += 8) {
+#pragma unroll
+                    for (int k = 0; k < OPT; ++k)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (c0 + c < nchunks) mm[k] = fmaxf(mm[k], a.ws_m[bse[k] + c0 + c]);
+                }
+#pragma unroll
+                for (int k = 0; k < OPT; ++k) {
+                    const float own = x[gg[k]];
+                    const float e0 = own == -INFINITY ? 0.f : exp2_approx(own - mm[k]);
+                    num[k] = e0 * x[2 * G + gg[k] * D + dd[k]];
+                    den[k] = e0 * x[G + gg[k]];
+                }
+                for (int c0 = 0; c0 < nchunks; c0 += 8) {
+#pragma unroll
+                    for (int k = 0; k < OPT; ++k)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (c0 + c < nchunks) {
+                                const size_t sl = bse[k] + c0 + c;
+                                const float ec = exp2_approx(a.ws_m[sl] - mm[k]);
+                                num[k] = fmaf(ec, a.ws_o[sl * D + dd[k]], num[k]);
+                                den[k] = fmaf(ec, a.ws_l[sl], den[k]);
+                            }
+                }
+#pragma unroll
+                for (int k = 0; k < OPT; ++k)
+                    if (threadIdx.x + k * NT < G * D)
+                        store_out(out + (head0 + gg[k]) * D + dd[k],
+                                  den[k] > 0.f ? num[k] / den[k] : 0.f);
             }
             return;
         }
