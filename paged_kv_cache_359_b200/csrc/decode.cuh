@@ -191,7 +191,13 @@ __device__ __forceinline__ void append_row(const DecodeArgs& a, int seq, int kvh
     fence_proxy_async_global();
 }
 
-enum class Mode { Decode, Split };
+// Kernel instances: Decode = pa_decode's longest-first grid (one CTA per
+// item), Cluster = pa_decode with several CTAs per item merged through
+// distributed shared memory, Split = pa_decode_split's partitions, Own = the
+// shared-prefix decode's own-token pass (longest-first, half the warps of
+// Decode so that two CTAs fit an SM beside a shared-pass CTA).  Each is its
+// own instance so that a kernel carries only its own path's code.
+enum class Mode { Decode, Cluster, Split, Own };
 
 // ============================================================ CoreUnit ==
 // fp32 FMA unit: a K/V row is spread over LPR lanes (16 bytes per lane), each
@@ -584,14 +590,15 @@ using UnitFor = typename std::conditional<(std::is_same<T, __nv_bfloat16>::value
                                           MmaUnit<D, BS, G>, CoreUnit<T, D, BS, G>>::type;
 
 // ---------------------------------------------------- kernel geometry ----
-template <class U>
+template <class U, bool HALF_WARPS = false>
 struct Layout {
     static constexpr int UNIT_BYTES = U::R * U::D * (int)sizeof(typename U::T);
     static constexpr int STAGE_BYTES = 2 * UNIT_BYTES;
     // warps per CTA: four, or two when a stage is 16 KiB (head_dim 256 on
     // the tensor-core unit), so that three CTAs still fit an SM with a
-    // two-stage ring per warp (about 192 KiB of loads in flight per SM)
-    static constexpr int NW = STAGE_BYTES >= 16384 ? 2 : 4;
+    // two-stage ring per warp (about 192 KiB of loads in flight per SM);
+    // half of that for the shared-prefix decode's own-token pass
+    static constexpr int NW = (STAGE_BYTES >= 16384 ? 2 : 4) / (HALF_WARPS ? 2 : 1);
     // stages per warp: about 12 KiB of ring per warp, at least two; with
     // 4 KiB stages (head_dim 64) the smaller CTA lets four CTAs share an SM,
     // which hides the per-CTA prologue and merge of these short items better
@@ -625,13 +632,12 @@ struct Ctx {
 // over the NW warps, then merge the warps into shared memory.  Returns with
 // the CTA-merged (max, sum, unnormalised output) per (g, d) computed by
 // `epilogue`.  Every thread of the CTA must call it (it holds barriers).
-template <class U, class Epi>
+template <class U, class Ly, class Epi>
 __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
                                          const CUtensorMap* tm_v, const DecodeArgs& a, int seq,
                                          int kvh, int L, int u_begin, int u_end, int ctas,
                                          int crank, Epi&& epilogue) {
     using T = typename U::T;
-    using Ly = Layout<U>;
     constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
     const int warp = cx.warp, lane = cx.lane;
     const int ustride = ctas * NW;
@@ -765,11 +771,11 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
 }
 
 template <class U, Mode MODE>
-__global__ void __launch_bounds__(Layout<U>::NW * 32)
+__global__ void __launch_bounds__(Layout<U, MODE == Mode::Own>::NW * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
     using T = typename U::T;
-    using Ly = Layout<U>;
+    using Ly = Layout<U, MODE == Mode::Own>;
     constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
     constexpr int NT = NW * 32;
     // The own-token pass of the shared-prefix decode reads nothing the
@@ -779,7 +785,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
     // the shared pass only before the merge, so the two overlap where SMs
     // are free; every CTA still waits before it leaves, which keeps the
     // stream's completion order.  Every other launch waits here.
-    const bool late_wait = MODE == Mode::Decode && a.sched == SCHED_LPT && a.group_starts;
+    const bool late_wait = MODE == Mode::Own;
     if (!late_wait) pdl_wait();
     pdl_launch_dependents();
 
@@ -842,7 +848,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
         const int u_begin = nparts == 1 && part == 0 ? 0 : part * pu;
         const int u_end = nparts == 1 ? total_units : cmin(u_begin + pu, total_units);
         const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
-        run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, u_begin, u_end, 1, 0,
+        run_item<U, Ly>(cx, &tm_k, &tm_v, a, seq, kvh, L, u_begin, u_end, 1, 0,
                     [&](int g, int d, float big, float num, float den, float*) {
                         if (nparts > 1) {
                             const size_t slot = (head0 + g) * a.slot_stride + part;
@@ -857,7 +863,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                     });
         return;
     } else {
-        if (a.sched == SCHED_CLUSTER) {
+        if constexpr (MODE == Mode::Cluster) {
             seq = blockIdx.z;
             kvh = blockIdx.y;
             L = clamp_len(seq);
@@ -870,7 +876,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                     __syncthreads();
             }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
-            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, ctas, blockIdx.x,
+            run_item<U, Ly>(cx, &tm_k, &tm_v, a, seq, kvh, L, 0, (L + R - 1) / R, ctas, blockIdx.x,
                         [&](int g, int d, float big, float num, float den, float* x) {
                             // x: [G] max, [G] sum, [G][D] unnormalised output
                             if (ctas > 1) {
@@ -907,9 +913,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
                 cluster.sync();                        // keep xch alive until rank 0 is done
             }
             return;
-        }
-
-        if (a.sched == SCHED_LPT) {
+        } else {
             // Which sequence sits at rank r = blockIdx.x / Hk of the list sorted
             // by (tokens this pass reads descending, index ascending)?  Warp 0
             // selects it (rank_select); up to 256 sequences it holds the
@@ -995,7 +999,7 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             // x: this CTA's own part, [G] max, [G] sum, [G][D] unnormalised output,
             // kept after the exchange area when it is merged with prefix chunks
             float* x = reinterpret_cast<float*>(smem) + NW * G * (D + 2);
-            run_item<U>(cx, &tm_k, &tm_v, a, seq, kvh, L, tok0 / R, (L + R - 1) / R, 1, 0,
+            run_item<U, Ly>(cx, &tm_k, &tm_v, a, seq, kvh, L, tok0 / R, (L + R - 1) / R, 1, 0,
                         [&](int g, int d, float big, float num, float den, float*) {
                             if (nchunks) {
                                 if (d == 0) {
@@ -1010,54 +1014,70 @@ __global__ void __launch_bounds__(Layout<U>::NW * 32)
             pdl_wait();                                // the shared pass is complete
             if (nchunks) {
                 // merge with the shared pass's chunks of each head.  A thread
-                // writes OPT outputs (g, d); for each batch of up to 8 chunks it
-                // first loads the chunk maxima of all its outputs' heads, then
-                // their outputs and sums, every load of a phase in flight at
-                // once: two L2 round trips per 8 chunks
+                // writes OPT groups of 4 outputs (g, d .. d+3); it first loads
+                // the chunk maxima of its heads, then the chunks' float4
+                // outputs and sums, CB chunks of every output at a time, all
+                // loads of a batch in flight at once (about 8 float4 per
+                // thread, which keeps them in registers at every head_dim)
                 __syncthreads();                       // x is complete
-                constexpr int OPT = (G * D + NT - 1) / NT;
-                float mm[OPT], num[OPT], den[OPT];
-                size_t bse[OPT];
-                int dd[OPT], gg[OPT];
+                constexpr int Q4 = D / 4;                        // float4 per head row
+                constexpr int OPT = (G * Q4 + NT - 1) / NT;
+                constexpr int CB = OPT >= 8 ? 1 : 8 / OPT;     // chunks per batch
+                float mm[OPT], den[OPT];
+                float4 num[OPT];
+                int gg[OPT], qq[OPT];
 #pragma unroll
                 for (int k = 0; k < OPT; ++k) {
                     const int idx = threadIdx.x + k * NT;
-                    gg[k] = idx < G * D ? idx / D : 0;
-                    dd[k] = idx % D;
-                    bse[k] = (head0 + gg[k]) * a.slot_stride + a.prefix_slot0;
+                    gg[k] = idx < G * Q4 ? idx / Q4 : 0;
+                    qq[k] = idx % Q4;
                     mm[k] = x[gg[k]];
                 }
+                auto slot_of = [&](int k, int c) {
+                    return (head0 + gg[k]) * a.slot_stride + a.prefix_slot0 + c;
+                };
                 for (int c0 = 0; c0 < nchunks; c0 += 8) {
 #pragma unroll
                     for (int k = 0; k < OPT; ++k)
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
-                            if (c0 + c < nchunks) mm[k] = fmaxf(mm[k], a.ws_m[bse[k] + c0 + c]);
+                            if (c0 + c < nchunks) mm[k] = fmaxf(mm[k], a.ws_m[slot_of(k, c0 + c)]);
                 }
 #pragma unroll
                 for (int k = 0; k < OPT; ++k) {
                     const float own = x[gg[k]];
                     const float e0 = own == -INFINITY ? 0.f : exp2_approx(own - mm[k]);
-                    num[k] = e0 * x[2 * G + gg[k] * D + dd[k]];
+                    const float* xo = x + 2 * G + gg[k] * D + 4 * qq[k];
+                    num[k] = make_float4(e0 * xo[0], e0 * xo[1], e0 * xo[2], e0 * xo[3]);
                     den[k] = e0 * x[G + gg[k]];
                 }
-                for (int c0 = 0; c0 < nchunks; c0 += 8) {
+                for (int c0 = 0; c0 < nchunks; c0 += CB) {
 #pragma unroll
                     for (int k = 0; k < OPT; ++k)
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
+                        for (int c = 0; c < CB; ++c)
                             if (c0 + c < nchunks) {
-                                const size_t sl = bse[k] + c0 + c;
+                                const size_t sl = slot_of(k, c0 + c);
                                 const float ec = exp2_approx(a.ws_m[sl] - mm[k]);
-                                num[k] = fmaf(ec, a.ws_o[sl * D + dd[k]], num[k]);
+                                const float4 o4 =
+                                    reinterpret_cast<const float4*>(a.ws_o + sl * D)[qq[k]];
+                                num[k].x = fmaf(ec, o4.x, num[k].x);
+                                num[k].y = fmaf(ec, o4.y, num[k].y);
+                                num[k].z = fmaf(ec, o4.z, num[k].z);
+                                num[k].w = fmaf(ec, o4.w, num[k].w);
                                 den[k] = fmaf(ec, a.ws_l[sl], den[k]);
                             }
                 }
 #pragma unroll
                 for (int k = 0; k < OPT; ++k)
-                    if (threadIdx.x + k * NT < G * D)
-                        store_out(out + (head0 + gg[k]) * D + dd[k],
-                                  den[k] > 0.f ? num[k] / den[k] : 0.f);
+                    if (threadIdx.x + k * NT < G * Q4) {
+                        T* o = out + (head0 + gg[k]) * D + 4 * qq[k];
+                        const float inv = den[k] > 0.f ? 1.f / den[k] : 0.f;
+                        store_out(o + 0, den[k] > 0.f ? num[k].x * inv : 0.f);
+                        store_out(o + 1, den[k] > 0.f ? num[k].y * inv : 0.f);
+                        store_out(o + 2, den[k] > 0.f ? num[k].z * inv : 0.f);
+                        store_out(o + 3, den[k] > 0.f ? num[k].w * inv : 0.f);
+                    }
             }
             return;
         }

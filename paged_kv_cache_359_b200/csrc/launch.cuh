@@ -29,8 +29,11 @@ struct DecodeLaunch {
     cudaStream_t stream;
 };
 
-// Opt a kernel into `bytes` of dynamic shared memory, once per device.
-// `done` must be distinct for every kernel (one static per instantiation).
+// Opt a kernel into `bytes` of dynamic shared memory, once per device, and
+// prefer all of L1 as shared memory: the decode kernels fill an SM's shared
+// memory anyway, and the cascade's two kernels can then share an SM (a
+// decode CTA beside a shared-pass CTA).  `done` must be distinct for every
+// kernel (one static per instantiation).
 template <class K>
 inline pa_status allow_smem(K kernel, int bytes, std::atomic<unsigned long long>& done) {
     int dev = 0;
@@ -38,6 +41,8 @@ inline pa_status allow_smem(K kernel, int bytes, std::atomic<unsigned long long>
     const unsigned long long bit = 1ull << (dev & 63);
     if (done.load(std::memory_order_relaxed) & bit) return PA_OK;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess)
         return fail(PA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     done.fetch_or(bit);
@@ -98,6 +103,18 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
                 if (e != cudaSuccess)
                     return fail(PA_ERR_CUDA, "shared-prefix launch: %s", cudaGetErrorString(e));
             }
+            // the own-token pass: longest-first, half-width CTAs
+            using Lo = Layout<U, true>;
+            static std::atomic<unsigned long long> done_o{0};
+            auto ok = paged_decode_kernel<U, Mode::Own>;
+            if (pa_status s = allow_smem(ok, Lo::SMEM_BYTES, done_o)) return s;
+            cfg.blockDim = dim3(Lo::NW * 32);
+            cfg.dynamicSmemBytes = Lo::SMEM_BYTES;
+            cfg.gridDim = dim3((unsigned)((long long)l.num_seqs * l.num_kv_heads));
+            e = cudaLaunchKernelEx(&cfg, ok, mk, mv, l.args);
+            if (e != cudaSuccess)
+                return fail(PA_ERR_CUDA, "own-token launch: %s", cudaGetErrorString(e));
+            return PA_OK;
         } else {
             return fail(PA_ERR_UNSUPPORTED, "shared-prefix decode needs bf16");
         }
@@ -118,21 +135,23 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
             add_pdl_attr(rattr, &rc.numAttrs);
             e = cudaLaunchKernelEx(&rc, lse_reduce_kernel<T, D>, l.args);
         }
-    } else {
+    } else if (l.args.sched == SCHED_LPT) {
         static std::atomic<unsigned long long> done{0};
         auto kern = paged_decode_kernel<U, Mode::Decode>;
         if (pa_status s = allow_smem(kern, Ly::SMEM_BYTES, done)) return s;
-        if (l.args.sched == SCHED_LPT) {
-            cfg.gridDim = dim3((unsigned)((long long)l.num_seqs * l.num_kv_heads));
-        } else {
-            cfg.gridDim = dim3(l.ctas, l.num_kv_heads, l.num_seqs);
-            if (l.ctas > 1) {
-                cudaLaunchAttribute& c = attr[cfg.numAttrs++];
-                c.id = cudaLaunchAttributeClusterDimension;
-                c.val.clusterDim.x = l.ctas;
-                c.val.clusterDim.y = 1;
-                c.val.clusterDim.z = 1;
-            }
+        cfg.gridDim = dim3((unsigned)((long long)l.num_seqs * l.num_kv_heads));
+        e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
+    } else {
+        static std::atomic<unsigned long long> done{0};
+        auto kern = paged_decode_kernel<U, Mode::Cluster>;
+        if (pa_status s = allow_smem(kern, Ly::SMEM_BYTES, done)) return s;
+        cfg.gridDim = dim3(l.ctas, l.num_kv_heads, l.num_seqs);
+        if (l.ctas > 1) {
+            cudaLaunchAttribute& c = attr[cfg.numAttrs++];
+            c.id = cudaLaunchAttributeClusterDimension;
+            c.val.clusterDim.x = l.ctas;
+            c.val.clusterDim.y = 1;
+            c.val.clusterDim.z = 1;
         }
         e = cudaLaunchKernelEx(&cfg, kern, mk, mv, l.args);
     }

@@ -14,24 +14,25 @@
 // CTA = (prefix chunk of CH tokens, kv head, group x 128-row block); CH is
 // 256 (head_dim <= 128) or 128 (head_dim 256).  Roles:
 //  * producer warp: TMA loads of the CTA's 128 query rows (a 3-D box over
-//    q [S][Hq][D]: members x G heads, row = member * G + head), the chunk's K
-//    tiles in groups of 64 tokens, then its V tiles, all 128-byte swizzled;
-//    a unit past the prefix is loaded from outside the pool map, which TMA
+//    q [S][Hq][D]: members x G heads, row = member * G + head) and of the
+//    chunk's K tiles in groups of 64 tokens, all 128-byte swizzled; once the
+//    first MMA has read Q, the chunk's V tiles into Q's space (so the CTA
+//    needs ~128 KB of shared memory and a decode CTA fits beside it); a
+//    unit past the prefix is loaded from outside the pool map, which TMA
 //    fills with zeros;
 //  * MMA warp (one elected thread): S = Q K^T into TMEM (M = 128 rows,
 //    N = 64 tokens per group as its K tiles land, K = head_dim), commit;
 //    then, once P is in shared memory, O = P V into TMEM (M = 128,
 //    N = head_dim, K = CH tokens, V read MN-major), commit;
-//  * eight softmax warps, two per TMEM lane quarter: a thread holds half of
-//    one query row's scores in registers (one TMEM read), the two halves
-//    exchange their maxima through shared memory, and each writes
-//    p = 2^(s * scale * log2 e - max), rounded to bf16, into its half of the
-//    swizzled P tile (which reuses the K tile's space) and sums p in fp32;
-//    after the second MMA each thread stages its half of the row's output in
-//    the (now free) shared memory, and the warps write whole 512-byte rows
-//    to the workspace slot prefix_slot0 + chunk with coalesced stores, with
-//    the row's maximum and sum; pa_decode's CTAs for each sequence's own
-//    tokens merge these into the output.
+//  * four softmax warps, one TMEM lane (query row) per thread: the exact
+//    maximum of the row's scores over the chunk (masked past the prefix),
+//    then p = 2^(s * scale * log2 e - max), rounded to bf16, into the
+//    swizzled P tile (which reuses the K tile's space) and the fp32 sum of p;
+//    after the second MMA the threads stage the rows' output in the (now
+//    free) tiles, up to 128 columns at a time, and the warps write whole
+//    rows to the workspace slot prefix_slot0 + chunk with coalesced stores,
+//    with each row's maximum and sum; pa_decode's CTAs for each sequence's
+//    own tokens merge these into the output.
 // Every wait is bounded; a wait that runs out sets PA_DEVERR_WAIT_TIMEOUT,
 // the CTA skips what depends on it, waits (bounded) for its own loads and
 // MMAs, frees its TMEM and leaves without writing.
@@ -55,19 +56,22 @@ struct PrefixCfg {
     static constexpr int KV_BYTES = KSL * CH * 128;
     static constexpr int P_BYTES = NG * M * 128;
     static constexpr int KP_BYTES = KV_BYTES > P_BYTES ? KV_BYTES : P_BYTES;
-    static constexpr int Q_OFF = 0, K_OFF = Q_BYTES, V_OFF = Q_BYTES + KP_BYTES;
-    static constexpr int BAR_OFF = V_OFF + KV_BYTES;
+    static constexpr int QV_BYTES = KV_BYTES > Q_BYTES ? KV_BYTES : Q_BYTES;
+    // Q, then V over the same bytes; K, then P over the same bytes
+    static constexpr int QV_OFF = 0, K_OFF = QV_BYTES;
+    static constexpr int BAR_OFF = QV_BYTES + KP_BYTES;
     // q_full, k_full[NG], v_full, s_full, p_full, o_full; then the TMEM address
     static constexpr int NBARS = NG + 5;
-    // barriers, the TMEM address, the softmax exchange (max and sum per half
-    // row, agreement flags), then alignment slack
-    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 4 * M * 4 + 2 * 8 * 4 + 1024;
-    static constexpr int TMEM_COLS = 512;             // S at column 0, O at column CH
-    static constexpr int SOFT_WARPS = 8;              // two per TMEM lane quarter
+    static constexpr int SOFT_WARPS = 4;
     static constexpr int PRODUCER = SOFT_WARPS, MMA_WARP = SOFT_WARPS + 1;
     static constexpr int THREADS = (SOFT_WARPS + 2) * 32;
-    static constexpr int HALF = CH / 2;               // score columns per softmax thread
-    static constexpr int OSTRIDE = D + 4;             // staged output row (floats), padded
+    // the output is staged OCOLS columns at a time, rows padded by 4 floats
+    static constexpr int OCOLS = D < 128 ? D : 128;
+    static constexpr int OSTRIDE = OCOLS + 4;
+    // barriers, the TMEM address, each row's maximum and sum, agreement
+    // flags, then alignment slack
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 2 * M * 4 + 2 * 4 * 4 + 1024;
+    static constexpr int TMEM_COLS = 512;             // S at column 0, O at column CH
     static_assert(M * OSTRIDE * 4 <= BAR_OFF, "staged output fits the freed tiles");
     static_assert((BS % R == 0 || BS == 8) && D % 64 == 0, "shared-prefix shape");
     static_assert(CH + D <= TMEM_COLS, "S and O must fit TMEM");
@@ -111,9 +115,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* qs = smem + C::Q_OFF;
+    unsigned char* qs = smem + C::QV_OFF;                 // Q, then V
     unsigned char* ks = smem + C::K_OFF;                  // K tiles, then P
-    unsigned char* vs = smem + C::V_OFF;
+    unsigned char* vs = qs;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;                          // [NG]
@@ -122,6 +126,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     uint64_t* p_full = v_full + 2;
     uint64_t* o_full = v_full + 3;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+    float* row_m = reinterpret_cast<float*>(tmem_slot + 4);     // [M]
+    float* row_l = row_m + M;                                    // [M]
+    int* okw = reinterpret_cast<int*>(row_l + M);                // [2][SOFT_WARPS]
     // set by a role that gave up, read by the others after the final barrier
     __shared__ int failed;
 
@@ -140,6 +147,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t s_tmem = tmem, o_tmem = tmem + CH;
+    bool v_issued = false;                                // producer lane 0 only
 
     if (warp == C::PRODUCER) {
         // ------------------------------------------------ producer (lane 0) --
@@ -182,8 +190,15 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                 mbar_arrive_expect_tx(&k_full[g], 4 * KSL * R * 128 + a.tx_extra);
                 for (int j = 4 * g; j < 4 * g + 4; ++j) load_unit(&tm_k, ks, &k_full[g], j);
             }
-            mbar_arrive_expect_tx(v_full, C::KV_BYTES + a.tx_extra);
-            for (int j = 0; j < C::U; ++j) load_unit(&tm_v, vs, v_full, j);
+            // V goes over Q once the first MMA has read it
+            if (mbar_wait_bounded(s_full, 0, a.wait_ns)) {
+                mbar_arrive_expect_tx(v_full, C::KV_BYTES + a.tx_extra);
+                for (int j = 0; j < C::U; ++j) load_unit(&tm_v, vs, v_full, j);
+                v_issued = true;
+            } else {
+                raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+                failed = 1;
+            }
         }
     } else if (warp == C::MMA_WARP) {
         // --------------------------------------------- MMA issuer (lane 0) --
@@ -237,13 +252,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             else if (s_issued) (void)mbar_wait_bounded(s_full, 0, a.wait_ns);
         }
     } else {
-        // ------------------------------- softmax and epilogue: warps 0-7 --
-        // thread = (row r of TMEM lane quarter warp % 4, column half hf)
-        const int r = 32 * (warp & 3) + lane, hf = warp >> 2;
-        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-        float* xm = reinterpret_cast<float*>(smem + C::BAR_OFF + C::NBARS * 8 + 16);   // [2][M]
-        float* xl = xm + 2 * M;                                                        // [2][M]
-        int* okw = reinterpret_cast<int*>(xl + 2 * M);                                 // [2][8]
+        // -------------------------------- softmax and epilogue: warps 0-3 --
+        const int r = 32 * warp + lane;                   // this thread's query row / TMEM lane
+        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
         auto soft_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(32 * C::SOFT_WARPS) : "memory"); };
         // every softmax warp must agree before it depends on the others
         // (each agreement point has its own flags: a fast warp must not
@@ -257,108 +268,109 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             for (int w = 0; w < C::SOFT_WARPS; ++w) ok &= f[w];
             return ok != 0;
         };
-        float v[C::HALF];
-        float mloc = -INFINITY;
-        const bool s_ok = __all_sync(FULL_MASK, mbar_wait_bounded(s_full, 0, a.wait_ns));
-        if (s_ok) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int c = 0; c < C::HALF / 32; ++c) {
-                float t[32];
-                tmem_ld32(s_tmem + lane_off + hf * C::HALF + 32 * c, t);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[32 * c + j] = t[j];
-            }
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < C::HALF; ++j) {
-                v[j] = hf * C::HALF + j < valid ? v[j] * a.scale_log2 : -INFINITY;
-                mloc = fmaxf(mloc, v[j]);
-            }
-            xm[hf * M + r] = mloc;
-        }
-        bool ok = all_ok(0, s_ok);
-        float m = -INFINITY, lsum = 0.f;
+        float m = -INFINITY, l = 0.f;
+        bool ok = __all_sync(FULL_MASK, mbar_wait_bounded(s_full, 0, a.wait_ns));
         if (ok) {
-            m = fmaxf(xm[r], xm[M + r]);
-            // p = 2^(x - m) into this half of the P tile (bf16, 128-byte swizzle)
+            tc_fence_after_sync();
+            // pass 1: the row's maximum over the chunk's prefix tokens (log2
+            // units), 64 columns per TMEM round trip
+#pragma unroll 1
+            for (int c = 0; c < CH / 64; ++c) {
+                float v0[32], v1[32];
+                tmem_ld32(s_tmem + lane_off + 64 * c, v0);
+                tmem_ld32(s_tmem + lane_off + 64 * c + 32, v1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    if (64 * c + j < valid) m = fmaxf(m, v0[j] * a.scale_log2);
+                    if (64 * c + 32 + j < valid) m = fmaxf(m, v1[j] * a.scale_log2);
+                }
+            }
+            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum of p;
+            // 64 tokens = one slab row of 128 bytes per round trip
             const uint32_t prow = smem_addr(ks) + (uint32_t)r * 128;
+#pragma unroll 1
+            for (int c = 0; c < CH / 64; ++c) {
+                float v[64];
+                tmem_ld32(s_tmem + lane_off + 64 * c, *reinterpret_cast<float(*)[32]>(v));
+                tmem_ld32(s_tmem + lane_off + 64 * c + 32,
+                          *reinterpret_cast<float(*)[32]>(v + 32));
+                tmem_ld_wait();
+                uint32_t w[32];
 #pragma unroll
-            for (int c = 0; c < C::HALF / 32; ++c) {
-                uint32_t w[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float p0 = exp2_approx(v[32 * c + 2 * j] - m);
-                    const float p1 = exp2_approx(v[32 * c + 2 * j + 1] - m);
-                    lsum += p0 + p1;
+                for (int j = 0; j < 32; ++j) {
+                    const int t = 64 * c + 2 * j;
+                    const float p0 = t < valid ? exp2_approx(v[2 * j] * a.scale_log2 - m) : 0.f;
+                    const float p1 =
+                        t + 1 < valid ? exp2_approx(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
+                    l += p0 + p1;
                     w[j] = pack_bf16x2(p0, p1);
                 }
-                // tokens t0 .. t0+31 of the chunk: slab t0 / 64, 16-byte chunks 4 ((t0 / 32) % 2) ..
-                const int t0 = hf * C::HALF + 32 * c;
-                const uint32_t base = prow + (uint32_t)(t0 / 64) * (M * 128);
+                const uint32_t base = prow + (uint32_t)c * (M * 128);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int ch = 4 * ((t0 / 32) % 2) + q;
-                    const uint32_t addr = base + (uint32_t)((ch ^ (r & 7)) << 4);
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t addr = base + (uint32_t)((q ^ (r & 7)) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
                                  "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]),
                                  "r"(w[4 * q + 3])
                                  : "memory");
                 }
             }
-            xl[hf * M + r] = lsum;
+            row_m[r] = m;
+            row_l[r] = l;
             fence_proxy_async_smem();                   // P is read by the tensor cores
             tc_fence_before_sync();
             mbar_arrive(p_full);
-            const bool o_ok = __all_sync(FULL_MASK, mbar_wait_bounded(o_full, 0, a.wait_ns));
-            ok = all_ok(1, o_ok);
+            ok = __all_sync(FULL_MASK, mbar_wait_bounded(o_full, 0, a.wait_ns));
         }
+        ok = all_ok(0, ok);
         if (!ok) {
-            if (lane == 0 && warp == 0) {
+            if (r == 0) {
                 raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
                 failed = 1;
             }
         } else {
             tc_fence_after_sync();
-            // this thread's half of the row's output, staged row-major (padded
-            // rows) over the tiles, which no MMA or load uses any more
+            // the rows' output, OCOLS columns at a time: staged row-major
+            // (padded rows) over the tiles, which no MMA or load uses any more,
+            // then written as whole row segments with coalesced stores
             float* os = reinterpret_cast<float*>(smem);
-            constexpr int OH = D / 2;
+            constexpr int LPR = C::OCOLS / 4 < 32 ? C::OCOLS / 4 : 32;   // lanes per row
+            constexpr int VPL = C::OCOLS / 4 / LPR;                      // float4 per lane
+            const int tw = threadIdx.x;                                  // 0 .. 127
+#pragma unroll 1
+            for (int cb = 0; cb < D / C::OCOLS; ++cb) {
 #pragma unroll
-            for (int c = 0; c < OH / 32; ++c) {
-                float t[32];
-                tmem_ld32(o_tmem + lane_off + hf * OH + 32 * c, t);
-                tmem_ld_wait();
+                for (int c = 0; c < C::OCOLS / 32; ++c) {
+                    float t[32];
+                    tmem_ld32(o_tmem + lane_off + cb * C::OCOLS + 32 * c, t);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<float4*>(os + r * C::OSTRIDE + hf * OH + 32 * c + 4 * j) =
-                        make_float4(t[4 * j], t[4 * j + 1], t[4 * j + 2], t[4 * j + 3]);
-            }
-            soft_sync();
-            // whole rows to the workspace: D / 4 float4 per row, lanes split over rows
-            constexpr int LPR = D / 4 < 32 ? D / 4 : 32;           // lanes per row
-            constexpr int RPI = 32 / LPR;                          // rows per instruction
-            constexpr int VPL = D / 4 / LPR;                       // float4 per lane
-            const int tw = warp * 32 + lane;
-            for (int rr = tw / LPR; rr < M; rr += 32 * C::SOFT_WARPS / LPR) {
-                const int row = row0 + rr;
-                if (row >= rows) continue;
-                const int seq = gs + row / G, h = kvh * G + row % G;
-                const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride +
-                                    a.prefix_slot0 + chunk;
-                const int c4 = tw % LPR;
-#pragma unroll
-                for (int k = 0; k < VPL; ++k)
-                    reinterpret_cast<float4*>(a.ws_o + slot * D)[c4 + LPR * k] =
-                        *reinterpret_cast<const float4*>(os + rr * C::OSTRIDE + 4 * (c4 + LPR * k));
-                if (c4 == 0) {
-                    a.ws_m[slot] = fmaxf(xm[rr], xm[M + rr]);
-                    a.ws_l[slot] = xl[rr] + xl[M + rr];
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(os + r * C::OSTRIDE + 32 * c + 4 * j) =
+                            make_float4(t[4 * j], t[4 * j + 1], t[4 * j + 2], t[4 * j + 3]);
                 }
+                soft_sync();
+                for (int rr = tw / LPR; rr < M; rr += 32 * C::SOFT_WARPS / LPR) {
+                    const int row = row0 + rr;
+                    if (row >= rows) continue;
+                    const int seq = gs + row / G, h = kvh * G + row % G;
+                    const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride +
+                                        a.prefix_slot0 + chunk;
+                    const int c4 = tw % LPR;
+                    float4* dst = reinterpret_cast<float4*>(a.ws_o + slot * D + cb * C::OCOLS);
+#pragma unroll
+                    for (int k = 0; k < VPL; ++k)
+                        dst[c4 + LPR * k] = *reinterpret_cast<const float4*>(
+                            os + rr * C::OSTRIDE + 4 * (c4 + LPR * k));
+                    if (cb == 0 && c4 == 0) {
+                        a.ws_m[slot] = row_m[rr];
+                        a.ws_l[slot] = row_l[rr];
+                    }
+                }
+                soft_sync();                            // the staging area is reused
             }
-            (void)RPI;
         }
-        (void)m;
     }
 
     // ---------------- teardown: every role is done with TMEM and shared memory --
@@ -368,7 +380,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
         // loads may still be in flight after a role gave up: wait (bounded) for them
         (void)mbar_wait_bounded(q_full, 0, a.wait_ns);
         for (int g = 0; g < NG; ++g) (void)mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
-        (void)mbar_wait_bounded(v_full, 0, a.wait_ns);
+        if (v_issued) (void)mbar_wait_bounded(v_full, 0, a.wait_ns);
     }
     if (warp == C::MMA_WARP) {
         tc_fence_after_sync();
