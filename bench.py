@@ -18,7 +18,11 @@ pool 110 % of the blocks in use, synthetic N(0,1) data.
 Reported line (rank 0):
   value      KV-read GB/s over the K timed steps, inputs resident in HBM
              (per-step allocator outputs are computed before timing), max
-             over ranks, whole job (all replicas).
+             over ranks, whole job (all replicas).  The K steps are captured
+             once into a CUDA graph and replayed once in the timed region
+             (the same launches without the host's issue cost between them,
+             as a serving loop replays its decode step); --eager launches
+             them one by one from Python instead.
   e2e        the same metric through the public API with host buffers: the
              live allocator on the host, pinned H2D copies of each step's
              q / new K,V / slots / lengths / copy-on-write pairs, the table
@@ -581,15 +585,16 @@ def run_other_configs(dev, local, peak, steps=10, warmup=3):
     """The other decode workloads, measured briefly after the headline run:
     MHA batch 64 (fused append + decode), the long-context split at the
     config's 512-token partitions, and the prefix-sharing batch (block 16,
-    head_dim 128) with plain decode and with the cascade.  Each builds its
-    own pool, runs ``warmup`` + ``steps`` device-timed steps and is freed."""
+    head_dim 128) with plain decode (fused append + decode) and with the
+    cascade.  Each builds its own pool, runs ``warmup`` eager steps and
+    ``steps`` device-timed steps replayed as one CUDA graph, and is freed."""
     out = []
     extra = 2 * (steps + warmup) + 4
 
     def run(build, label, kernel, fused=False, unique=False):
         loop = build()
         loop.fused = fused
-        res = run_device_timed(loop, steps, warmup, 1, local, unique=unique)
+        res = run_device_timed(loop, steps, warmup, 1, local, unique=unique, graph=True)
         out.append(_config_entry(loop, res, steps, peak, label, kernel))
         del loop
         torch.cuda.synchronize()
@@ -601,7 +606,7 @@ def run_other_configs(dev, local, peak, steps=10, warmup=3):
     run(lambda: DecodeLoop(make_problem("long", extra, 0), dev, "split", 512),
         "long_context_split_p512", "pa_decode_split")
     plain = run(lambda: build_prefix_loop(dev, extra, "decode", 512, 16, 128),
-                "prefix_sharing_b64_bs16_d128", "pa_decode", unique=True)
+                "prefix_sharing_b64_bs16_d128", "pa_decode_append", fused=True, unique=True)
     casc = run(lambda: build_prefix_loop(dev, extra, "cascade", 512, 16, 128),
                "prefix_sharing_b64_bs16_d128", "pa_decode_shared_prefix", unique=True)
     casc["speedup_vs_pa_decode"] = round(plain["ms_per_step"] / casc["ms_per_step"], 3)
@@ -887,8 +892,8 @@ def workload_config(p, args):
             "kernel": args.kernel + ("+append (fused)" if args.fused else ""),
             "partition": args.partition,
             "pdl": not getattr(args, "no_pdl", False),
-            "timed_steps": "one CUDA graph replay" if getattr(args, "graph", False)
-                           else "eager launches",
+            "timed_steps": "eager launches" if getattr(args, "eager", False)
+                           else "one CUDA graph replay",
             "l2": "inputs larger than L2 (KV cache %.2f GB vs 126 MB L2), no flush" %
                   (decode_kv_bytes(lens, p) / 1e9)}
 
@@ -918,9 +923,10 @@ def main():
                     help="gqa / prefix workloads: block size (default 16)")
     ap.add_argument("--head-dim", type=int, default=None,
                     help="gqa / prefix workloads: head_dim (default 128)")
-    ap.add_argument("--graph", action="store_true",
-                    help="device-timed loop: capture the timed steps in one CUDA graph and "
-                         "replay it (same launches, no host issue cost between them)")
+    ap.add_argument("--eager", action="store_true",
+                    help="device-timed loop: launch the timed steps one by one from Python "
+                         "instead of replaying them as one CUDA graph (the default: the same "
+                         "launches without the host's issue cost between them)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch (PA_OPT_PDL 0)")
     ap.add_argument("--compact", action="store_true",
@@ -975,7 +981,7 @@ def main():
             loop = DecodeLoop(p, dev, args.kernel, args.partition)
         loop.fused = args.fused
         res = run_device_timed(loop, args.steps, args.warmup, world, local,
-                               unique=args.workload == "prefix", graph=args.graph)
+                               unique=args.workload == "prefix", graph=not args.eager)
         e2e = None if args.no_e2e else run_e2e(loop, args.steps, args.warmup, world)
 
         ms = reduce_scalar(res["ms"], "max", world, dev)

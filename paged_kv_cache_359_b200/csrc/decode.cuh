@@ -194,9 +194,11 @@ __device__ __forceinline__ void append_row(const DecodeArgs& a, int seq, int kvh
 // Kernel instances: Decode = pa_decode's longest-first grid (one CTA per
 // item), Cluster = pa_decode with several CTAs per item merged through
 // distributed shared memory, Split = pa_decode_split's partitions, Own = the
-// shared-prefix decode's own-token pass (longest-first, half the warps of
-// Decode so that two CTAs fit an SM beside a shared-pass CTA).  Each is its
-// own instance so that a kernel carries only its own path's code.
+// shared-prefix decode's own-token pass (longest-first; at head_dim 64 and
+// 256 with half the warps of Decode, so that more of its CTAs fit the SMs
+// beside the shared-pass CTAs -- measured faster there; at head_dim 128 the
+// full-width CTA, whose shorter items win).  Each is its own instance so
+// that a kernel carries only its own path's code.
 enum class Mode { Decode, Cluster, Split, Own };
 
 // ============================================================ CoreUnit ==
@@ -770,12 +772,16 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
     fence_proxy_async_smem();
 }
 
+// Whether the own-token pass of the shared-prefix decode runs half-width CTAs.
+template <class U>
+__host__ __device__ constexpr bool own_half_width() { return U::D != 128; }
+
 template <class U, Mode MODE>
-__global__ void __launch_bounds__(Layout<U, MODE == Mode::Own>::NW * 32)
+__global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<U>()>::NW * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeArgs a) {
     using T = typename U::T;
-    using Ly = Layout<U, MODE == Mode::Own>;
+    using Ly = Layout<U, MODE == Mode::Own && own_half_width<U>()>;
     constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
     constexpr int NT = NW * 32;
     // The own-token pass of the shared-prefix decode reads nothing the

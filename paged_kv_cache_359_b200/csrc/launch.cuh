@@ -103,8 +103,8 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
                 if (e != cudaSuccess)
                     return fail(PA_ERR_CUDA, "shared-prefix launch: %s", cudaGetErrorString(e));
             }
-            // the own-token pass: longest-first, half-width CTAs
-            using Lo = Layout<U, true>;
+            // the own-token pass: longest-first (half-width CTAs but at head_dim 128)
+            using Lo = Layout<U, own_half_width<U>()>;
             static std::atomic<unsigned long long> done_o{0};
             auto ok = paged_decode_kernel<U, Mode::Own>;
             if (pa_status s = allow_smem(ok, Lo::SMEM_BYTES, done_o)) return s;
