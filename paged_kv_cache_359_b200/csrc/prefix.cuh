@@ -28,11 +28,11 @@
 //    maximum of the row's scores over the chunk (masked past the prefix),
 //    then p = 2^(s * scale * log2 e - max), rounded to bf16, into the
 //    swizzled P tile (which reuses the K tile's space) and the fp32 sum of p;
-//    after the second MMA the threads stage the rows' output in the (now
-//    free) tiles, up to 128 columns at a time, and the warps write whole
-//    rows to the workspace slot prefix_slot0 + chunk with coalesced stores,
-//    with each row's maximum and sum; pa_decode's CTAs for each sequence's
-//    own tokens merge these into the output.
+//    after the second MMA each thread stages its row's output in the (now
+//    free) tiles, up to 128 columns at a time, and sends it with one TMA
+//    bulk copy to the workspace slot prefix_slot0 + chunk, with the row's
+//    maximum and sum; pa_decode's CTAs for each sequence's own tokens merge
+//    these into the output.
 // Every wait is bounded; a wait that runs out sets PA_DEVERR_WAIT_TIMEOUT,
 // the CTA skips what depends on it, waits (bounded) for its own loads and
 // MMAs, frees its TMEM and leaves without writing.
@@ -68,9 +68,8 @@ struct PrefixCfg {
     // the output is staged OCOLS columns at a time, rows padded by 4 floats
     static constexpr int OCOLS = D < 128 ? D : 128;
     static constexpr int OSTRIDE = OCOLS + 4;
-    // barriers, the TMEM address, each row's maximum and sum, agreement
-    // flags, then alignment slack
-    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 2 * M * 4 + 2 * 4 * 4 + 1024;
+    // barriers, the TMEM address, agreement flags, then alignment slack
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 2 * 4 * 4 + 1024;
     static constexpr int TMEM_COLS = 512;             // S at column 0, O at column CH
     static_assert(M * OSTRIDE * 4 <= BAR_OFF, "staged output fits the freed tiles");
     static_assert((BS % R == 0 || BS == 8) && D % 64 == 0, "shared-prefix shape");
@@ -126,9 +125,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     uint64_t* p_full = v_full + 2;
     uint64_t* o_full = v_full + 3;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
-    float* row_m = reinterpret_cast<float*>(tmem_slot + 4);     // [M]
-    float* row_l = row_m + M;                                    // [M]
-    int* okw = reinterpret_cast<int*>(row_l + M);                // [2][SOFT_WARPS]
+    int* okw = reinterpret_cast<int*>(tmem_slot + 4);             // [2][SOFT_WARPS]
     // set by a role that gave up, read by the others after the final barrier
     __shared__ int failed;
 
@@ -204,6 +201,11 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
         // --------------------------------------------- MMA issuer (lane 0) --
         if (lane == 0) {
             const uint32_t q0 = smem_addr(qs), k0 = smem_addr(ks), v0 = smem_addr(vs);
+            // base descriptors; a step's operand is the base plus a byte
+            // offset (>> 4) added to the start-address field, which stays
+            // inside its 14 bits for any shared-memory address
+            const uint64_t qd = sw128_desc(q0, 16, 1024), kd = sw128_desc(k0, 16, 1024);
+            const uint64_t pd = kd, vd = sw128_desc(v0, CH * 128, 1024);
             bool ok = mbar_wait_bounded(q_full, 0, a.wait_ns);
             bool s_issued = false;
             if (ok) {
@@ -213,10 +215,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                     tc_fence_after_sync();
 #pragma unroll
                     for (int kk = 0; kk < 4 * KSL; ++kk) {
-                        const uint64_t ad = sw128_desc(q0 + (kk / 4) * M * 128 + (kk % 4) * 32,
-                                                       16, 1024);
-                        const uint64_t bd = sw128_desc(
-                            k0 + (kk / 4) * CH * 128 + g * 64 * 128 + (kk % 4) * 32, 16, 1024);
+                        const uint64_t ad = qd + (uint64_t)(((kk / 4) * M * 128 + (kk % 4) * 32) >> 4);
+                        const uint64_t bd =
+                            kd + (uint64_t)(((kk / 4) * CH * 128 + g * 64 * 128 + (kk % 4) * 32) >> 4);
                         umma_bf16(s_tmem + 64 * g, ad, bd, umma_idesc_bf16(M, 64, false),
                                   kk > 0);
                     }
@@ -233,11 +234,10 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                 tc_fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < CH / 16; ++kk) {
-                    const uint64_t ad =
-                        sw128_desc(k0 + (kk / 4) * M * 128 + (kk % 4) * 32, 16, 1024);
+                    const uint64_t ad = pd + (uint64_t)(((kk / 4) * M * 128 + (kk % 4) * 32) >> 4);
                     // V as B, MN-major: 64-dim slabs CH * 128 bytes apart (leading
                     // offset), 8-token atoms 1 KiB apart (stride offset)
-                    const uint64_t bd = sw128_desc(v0 + kk * 16 * 128, CH * 128, 1024);
+                    const uint64_t bd = vd + (uint64_t)((kk * 16 * 128) >> 4);
                     umma_bf16(o_tmem, ad, bd, umma_idesc_bf16(M, D, true), kk > 0);
                 }
                 umma_commit(o_full);
@@ -273,51 +273,57 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
         if (ok) {
             tc_fence_after_sync();
             // pass 1: the row's maximum over the chunk's prefix tokens (log2
-            // units), 64 columns per TMEM round trip
+            // units); a TMEM load costs a round trip of several hundred
+            // cycles, so each one brings TW columns (four 32-column loads,
+            // one wait)
+            constexpr int TW = CH < 128 ? CH : 128;
 #pragma unroll 1
-            for (int c = 0; c < CH / 64; ++c) {
-                float v0[32], v1[32];
-                tmem_ld32(s_tmem + lane_off + 64 * c, v0);
-                tmem_ld32(s_tmem + lane_off + 64 * c + 32, v1);
+            for (int c = 0; c < CH / TW; ++c) {
+                float v[TW];
+#pragma unroll
+                for (int q = 0; q < TW / 32; ++q)
+                    tmem_ld32(s_tmem + lane_off + TW * c + 32 * q,
+                              *reinterpret_cast<float(*)[32]>(v + 32 * q));
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    if (64 * c + j < valid) m = fmaxf(m, v0[j] * a.scale_log2);
-                    if (64 * c + 32 + j < valid) m = fmaxf(m, v1[j] * a.scale_log2);
-                }
+                for (int j = 0; j < TW; ++j)
+                    if (TW * c + j < valid) m = fmaxf(m, v[j] * a.scale_log2);
             }
-            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum of p;
-            // 64 tokens = one slab row of 128 bytes per round trip
+            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum
+            // of p; 64 tokens make one 128-byte row of a P slab
             const uint32_t prow = smem_addr(ks) + (uint32_t)r * 128;
 #pragma unroll 1
-            for (int c = 0; c < CH / 64; ++c) {
-                float v[64];
-                tmem_ld32(s_tmem + lane_off + 64 * c, *reinterpret_cast<float(*)[32]>(v));
-                tmem_ld32(s_tmem + lane_off + 64 * c + 32,
-                          *reinterpret_cast<float(*)[32]>(v + 32));
+            for (int c = 0; c < CH / TW; ++c) {
+                float v[TW];
+#pragma unroll
+                for (int q = 0; q < TW / 32; ++q)
+                    tmem_ld32(s_tmem + lane_off + TW * c + 32 * q,
+                              *reinterpret_cast<float(*)[32]>(v + 32 * q));
                 tmem_ld_wait();
-                uint32_t w[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int t = 64 * c + 2 * j;
-                    const float p0 = t < valid ? exp2_approx(v[2 * j] * a.scale_log2 - m) : 0.f;
-                    const float p1 =
-                        t + 1 < valid ? exp2_approx(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
-                    l += p0 + p1;
-                    w[j] = pack_bf16x2(p0, p1);
-                }
-                const uint32_t base = prow + (uint32_t)c * (M * 128);
+                for (int h = 0; h < TW / 64; ++h) {
+                    const int t0 = TW * c + 64 * h;             // first token of this slab row
+                    uint32_t w[32];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t addr = base + (uint32_t)((q ^ (r & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                 "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]),
-                                 "r"(w[4 * q + 3])
-                                 : "memory");
+                    for (int j = 0; j < 32; ++j) {
+                        const int t = t0 + 2 * j;
+                        const float x0 = v[64 * h + 2 * j], x1 = v[64 * h + 2 * j + 1];
+                        const float p0 = t < valid ? exp2_approx(x0 * a.scale_log2 - m) : 0.f;
+                        const float p1 = t + 1 < valid ? exp2_approx(x1 * a.scale_log2 - m) : 0.f;
+                        l += p0 + p1;
+                        w[j] = pack_bf16x2(p0, p1);
+                    }
+                    const uint32_t base = prow + (uint32_t)(t0 / 64) * (M * 128);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t addr = base + (uint32_t)((q ^ (r & 7)) << 4);
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                     "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]),
+                                     "r"(w[4 * q + 3])
+                                     : "memory");
+                    }
                 }
             }
-            row_m[r] = m;
-            row_l[r] = l;
             fence_proxy_async_smem();                   // P is read by the tensor cores
             tc_fence_before_sync();
             mbar_arrive(p_full);
@@ -331,44 +337,38 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             }
         } else {
             tc_fence_after_sync();
-            // the rows' output, OCOLS columns at a time: staged row-major
-            // (padded rows) over the tiles, which no MMA or load uses any more,
-            // then written as whole row segments with coalesced stores
-            float* os = reinterpret_cast<float*>(smem);
-            constexpr int LPR = C::OCOLS / 4 < 32 ? C::OCOLS / 4 : 32;   // lanes per row
-            constexpr int VPL = C::OCOLS / 4 / LPR;                      // float4 per lane
-            const int tw = threadIdx.x;                                  // 0 .. 127
+            // the row's output, OCOLS columns at a time: this thread stages
+            // its row (padded rows, over the tiles no MMA or load uses any
+            // more) and sends it to the workspace with one bulk copy
+            float* os = reinterpret_cast<float*>(smem) + r * C::OSTRIDE;
+            const int row = row0 + r;
+            const bool mine = row < rows;
+            const int seq = gs + row / G, h = kvh * G + row % G;
+            const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride +
+                                a.prefix_slot0 + chunk;
 #pragma unroll 1
             for (int cb = 0; cb < D / C::OCOLS; ++cb) {
+                if (cb > 0) bulk_wait_read();           // the staging row is free again
+                float t[C::OCOLS];
 #pragma unroll
-                for (int c = 0; c < C::OCOLS / 32; ++c) {
-                    float t[32];
-                    tmem_ld32(o_tmem + lane_off + cb * C::OCOLS + 32 * c, t);
-                    tmem_ld_wait();
+                for (int c = 0; c < C::OCOLS / 32; ++c)
+                    tmem_ld32(o_tmem + lane_off + cb * C::OCOLS + 32 * c,
+                              *reinterpret_cast<float(*)[32]>(t + 32 * c));
+                tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<float4*>(os + r * C::OSTRIDE + 32 * c + 4 * j) =
-                            make_float4(t[4 * j], t[4 * j + 1], t[4 * j + 2], t[4 * j + 3]);
+                for (int j = 0; j < C::OCOLS / 4; ++j)
+                    *reinterpret_cast<float4*>(os + 4 * j) =
+                        make_float4(t[4 * j], t[4 * j + 1], t[4 * j + 2], t[4 * j + 3]);
+                if (mine) {
+                    fence_proxy_async_smem();           // the bulk copy reads the row
+                    bulk_store(a.ws_o + slot * D + cb * C::OCOLS, os, C::OCOLS * 4);
+                    bulk_commit();
                 }
-                soft_sync();
-                for (int rr = tw / LPR; rr < M; rr += 32 * C::SOFT_WARPS / LPR) {
-                    const int row = row0 + rr;
-                    if (row >= rows) continue;
-                    const int seq = gs + row / G, h = kvh * G + row % G;
-                    const size_t slot = ((size_t)seq * a.num_heads + h) * a.slot_stride +
-                                        a.prefix_slot0 + chunk;
-                    const int c4 = tw % LPR;
-                    float4* dst = reinterpret_cast<float4*>(a.ws_o + slot * D + cb * C::OCOLS);
-#pragma unroll
-                    for (int k = 0; k < VPL; ++k)
-                        dst[c4 + LPR * k] = *reinterpret_cast<const float4*>(
-                            os + rr * C::OSTRIDE + 4 * (c4 + LPR * k));
-                    if (cb == 0 && c4 == 0) {
-                        a.ws_m[slot] = row_m[rr];
-                        a.ws_l[slot] = row_l[rr];
-                    }
-                }
-                soft_sync();                            // the staging area is reused
+            }
+            if (mine) {
+                a.ws_m[slot] = m;
+                a.ws_l[slot] = l;
+                bulk_wait();                            // complete before the CTA leaves
             }
         }
     }
