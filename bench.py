@@ -697,6 +697,7 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
 
     bufs = [Buf() for _ in range(ring)]
     counts = {"h2d": 0, "d2h": 0, "kv": 0}
+    pairs_h = np.zeros((s, 2), dtype=np.int32)          # copy-on-write pairs of a step
 
     def read_back(b):
         b.d2h.synchronize()
@@ -707,9 +708,10 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
         b = bufs[i % ring]
         if b.used:
             read_back(b)                               # step i - ring is done with b
-        sl, cw = loop.alloc.append_slots(tables_np, lens_np)
+        # the allocator writes the step's slots straight into the pinned metadata
+        _, cw = loop.alloc.append_slots(tables_np, lens_np, slots_out=b.slots_h,
+                                        pairs_out=pairs_h)
         b.lens_h[:] = lens_np
-        b.slots_h[:] = sl
         n = len(cw)
         if n:
             b.cows_h[:n] = cw

@@ -355,18 +355,26 @@ class BlockAllocator:
                                              ctypes.byref(dst)))
         return slot.value, ((src.value, dst.value) if src.value >= 0 else None), ln.value
 
-    def append_slots(self, tables: np.ndarray, lengths: np.ndarray):
+    def append_slots(self, tables: np.ndarray, lengths: np.ndarray, slots_out=None,
+                     pairs_out=None):
         """tables int32 [S, stride], lengths int32 [S] (both mutated).
-        Returns (slots int64 [S], cow_pairs int32 [n, 2])."""
+        Returns (slots int64 [S], cow_pairs int32 [n, 2]).  With slots_out
+        (int64 [S]) and pairs_out (int32 [S, 2]) given, the results are
+        written there and views of them returned (nothing is allocated)."""
         s = tables.shape[0]
-        slots = np.zeros(s, dtype=np.int64)
-        pairs = np.zeros((max(s, 1), 2), dtype=np.int32)
+        if lengths.dtype != np.intc or not lengths.flags["C_CONTIGUOUS"]:
+            raise ValueError("lengths must be a contiguous int32 array")
+        slots = np.zeros(s, dtype=np.int64) if slots_out is None else slots_out
+        pairs = np.zeros((max(s, 1), 2), dtype=np.int32) if pairs_out is None else pairs_out
+        if slots.dtype != np.int64 or slots.shape != (s,) or not slots.flags["C_CONTIGUOUS"]:
+            raise ValueError("slots_out must be a contiguous int64 [num_seqs] array")
+        if pairs.dtype != np.int32 or pairs.shape[0] < max(s, 1) or not pairs.flags["C_CONTIGUOUS"]:
+            raise ValueError("pairs_out must be a contiguous int32 [num_seqs, 2] array")
         n = ctypes.c_int(0)
         self._check(lib().pa_seq_append_slots(
-            self._h, _i32(tables), tables.shape[1],
-            lengths.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), s,
-            slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _i32(pairs), ctypes.byref(n)))
-        return slots, pairs[: n.value].copy()
+            self._h, _i32(tables), tables.shape[1], lengths.ctypes.data, s,
+            slots.ctypes.data, pairs.ctypes.data, ctypes.byref(n)))
+        return slots, (pairs[: n.value].copy() if pairs_out is None else pairs[: n.value])
 
     def extend(self, table: np.ndarray, length: int, num_tokens: int, want_slots: bool = True):
         ln = ctypes.c_int(length)

@@ -72,7 +72,7 @@ SIGNATURES = {
     "pa_alloc_ref_count": (_c_int, [_vp, ctypes.c_int32]),
     "pa_alloc_free_order": (_c_int, [_vp, _i32p, _c_int, _intp]),
     "pa_seq_append_slot": (_c_int, [_vp, _i32p, _c_int, _intp, _i64p, _i32p, _i32p]),
-    "pa_seq_append_slots": (_c_int, [_vp, _i32p, _c_int, _intp, _c_int, _i64p, _i32p, _intp]),
+    "pa_seq_append_slots": (_c_int, [_vp, _i32p, _c_int, _vp, _c_int, _vp, _vp, _intp]),
     "pa_seq_extend": (_c_int, [_vp, _i32p, _c_int, _intp, _c_int, _i64p, _i32p, _i32p]),
     "pa_seq_fork": (_c_int, [_vp, _i32p, _c_int, _i32p]),
     "pa_seq_free": (_c_int, [_vp, _i32p, _c_int]),

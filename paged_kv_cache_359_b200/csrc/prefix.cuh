@@ -273,55 +273,47 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
         if (ok) {
             tc_fence_after_sync();
             // pass 1: the row's maximum over the chunk's prefix tokens (log2
-            // units); a TMEM load costs a round trip of several hundred
-            // cycles, so each one brings TW columns (four 32-column loads,
-            // one wait)
-            constexpr int TW = CH < 128 ? CH : 128;
+            // units), 64 columns per TMEM round trip
 #pragma unroll 1
-            for (int c = 0; c < CH / TW; ++c) {
-                float v[TW];
-#pragma unroll
-                for (int q = 0; q < TW / 32; ++q)
-                    tmem_ld32(s_tmem + lane_off + TW * c + 32 * q,
-                              *reinterpret_cast<float(*)[32]>(v + 32 * q));
+            for (int c = 0; c < CH / 64; ++c) {
+                float v0[32], v1[32];
+                tmem_ld32(s_tmem + lane_off + 64 * c, v0);
+                tmem_ld32(s_tmem + lane_off + 64 * c + 32, v1);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < TW; ++j)
-                    if (TW * c + j < valid) m = fmaxf(m, v[j] * a.scale_log2);
+                for (int j = 0; j < 32; ++j) {
+                    if (64 * c + j < valid) m = fmaxf(m, v0[j] * a.scale_log2);
+                    if (64 * c + 32 + j < valid) m = fmaxf(m, v1[j] * a.scale_log2);
+                }
             }
-            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum
-            // of p; 64 tokens make one 128-byte row of a P slab
+            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum of p;
+            // 64 tokens = one slab row of 128 bytes per round trip
             const uint32_t prow = smem_addr(ks) + (uint32_t)r * 128;
 #pragma unroll 1
-            for (int c = 0; c < CH / TW; ++c) {
-                float v[TW];
-#pragma unroll
-                for (int q = 0; q < TW / 32; ++q)
-                    tmem_ld32(s_tmem + lane_off + TW * c + 32 * q,
-                              *reinterpret_cast<float(*)[32]>(v + 32 * q));
+            for (int c = 0; c < CH / 64; ++c) {
+                float v[64];
+                tmem_ld32(s_tmem + lane_off + 64 * c, *reinterpret_cast<float(*)[32]>(v));
+                tmem_ld32(s_tmem + lane_off + 64 * c + 32,
+                          *reinterpret_cast<float(*)[32]>(v + 32));
                 tmem_ld_wait();
+                uint32_t w[32];
 #pragma unroll
-                for (int h = 0; h < TW / 64; ++h) {
-                    const int t0 = TW * c + 64 * h;             // first token of this slab row
-                    uint32_t w[32];
+                for (int j = 0; j < 32; ++j) {
+                    const int t = 64 * c + 2 * j;
+                    const float p0 = t < valid ? exp2_approx(v[2 * j] * a.scale_log2 - m) : 0.f;
+                    const float p1 =
+                        t + 1 < valid ? exp2_approx(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
+                    l += p0 + p1;
+                    w[j] = pack_bf16x2(p0, p1);
+                }
+                const uint32_t base = prow + (uint32_t)c * (M * 128);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int t = t0 + 2 * j;
-                        const float x0 = v[64 * h + 2 * j], x1 = v[64 * h + 2 * j + 1];
-                        const float p0 = t < valid ? exp2_approx(x0 * a.scale_log2 - m) : 0.f;
-                        const float p1 = t + 1 < valid ? exp2_approx(x1 * a.scale_log2 - m) : 0.f;
-                        l += p0 + p1;
-                        w[j] = pack_bf16x2(p0, p1);
-                    }
-                    const uint32_t base = prow + (uint32_t)(t0 / 64) * (M * 128);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint32_t addr = base + (uint32_t)((q ^ (r & 7)) << 4);
-                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                                     "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]),
-                                     "r"(w[4 * q + 3])
-                                     : "memory");
-                    }
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t addr = base + (uint32_t)((q ^ (r & 7)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]),
+                                 "r"(w[4 * q + 3])
+                                 : "memory");
                 }
             }
             fence_proxy_async_smem();                   // P is read by the tensor cores
@@ -349,16 +341,16 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
 #pragma unroll 1
             for (int cb = 0; cb < D / C::OCOLS; ++cb) {
                 if (cb > 0) bulk_wait_read();           // the staging row is free again
-                float t[C::OCOLS];
 #pragma unroll
-                for (int c = 0; c < C::OCOLS / 32; ++c)
-                    tmem_ld32(o_tmem + lane_off + cb * C::OCOLS + 32 * c,
-                              *reinterpret_cast<float(*)[32]>(t + 32 * c));
-                tmem_ld_wait();
+                for (int c = 0; c < C::OCOLS / 32; ++c) {
+                    float t[32];
+                    tmem_ld32(o_tmem + lane_off + cb * C::OCOLS + 32 * c, t);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < C::OCOLS / 4; ++j)
-                    *reinterpret_cast<float4*>(os + 4 * j) =
-                        make_float4(t[4 * j], t[4 * j + 1], t[4 * j + 2], t[4 * j + 3]);
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(os + 32 * c + 4 * j) =
+                            make_float4(t[4 * j], t[4 * j + 1], t[4 * j + 2], t[4 * j + 3]);
+                }
                 if (mine) {
                     fence_proxy_async_smem();           // the bulk copy reads the row
                     bulk_store(a.ws_o + slot * D + cb * C::OCOLS, os, C::OCOLS * 4);
