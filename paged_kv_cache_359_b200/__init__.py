@@ -304,13 +304,17 @@ class BlockAllocator:
         if not h:
             raise PagedAttnError(1, lib().pa_last_error().decode())
         self._h = ctypes.c_void_p(h)
+        # held here so that destruction works during interpreter shutdown,
+        # when module globals may already be gone
+        self._destroy = lib().pa_alloc_destroy
         self.num_blocks = num_blocks
         self.block_size = block_size
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            lib().pa_alloc_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self._h = None
 
     @staticmethod

@@ -73,6 +73,21 @@ inline void append_one(pa_allocator* a, int32_t* table, int* length, int64_t* sl
     *length = len + 1;
 }
 
+// The table entry an append reads: the block holding the last token, when
+// that block still has room (a full last block is not read: a fresh one
+// follows).  An append touches nothing else, so this is the only entry it
+// needs to trust; checking the whole table on every step would cost a random
+// read per block of every sequence.
+pa_status check_last_entry(const pa_allocator* a, const int32_t* table, int len) {
+    const int bs = a->block_size;
+    if (len % bs == 0) return PA_OK;
+    const int32_t b = table[len / bs];
+    if (!valid_block(a, b) || a->ref[b] <= 0)
+        return pa::fail(PA_ERR_BAD_BLOCK_ID, "table entry %d (%d) is not an allocated block",
+                        len / bs, (int)b);
+    return PA_OK;
+}
+
 pa_status check_table(const pa_allocator* a, const int32_t* table, int n) {
     for (int i = 0; i < n; ++i) {
         if (!valid_block(a, table[i]) || a->ref[table[i]] <= 0)
@@ -159,8 +174,7 @@ pa_status pa_seq_append_slot(pa_allocator* a, int32_t* table, int capacity, int*
         return pa::fail(PA_ERR_INVALID_ARG, "null argument or negative length");
     const int bs = a->block_size;
     const int len = *length;
-    const int nb = blocks_for(len, bs);
-    if (pa_status s = check_table(a, table, nb)) return s;
+    if (pa_status s = check_last_entry(a, table, len)) return s;
     const bool fresh = len % bs == 0;
     if (fresh && len / bs >= capacity)
         return pa::fail(PA_ERR_INVALID_ARG, "block table full (capacity %d)", capacity);
@@ -184,7 +198,7 @@ pa_status pa_seq_append_slots(pa_allocator* a, int32_t* tables, int stride, int*
         const int len = lengths[i];
         if (len < 0) return pa::fail(PA_ERR_INVALID_ARG, "negative length for sequence %d", i);
         int32_t* t = tables + (int64_t)i * stride;
-        if (pa_status s = check_table(a, t, blocks_for(len, bs))) return s;
+        if (pa_status s = check_last_entry(a, t, len)) return s;
         if (len % bs == 0) {
             if (len / bs >= stride)
                 return pa::fail(PA_ERR_INVALID_ARG, "block table %d full (stride %d)", i, stride);
