@@ -708,6 +708,10 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
         b = bufs[i % ring]
         if b.used:
             read_back(b)                               # step i - ring is done with b
+        # q and the new rows do not depend on the allocator: their upload goes
+        # out first, and the allocator's work overlaps it
+        with torch.cuda.stream(up):
+            b.inp.copy_(host[i], non_blocking=True)
         # the allocator writes the step's slots straight into the pinned metadata
         _, cw = loop.alloc.append_slots(tables_np, lens_np, slots_out=b.slots_h,
                                         pairs_out=pairs_h)
@@ -717,7 +721,6 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
             b.cows_h[:n] = cw
         meta_used = cow_off + 16 * n                   # lengths, slots, this step's pairs
         with torch.cuda.stream(up):
-            b.inp.copy_(host[i], non_blocking=True)
             b.meta[:meta_used].copy_(b.meta_h[:meta_used], non_blocking=True)
             b.h2d.record(up)
         comp.wait_event(b.h2d)
