@@ -60,8 +60,8 @@ struct PrefixCfg {
     // Q, then V over the same bytes; K, then P over the same bytes
     static constexpr int QV_OFF = 0, K_OFF = QV_BYTES;
     static constexpr int BAR_OFF = QV_BYTES + KP_BYTES;
-    // q_full, k_full[NG], v_full, s_full, p_full, o_full; then the TMEM address
-    static constexpr int NBARS = NG + 5;
+    // q_full, k_full[NG], v_full, s_full[NG], p_full, o_full; then the TMEM address
+    static constexpr int NBARS = 2 * NG + 4;
     static constexpr int SOFT_WARPS = 4;
     static constexpr int PRODUCER = SOFT_WARPS, MMA_WARP = SOFT_WARPS + 1;
     static constexpr int THREADS = (SOFT_WARPS + 2) * 32;
@@ -121,9 +121,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;                          // [NG]
     uint64_t* v_full = bars + 1 + NG;
-    uint64_t* s_full = v_full + 1;
-    uint64_t* p_full = v_full + 2;
-    uint64_t* o_full = v_full + 3;
+    uint64_t* s_full = v_full + 1;                        // [NG]: S of 64-token group g done
+    uint64_t* p_full = s_full + NG;
+    uint64_t* o_full = p_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
     int* okw = reinterpret_cast<int*>(tmem_slot + 4);             // [2][SOFT_WARPS]
     // set by a role that gave up, read by the others after the final barrier
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     if (threadIdx.x == 0) {
         failed = 0;
         for (int i = 0; i < C::NBARS; ++i)
-            mbar_init(&bars[i], i == NG + 3 ? 32 * C::SOFT_WARPS : 1);
+            mbar_init(&bars[i], i == 2 * NG + 2 ? 32 * C::SOFT_WARPS : 1);
         fence_mbar_init();
     }
     if (warp == C::MMA_WARP) {                            // the MMA warp owns TMEM
@@ -187,8 +187,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                 mbar_arrive_expect_tx(&k_full[g], 4 * KSL * R * 128 + a.tx_extra);
                 for (int j = 4 * g; j < 4 * g + 4; ++j) load_unit(&tm_k, ks, &k_full[g], j);
             }
-            // V goes over Q once the first MMA has read it
-            if (mbar_wait_bounded(s_full, 0, a.wait_ns)) {
+            // V goes over Q once the first MMA has read it (the last group's
+            // commit covers every S MMA)
+            if (mbar_wait_bounded(&s_full[NG - 1], 0, a.wait_ns)) {
                 mbar_arrive_expect_tx(v_full, C::KV_BYTES + a.tx_extra);
                 for (int j = 0; j < C::U; ++j) load_unit(&tm_v, vs, v_full, j);
                 v_issued = true;
@@ -221,9 +222,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                         umma_bf16(s_tmem + 64 * g, ad, bd, umma_idesc_bf16(M, 64, false),
                                   kk > 0);
                     }
-                }
-                if (ok) {
-                    umma_commit(s_full);
+                    umma_commit(&s_full[g]);          // the softmax starts on this group
                     s_issued = true;
                 }
             }
@@ -249,7 +248,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             }
             // nothing this thread issued may still run when TMEM is freed
             if (o_issued) (void)mbar_wait_bounded(o_full, 0, a.wait_ns);
-            else if (s_issued) (void)mbar_wait_bounded(s_full, 0, a.wait_ns);
+            else if (s_issued)   // the last group committed covers every earlier MMA
+                for (int g = NG - 1; g >= 0; --g)
+                    if (mbar_wait_bounded(&s_full[g], 0, a.wait_ns)) break;
         }
     } else {
         // -------------------------------- softmax and epilogue: warps 0-3 --
@@ -269,13 +270,14 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             return ok != 0;
         };
         float m = -INFINITY, l = 0.f;
-        bool ok = __all_sync(FULL_MASK, mbar_wait_bounded(s_full, 0, a.wait_ns));
-        if (ok) {
-            tc_fence_after_sync();
-            // pass 1: the row's maximum over the chunk's prefix tokens (log2
-            // units), 64 columns per TMEM round trip
+        // pass 1: the row's maximum over the chunk's prefix tokens (log2 units),
+        // one 64-token group at a time as its S MMAs complete
+        bool ok = true;
 #pragma unroll 1
-            for (int c = 0; c < CH / 64; ++c) {
+        for (int c = 0; c < CH / 64 && ok; ++c) {
+            ok = __all_sync(FULL_MASK, mbar_wait_bounded(&s_full[c], 0, a.wait_ns));
+            if (ok) {
+                tc_fence_after_sync();
                 float v0[32], v1[32];
                 tmem_ld32(s_tmem + lane_off + 64 * c, v0);
                 tmem_ld32(s_tmem + lane_off + 64 * c + 32, v1);
@@ -286,6 +288,8 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                     if (64 * c + 32 + j < valid) m = fmaxf(m, v1[j] * a.scale_log2);
                 }
             }
+        }
+        if (ok) {
             // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum of p;
             // 64 tokens = one slab row of 128 bytes per round trip
             const uint32_t prow = smem_addr(ks) + (uint32_t)r * 128;
@@ -300,9 +304,10 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int t = 64 * c + 2 * j;
+                    // half the exponentials on the SFU, half on the FMA pipe
                     const float p0 = t < valid ? exp2_approx(v[2 * j] * a.scale_log2 - m) : 0.f;
                     const float p1 =
-                        t + 1 < valid ? exp2_approx(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
+                        t + 1 < valid ? exp2_poly(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
                     l += p0 + p1;
                     w[j] = pack_bf16x2(p0, p1);
                 }
