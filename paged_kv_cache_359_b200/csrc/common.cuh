@@ -57,22 +57,6 @@ __device__ __forceinline__ float exp2_approx(float x) {
     return y;
 }
 
-// 2^x for x <= 0 on the FMA and integer pipes, to share the work of
-// exp2_approx's SFU: x = j + f with j the nearest integer (adding 1.5 * 2^23
-// rounds x to an integer in the low mantissa bits) and f in [-0.5, 0.5]; 2^f
-// from a cubic fitted to 2^f on that interval by least squares in the
-// relative error (maximum relative error 7.8e-5, ample for weights rounded to
-// bf16); 2^j goes into the exponent field.  x is clamped at -126 (results
-// below 2^-126 come out tiny instead of zero).
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -126.f);
-    const float t = __fadd_rn(x, 12582912.f);
-    const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
-    const float p = fmaf(fmaf(fmaf(0.05508868f, f, 0.24260405f), f, 0.69327623f), f, 0.99992895f);
-    const int j = __float_as_int(t) - 0x4B400000;
-    return __int_as_float(__float_as_int(p) + (j << 23));
-}
-
 __device__ __forceinline__ unsigned long long global_ns() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

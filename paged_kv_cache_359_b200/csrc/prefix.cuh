@@ -304,10 +304,9 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int t = 64 * c + 2 * j;
-                    // half the exponentials on the SFU, half on the FMA pipe
                     const float p0 = t < valid ? exp2_approx(v[2 * j] * a.scale_log2 - m) : 0.f;
                     const float p1 =
-                        t + 1 < valid ? exp2_poly(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
+                        t + 1 < valid ? exp2_approx(v[2 * j + 1] * a.scale_log2 - m) : 0.f;
                     l += p0 + p1;
                     w[j] = pack_bf16x2(p0, p1);
                 }

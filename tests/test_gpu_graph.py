@@ -103,3 +103,91 @@ def test_graph_replay_matches_eager_and_the_oracle():
     assert_close(got[-1], ref)
     del graph
     device_clean()
+
+
+def _forked_batch(d=128, prefix=768, members=24, seed=91):
+    """`members` sequences forked from one `prefix`-token prompt, own tails of
+    up to 300 tokens, 32 q / 8 kv heads, block 16, bf16."""
+    rng = np.random.default_rng(seed)
+    hq, hk, bs = 32, 8, 16
+    tails = rng.integers(1, 300, size=members)
+    lens = (prefix + tails).astype(np.int32)
+    nb = prefix // bs + int(sum(-(-int(t) // bs) for t in tails)) + 8
+    order = rng.permutation(nb).astype(np.int32)
+    cap = -(-int(lens.max()) // bs) + 1
+    tables = np.full((members, cap), -1, dtype=np.int32)
+    tables[:, : prefix // bs] = order[: prefix // bs]
+    nxt = prefix // bs
+    for i, t in enumerate(tails):
+        k = -(-int(t) // bs)
+        tables[i, prefix // bs: prefix // bs + k] = order[nxt: nxt + k]
+        nxt += k
+    problem = pa_inputs.PagedProblem(
+        name="fork", num_heads=hq, num_kv_heads=hk, head_dim=d, block_size=bs, num_blocks=nb,
+        dtype="bf16", context_lens=lens, free_order=order, block_tables=tables, seed=seed,
+        scale=1.0 / np.sqrt(d))
+    return problem, pa_inputs.materialize(problem, "cuda")
+
+
+def _replay_equals_eager(call, out_shape_like):
+    """call(out) launches the library's kernels on the current stream."""
+    eager = torch.empty_like(out_shape_like)
+    call(eager)
+    torch.cuda.synchronize()
+    out = torch.full_like(out_shape_like, float("nan"))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call(out)                               # warm-up outside the capture
+        torch.cuda.synchronize()
+        out.fill_(float("nan"))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            call(out)
+    torch.cuda.current_stream().wait_stream(side)
+    graph.replay()
+    graph.replay()
+    torch.cuda.synchronize()
+    del graph
+    return eager, out
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_shared_prefix_decode_replays_from_a_graph(d):
+    # the shared pass (tcgen05) and the own-token pass, which streams before
+    # it waits for the shared pass, captured with programmatic dependent launch
+    problem, data = _forked_batch(d=d)
+    s, prefix = problem.num_seqs, 768
+    starts = torch.tensor([0, s], dtype=torch.int32, device="cuda")
+    plen = torch.tensor([prefix], dtype=torch.int32, device="cuda")
+    ws = torch.empty(pa.pa_decode_shared_prefix_workspace_bytes(s, 32, d, prefix),
+                     dtype=torch.uint8, device="cuda")
+
+    def call(out):
+        pa.pa_decode_shared_prefix(out, data["q"], data["k_cache"], data["v_cache"],
+                                   data["block_tables"], data["context_lens"], problem.scale,
+                                   starts, plen, s, prefix, ws)
+
+    eager, got = _replay_equals_eager(call, data["q"])
+    assert same_bits(got, eager)
+    ref = oracle.paged_decode(data["q"].cpu(), data["k_cache"].cpu(), data["v_cache"].cpu(),
+                              problem.block_tables, problem.context_lens, problem.scale)
+    assert_close(got, ref)
+    device_clean()
+
+
+def test_split_decode_replays_from_a_graph():
+    # partitions merged in chunks (arrival counts zeroed by the first kernel)
+    problem, data = _forked_batch(prefix=4096, members=3, seed=92)
+    longest = int(problem.context_lens.max())
+    ws = torch.empty(pa.pa_decode_split_workspace_bytes(3, 32, 128, longest, 128),
+                     dtype=torch.uint8, device="cuda")
+
+    def call(out):
+        pa.pa_decode_split(out, data["q"], data["k_cache"], data["v_cache"],
+                           data["block_tables"], data["context_lens"], problem.scale,
+                           longest, 128, ws)
+
+    eager, got = _replay_equals_eager(call, data["q"])
+    assert same_bits(got, eager)
+    device_clean()
