@@ -26,8 +26,9 @@ Reported line (rank 0):
   e2e        the same metric through the public API with host buffers: the
              live allocator on the host, pinned H2D copies of each step's
              q / new K,V / slots / lengths / copy-on-write pairs, the table
-             changes applied on the device (pa_update_block_tables), and a
-             D2H read of the step's output, all inside the timed region;
+             changes applied on the device (by pa_decode_step itself, or
+             pa_update_block_tables when unfused), and a D2H read of the
+             step's output, all inside the timed region;
              uploads and downloads run on their own streams through a ring
              of three buffer sets, overlapping the neighbouring steps'
              kernels as a serving loop would.
@@ -45,6 +46,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import gc
 import hashlib
 import json
 import math
@@ -273,7 +275,8 @@ def decode_kv_bytes(lens: np.ndarray, problem) -> int:
 
 def decode_alg_bytes(lens: np.ndarray, problem, fused: bool = False) -> int:
     """K/V rows read + q read + out written + block-table entries + lengths;
-    fused: + the new key/value rows read and written into the cache + slots."""
+    fused: + the new key/value rows read and written into the cache + slots
+    (pa_decode_step writes the new block's table entry instead of reading it)."""
     s = len(lens)
     qo = 2 * s * problem.num_heads * problem.head_dim * problem.elem_bytes
     tab = 4 * int(sum(-(-int(x) // problem.block_size) for x in lens)) + 4 * s
@@ -398,11 +401,14 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
     Events cannot time launches inside a graph, so the decode launches of
     the same steps go into a second graph, replayed after the timed region:
     its time / K is the mean decode launch (back to back; the decode calls
-    are idempotent on the final state: the fused append rewrites the same
-    rows, the other decodes only read)."""
+    are idempotent on the final state: the fused step rewrites the same
+    rows and table entries, the other decodes only read)."""
     pa, p, dev = loop.pa, loop.p, loop.device
     total = steps + warmup
     slots, cows, tabs, lens = [], [], [], []
+    # the fused step keeps one device copy of the tables and updates it itself
+    # (pa_decode_step); the other paths take each step's tables as given
+    tab_live = torch.from_numpy(loop.tables).to(dev) if loop.fused else None
     for _ in range(total):
         sl, cw = loop.alloc.append_slots(loop.tables, loop.lens)
         slots.append(sl.copy())
@@ -425,8 +431,8 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
 
     def decode_only(i):
         if loop.fused:
-            pa.pa_decode_append(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
-                                slots_d[i], tabs_d[i], lens_d[i], p.scale)
+            pa.pa_decode_step(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
+                              slots_d[i], tab_live, lens_d[i], p.scale)
         else:
             loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
 
@@ -438,8 +444,8 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
         if timed_index is not None:
             dec_ev[timed_index][0].record()            # the current (or capturing) stream
         if loop.fused:
-            pa.pa_decode_append(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
-                                slots_d[i], tabs_d[i], lens_d[i], p.scale)
+            pa.pa_decode_step(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
+                              slots_d[i], tab_live, lens_d[i], p.scale)
         else:
             loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
         if timed_index is not None:
@@ -583,10 +589,10 @@ def _config_entry(loop, res, steps, peak, label, kernel):
 
 def run_other_configs(dev, local, peak, steps=10, warmup=3):
     """The other decode workloads, measured briefly after the headline run:
-    MHA batch 64 (fused append + decode), the long-context split at the
-    config's 512-token partitions, and the prefix-sharing batch (block 16,
-    head_dim 128) with plain decode (fused append + decode) and with the
-    cascade.  Each builds its own pool, runs ``warmup`` eager steps and
+    MHA batch 64 (pa_decode_step: mapping update, append and decode in one
+    launch), the long-context split at the config's 512-token partitions, and
+    the prefix-sharing batch (block 16, head_dim 128) with plain decode
+    (pa_decode_step) and with the cascade.  Each builds its own pool, runs ``warmup`` eager steps and
     ``steps`` device-timed steps replayed as one CUDA graph, and is freed."""
     out = []
     extra = 2 * (steps + warmup) + 4
@@ -602,11 +608,11 @@ def run_other_configs(dev, local, peak, steps=10, warmup=3):
         return out[-1]
 
     run(lambda: DecodeLoop(make_problem("mha", extra, 0), dev, "decode", 512),
-        "mha_decode_b64", "pa_decode_append", fused=True)
+        "mha_decode_b64", "pa_decode_step", fused=True)
     run(lambda: DecodeLoop(make_problem("long", extra, 0), dev, "split", 512),
         "long_context_split_p512", "pa_decode_split")
     plain = run(lambda: build_prefix_loop(dev, extra, "decode", 512, 16, 128),
-                "prefix_sharing_b64_bs16_d128", "pa_decode_append", fused=True, unique=True)
+                "prefix_sharing_b64_bs16_d128", "pa_decode_step", fused=True, unique=True)
     casc = run(lambda: build_prefix_loop(dev, extra, "cascade", 512, 16, 128),
                "prefix_sharing_b64_bs16_d128", "pa_decode_shared_prefix", unique=True)
     casc["speedup_vs_pa_decode"] = round(plain["ms_per_step"] / casc["ms_per_step"], 3)
@@ -627,6 +633,10 @@ def _view(buf, seg, dtype, shape):
     return buf[off:off + nbytes].view(dtype).view(shape)
 
 
+# untimed steps the end-to-end loop runs after its timed window (see run_e2e)
+E2E_TRAIL = 4
+
+
 def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3):
     """Through the public API from host buffers, as a serving loop runs it.
 
@@ -634,18 +644,30 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
     the lengths, slots and copy-on-write pairs straight into a pinned
     metadata buffer; the step's inputs go host->device from pinned memory
     (one copy for q and the new K/V rows, one for the metadata); on the
-    device pa_copy_blocks runs the copy-on-write pairs, pa_update_block_tables
+    device pa_copy_blocks runs the copy-on-write pairs, then pa_decode_step
     applies the step's table changes to the device-resident block tables
-    (one entry per sequence at most, derived from the lengths and slots
-    already uploaded, so the table itself never crosses the link), and the
-    decode runs; the step's output comes back device->host and the host
-    reads it.  A ring of ``ring`` buffer sets lets the host run up to
-    ring - 1 steps ahead of the last completed download: step i's uploads
-    go out as soon as step i - ring has been read back, on their own stream,
-    and downloads have a third stream, so copies overlap the neighbouring
-    steps' kernels.  The timed region spans every copy of every timed step."""
+    (one entry per sequence at most, taken from the slots already uploaded,
+    so the table itself never crosses the link), writes the new rows and
+    decodes, in one launch (unfused: pa_update_block_tables,
+    pa_reshape_and_cache, then the decode); the step's output comes back
+    device->host and the host reads it.  A ring of ``ring`` buffer sets lets
+    the host run up to ring - 1 steps ahead of the last completed download:
+    step i's uploads go out as soon as step i - ring has been read back, on
+    their own stream, and downloads have a third stream, so copies overlap
+    the neighbouring steps' kernels.  The timed region spans every copy of
+    every timed step.  Python's cyclic garbage collector is paused over it
+    (after a collection), as a serving loop does once it has started, so
+    that a collection pass does not stall the host in the middle.
+
+    The timed steps are a window of a loop that goes on: two warm-up steps
+    lead into it without a pause and E2E_TRAIL untimed steps follow it (t1
+    is on the compute stream before their kernels; only their uploads
+    overlap the window, which can only lengthen it).  On B200 boxes the last
+    steps issued before a loop stops ran up to twice as slow while their
+    host-to-device copies were in flight (measured per step with events;
+    SM clocks unchanged), an end effect a serving loop does not have."""
     pa, p, dev = loop.pa, loop.p, loop.device
-    total = steps + warmup
+    total = steps + warmup + E2E_TRAIL
     s, cap = loop.tables.shape
     dt = loop.q0.dtype
     esz = loop.q0.element_size()
@@ -726,11 +748,12 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
         comp.wait_event(b.h2d)
         if n:
             pa.pa_copy_blocks(loop.k_cache, loop.v_cache, b.cows[:n], stream=comp)
-        pa.pa_update_block_tables(tables_d, b.lens, b.slots, bs, p.num_blocks, stream=comp)
         if loop.fused:
-            pa.pa_decode_append(b.out, b.q, b.k, b.v, loop.k_cache, loop.v_cache, b.slots,
-                                tables_d, b.lens, p.scale, stream=comp)
+            # the mapping update, the cache write and the decode: one launch
+            pa.pa_decode_step(b.out, b.q, b.k, b.v, loop.k_cache, loop.v_cache, b.slots,
+                              tables_d, b.lens, p.scale, stream=comp)
         else:
+            pa.pa_update_block_tables(tables_d, b.lens, b.slots, bs, p.num_blocks, stream=comp)
             pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
             saved_out, loop.out = loop.out, b.out
             with torch.cuda.stream(comp):
@@ -754,23 +777,40 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
                 read_back(b)
 
     next_step = [0]
-    for i in range(warmup):
+    # the last two warm-up steps run after the synchronisation, right before
+    # the timed region, so that it opens on a busy GPU (running clocks,
+    # active copy links) as in a loop that has been serving for a while; t0
+    # follows their kernels on the compute stream and the timed uploads wait
+    # for it
+    pre = min(2, warmup)
+    for i in range(warmup - pre):
         step(i, False)
         next_step[0] = i + 1
     drain()
     torch.cuda.synchronize()
     barrier(world)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(comp)
-    up.wait_event(t0)
-    down.wait_event(t0)
-    for j in range(steps):
-        step(warmup + j, True)
-        next_step[0] = warmup + j + 1
-    for b in bufs:
-        if b.used:
-            comp.wait_event(b.d2h)
-    t1.record(comp)
+    gc.collect()
+    gc.disable()
+    try:
+        for i in range(warmup - pre, warmup):
+            step(i, False)
+            next_step[0] = i + 1
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(comp)
+        up.wait_event(t0)
+        down.wait_event(t0)
+        for j in range(steps):
+            step(warmup + j, True)
+            next_step[0] = warmup + j + 1
+        for b in bufs:
+            if b.used:
+                comp.wait_event(b.d2h)
+        t1.record(comp)
+        for i in range(warmup + steps, total):
+            step(i, False)
+            next_step[0] = i + 1
+    finally:
+        gc.enable()
     drain()
     torch.cuda.synchronize()
     barrier(world)
@@ -879,7 +919,7 @@ def pool_headroom_tokens(args) -> int:
     """Tokens each sequence may grow by during a run: the device-timed loop
     and the end-to-end loop each append one per step.  Both bench arms size
     their pool from this, so they run the same configuration."""
-    return 2 * (args.steps + args.warmup) + 4
+    return 2 * (args.steps + args.warmup) + E2E_TRAIL + 4
 
 
 def workload_config(p, args):
@@ -894,7 +934,8 @@ def workload_config(p, args):
             # internal fragmentation: unused rows of each sequence's last block
             "block_waste_frac": round(1.0 - float(lens.astype(np.int64).sum()) / float(sum(
                 -(-int(x) // p.block_size) * p.block_size for x in lens)), 5),
-            "kernel": args.kernel + ("+append (fused)" if args.fused else ""),
+            "kernel": args.kernel + (" step: table update + append + decode, one launch"
+                                     if args.fused else ""),
             "partition": args.partition,
             "pdl": not getattr(args, "no_pdl", False),
             "timed_steps": "eager launches" if getattr(args, "eager", False)
@@ -918,7 +959,8 @@ def main():
                          "4096 measures faster on B200)")
     ap.add_argument("--unfused", action="store_true",
                     help="decode kernel: pa_reshape_and_cache then pa_decode (two launches) "
-                         "instead of pa_decode_append (the cache write fused into the decode)")
+                         "instead of pa_decode_step (the table update and the cache write "
+                         "fused into the decode)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-configs", action="store_true",
@@ -1014,7 +1056,7 @@ def main():
             "tokens_per_s": round(tokens_all / secs, 1),
             "frac_of_nominal_8tbps": round(value / NOMINAL_HBM_GBS, 4),
             "roofline": {"bound": "hbm",
-                         "kernel": {"decode": "pa_decode_append" if args.fused else "pa_decode",
+                         "kernel": {"decode": "pa_decode_step" if args.fused else "pa_decode",
                                     "split": "pa_decode_split (partition + reduce)",
                                     "cascade": "pa_decode_shared_prefix (shared pass, then own "
                                                "tokens merged)"}[args.kernel],

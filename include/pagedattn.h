@@ -173,6 +173,34 @@ pa_status pa_decode_append(void* out_d, const void* q_d, const void* key_d,
                            int num_blocks, float scale, pa_dtype dtype, pa_stream_t stream);
 
 /*
+ * pa_decode_step -- one whole decode step in one launch: the mapping update
+ * of pa_update_block_tables, then pa_decode_append ([csdn-QA] 四 flow:
+ * allocate a free page, update the mapping, run the attention kernel).
+ * The block of each sequence's new token is taken from its slot
+ * (slot_mapping[s] / block_size) rather than from the table, and written
+ * into the table:
+ *   block_tables[s, (context_lens[s] - 1) / block_size] = slot_mapping[s] / block_size
+ * so the caller's device tables need not hold the new block (a fresh block
+ * or a copy-on-write replacement) before the call, and hold it after.
+ *   block_tables_d   int32 [num_seqs, max_blocks_per_seq]; the entries
+ *                    before a sequence's last block are read, the last one
+ *                    is written (for sequences with slot_mapping[s] >= 0)
+ * Other arguments and preconditions as pa_decode_append, except that a new
+ * slot need only lie on the new token's row (slot % block_size equal to
+ * (context_lens[s] - 1) % block_size) of a block no other sequence reads;
+ * validate mode checks that and the entries read.  Sequences without a new
+ * token (-1), slots outside the pool (PA_DEVERR_SLOT) and empty sequences
+ * keep their entry.  Results equal pa_update_block_tables followed by
+ * pa_decode_append on the same stream, bit for bit.
+ */
+pa_status pa_decode_step(void* out_d, const void* q_d, const void* key_d,
+                         const void* value_d, void* k_cache_d, void* v_cache_d,
+                         const int64_t* slot_mapping_d, int32_t* block_tables_d,
+                         int max_blocks_per_seq, const int32_t* context_lens_d, int num_seqs,
+                         int num_heads, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, float scale, pa_dtype dtype, pa_stream_t stream);
+
+/*
  * pa_update_block_tables -- the "update the mapping" step of a decode step
  * ([csdn-QA] 四 flow: allocate a free page, update the mapping, run the
  * attention kernel; [course] 2.4.2: a new block only when the last one is

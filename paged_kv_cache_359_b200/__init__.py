@@ -11,6 +11,7 @@ Functions carry the C names:
 * ``pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping)``
 * ``pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale)``
 * ``pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, ...)``
+* ``pa_decode_step(out, q, key, value, k_cache, v_cache, slot_mapping, block_tables, ...)``
 * ``pa_decode_split(out, q, ..., max_context_len, partition_size, workspace)``
 * ``pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size)``
 * ``pa_decode_shared_prefix(out, q, ..., group_starts, prefix_lens, ...)``
@@ -33,7 +34,8 @@ from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SP
                       PA_OPT_WAIT_LIMIT_US, PagedAttnError, check, lib)
 
 __all__ = [
-    "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_split", "pa_decode_split_workspace_bytes",
+    "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_step", "pa_decode_split",
+    "pa_decode_split_workspace_bytes",
     "pa_decode_split_noalloc", "pa_decode_shared_prefix", "pa_update_block_tables",
     "pa_decode_shared_prefix_workspace_bytes", "pa_copy_blocks", "pa_swap_blocks",
     "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
@@ -143,6 +145,22 @@ def pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, block_t
                                  _ptr(v_cache), _ptr(slot_mapping), _ptr(block_tables),
                                  block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb,
                                  float(scale), _dtype(q), _stream(stream)))
+    return out
+
+
+def pa_decode_step(out, q, key, value, k_cache, v_cache, slot_mapping, block_tables,
+                   context_lens, scale, stream=None):
+    """One decode step in one launch: each sequence's last table entry is set
+    from its new slot (``block_tables`` is updated in place), the new rows
+    are stored, then the batch is decoded -- pa_update_block_tables followed
+    by pa_decode_append."""
+    s, hq, d, nb, bs, hk = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens)
+    _dev(key, value, slot_mapping)
+    _new_rows(key, value, s, hk, d, k_cache.dtype, slot_mapping)
+    check(lib().pa_decode_step(_ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_cache),
+                               _ptr(v_cache), _ptr(slot_mapping), _ptr(block_tables),
+                               block_tables.shape[1], _ptr(context_lens), s, hq, hk, d, bs, nb,
+                               float(scale), _dtype(q), _stream(stream)))
     return out
 
 

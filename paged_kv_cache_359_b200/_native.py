@@ -45,6 +45,8 @@ SIGNATURES = {
                            _c_int, _c_int, _c_float, _c_int, _vp]),
     "pa_decode_append": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int,
                                   _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "pa_decode_step": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int,
+                                _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "pa_decode_split_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "pa_decode_split": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_float, _c_int, _c_int, _c_int, _vp,

@@ -120,12 +120,10 @@ bool copy_to_host(std::vector<T>& dst, const T* src, size_t n, cudaStream_t stre
     return cudaStreamSynchronize(stream) == cudaSuccess;
 }
 
-pa_status validate_decode(const int32_t* tables, int max_blocks, const int32_t* lens, int num_seqs,
-                          int block_size, int num_blocks, cudaStream_t stream) {
-    std::vector<int32_t> t, l;
-    if (!copy_to_host(l, lens, (size_t)num_seqs, stream) ||
-        !copy_to_host(t, tables, (size_t)num_seqs * max_blocks, stream))
-        return fail(PA_ERR_CUDA, "validation copy failed");
+// Every sequence's length fits its table row and the entries it reads are
+// blocks of the pool (host copies of the tables and lengths).
+pa_status check_tables(const std::vector<int32_t>& t, const std::vector<int32_t>& l,
+                       int max_blocks, int num_seqs, int block_size, int num_blocks) {
     for (int s = 0; s < num_seqs; ++s) {
         if (l[s] < 0 || (int64_t)l[s] > (int64_t)max_blocks * block_size)
             return fail(PA_ERR_BAD_BLOCK_ID, "context_lens[%d] = %d outside [0, %lld]", s, l[s],
@@ -139,6 +137,15 @@ pa_status validate_decode(const int32_t* tables, int max_blocks, const int32_t* 
         }
     }
     return PA_OK;
+}
+
+pa_status validate_decode(const int32_t* tables, int max_blocks, const int32_t* lens, int num_seqs,
+                          int block_size, int num_blocks, cudaStream_t stream) {
+    std::vector<int32_t> t, l;
+    if (!copy_to_host(l, lens, (size_t)num_seqs, stream) ||
+        !copy_to_host(t, tables, (size_t)num_seqs * max_blocks, stream))
+        return fail(PA_ERR_CUDA, "validation copy failed");
+    return check_tables(t, l, max_blocks, num_seqs, block_size, num_blocks);
 }
 
 pa_status check_decode_args(void* out, const void* q, const void* kc, const void* vc,
@@ -403,7 +410,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
                       const int32_t* context_lens, int num_seqs, int num_heads, int num_kv_heads,
                       int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
                       const void* new_k, const void* new_v, const int64_t* new_slots,
-                      pa_stream_t stream) {
+                      int32_t* table_out, pa_stream_t stream) {
     if (pa_status s = check_decode_args(out, q, k_cache, v_cache, block_tables,
                                         max_blocks_per_seq, context_lens, num_seqs, num_heads,
                                         num_kv_heads, head_dim, block_size, num_blocks, dtype,
@@ -414,7 +421,29 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     if (append && (!new_k || !new_v || !aligned16(new_k) || !aligned16(new_v)))
         return fail(PA_ERR_INVALID_ARG, "key and value rows must be 16-byte aligned device pointers");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (validate_enabled()) {
+    if (validate_enabled() && table_out) {
+        // the tables as the step leaves them: each new slot's block at its
+        // sequence's last position, the slot on the new token's row
+        std::vector<int32_t> t, l;
+        std::vector<int64_t> sl;
+        if (!copy_to_host(l, context_lens, (size_t)num_seqs, st) ||
+            !copy_to_host(t, block_tables, (size_t)num_seqs * max_blocks_per_seq, st) ||
+            !copy_to_host(sl, new_slots, (size_t)num_seqs, st))
+            return fail(PA_ERR_CUDA, "validation copy failed");
+        const int64_t num_slots = (int64_t)num_blocks * block_size;
+        for (int s = 0; s < num_seqs; ++s) {
+            if (sl[s] < 0) continue;
+            const int pos = l[s] - 1;
+            if (sl[s] >= num_slots || pos < 0 || (int64_t)pos >= (int64_t)max_blocks_per_seq * block_size ||
+                sl[s] % block_size != pos % block_size)
+                return fail(PA_ERR_BAD_BLOCK_ID,
+                            "new slot of sequence %d is %lld, not row %d of a pool block", s,
+                            (long long)sl[s], pos < 0 ? -1 : pos % block_size);
+            t[(size_t)s * max_blocks_per_seq + pos / block_size] = (int32_t)(sl[s] / block_size);
+        }
+        if (pa_status s = check_tables(t, l, max_blocks_per_seq, num_seqs, block_size, num_blocks))
+            return s;
+    } else if (validate_enabled()) {
         if (pa_status s = validate_decode(block_tables, max_blocks_per_seq, context_lens,
                                           num_seqs, block_size, num_blocks, st))
             return s;
@@ -455,6 +484,7 @@ pa_status decode_impl(void* out, const void* q, const void* k_cache, const void*
     l.args.new_k = new_k;
     l.args.new_v = new_v;
     l.args.new_slots = new_slots;
+    l.args.table_out = table_out;
     l.args.k_cache = const_cast<void*>(k_cache);
     l.args.v_cache = const_cast<void*>(v_cache);
     l.k_cache = k_cache;
@@ -486,7 +516,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     pa_stream_t stream) {
     return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                        num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                       scale, dtype, nullptr, nullptr, nullptr, stream);
+                       scale, dtype, nullptr, nullptr, nullptr, nullptr, stream);
 }
 
 pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value,
@@ -498,7 +528,19 @@ pa_status pa_decode_append(void* out, const void* q, const void* key, const void
     if (num_seqs > 0 && !slot_mapping) return fail(PA_ERR_INVALID_ARG, "null slot_mapping");
     return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                        num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                       scale, dtype, key, value, slot_mapping, stream);
+                       scale, dtype, key, value, slot_mapping, nullptr, stream);
+}
+
+pa_status pa_decode_step(void* out, const void* q, const void* key, const void* value,
+                         void* k_cache, void* v_cache, const int64_t* slot_mapping,
+                         int32_t* block_tables, int max_blocks_per_seq,
+                         const int32_t* context_lens, int num_seqs, int num_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                         float scale, pa_dtype dtype, pa_stream_t stream) {
+    if (num_seqs > 0 && !slot_mapping) return fail(PA_ERR_INVALID_ARG, "null slot_mapping");
+    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                       num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       scale, dtype, key, value, slot_mapping, block_tables, stream);
 }
 
 size_t pa_decode_split_workspace_bytes(int num_seqs, int num_heads, int head_dim,

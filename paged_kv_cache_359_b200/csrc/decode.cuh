@@ -99,6 +99,11 @@ struct DecodeArgs {
     const int64_t* new_slots;
     void* k_cache;                // written only by the fused append
     void* v_cache;
+    // pa_decode_step: the step's mapping update fused in.  Sequence s's last
+    // block is the new slot's block (new_slots[s] / block_size), not its
+    // table entry, and the CTA of kv head 0 writes it into the table
+    // (block_tables, writable); null otherwise
+    int32_t* table_out;
     // shared-prefix decode: sequences [group_starts[g], group_starts[g+1])
     // share their first group_prefix[g] tokens.  The shared pass leaves one
     // (max, sum, unnormalised output) per (sequence, head, prefix chunk) at
@@ -627,7 +632,27 @@ struct Ctx {
     uint64_t* bars;            // this warp's mbarriers
     int warp, lane;
     int ring;                  // units this warp has consumed so far
+    int sub_blk, sub_id;       // pa_decode_step: block sub_blk of the item is sub_id (-1: none)
 };
+
+// pa_decode_step: the block of sequence seq's new token comes from its slot.
+// Every CTA of the sequence reads it from there (none reads that table
+// entry, so the write cannot race with a read); the CTA of kv head 0 (rank 0
+// of a cluster) stores it in the table for the steps that follow.  Skipped
+// sequences, slots outside the pool and empty sequences keep their entry.
+template <class U>
+__device__ __forceinline__ void map_new_block(Ctx<U>& cx, const DecodeArgs& a, int seq, int L,
+                                              bool writer) {
+    cx.sub_blk = -1;
+    cx.sub_id = 0;
+    if (!a.table_out || L <= 0) return;
+    const int64_t slot = a.new_slots[seq];
+    if (slot < 0 || slot >= (int64_t)a.num_blocks * U::BS) return;
+    cx.sub_blk = (L - 1) / U::BS;
+    cx.sub_id = (int)(slot / U::BS);
+    if (writer && threadIdx.x == 0)
+        a.table_out[(size_t)seq * a.max_blocks + cx.sub_blk] = cx.sub_id;
+}
 
 // Run one item: stream this CTA's share of (seq, kvh)'s units in
 // [u_begin, u_end), interleaved over `ctas` CTAs (this one is `crank`) and
@@ -663,9 +688,11 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
         int id = 0, id1 = -1;
         if (k < nk) {
             const int t0 = (first + ustride * k) * R;
-            id = checked(__ldg(table + t0 / U::BS));
+            const int b0 = t0 / U::BS;
+            id = checked(b0 == cx.sub_blk ? cx.sub_id : __ldg(table + b0));
             if constexpr (HALVES == 2) {
-                if (t0 + U::BOX_ROWS < L) id1 = checked(__ldg(table + t0 / U::BS + 1));
+                if (t0 + U::BOX_ROWS < L)
+                    id1 = checked(b0 + 1 == cx.sub_blk ? cx.sub_id : __ldg(table + b0 + 1));
             }
         }
         win = id;
@@ -835,6 +862,8 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
     cx.warp = warp;
     cx.lane = lane;
     cx.ring = 0;
+    cx.sub_blk = -1;
+    cx.sub_id = 0;
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < DEPTH; ++s) mbar_init(&cx.bars[s], 1);
@@ -876,6 +905,7 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
             const int ctas = gridDim.x;
             if (a.new_slots) {
                 if (blockIdx.x == 0) append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
+                map_new_block(cx, a, seq, L, kvh == 0 && blockIdx.x == 0);
                 if (ctas > 1)
                     cg::this_cluster().sync();         // every rank loads after the write
                 else
@@ -998,6 +1028,7 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
             }
             if (a.new_slots) {
                 append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
+                map_new_block(cx, a, seq, L, kvh == 0);
                 __syncthreads();                       // the loads below see the new row
             }
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
