@@ -368,18 +368,35 @@ class DecodeLoop:
         return self.ws
 
     def launches_per_step(self, n_cow: int) -> int:
-        if self.fused:
-            return (1 if n_cow else 0) + 1
         per = {"split": 2, "cascade": 2}.get(self.kernel, 1)
+        if self.fused:
+            return (1 if n_cow else 0) + per
         return (1 if n_cow else 0) + 1 + per
+
+    def prefix_workspace(self):
+        need = self.pa.pa_decode_shared_prefix_workspace_bytes(
+            self.p.num_seqs, self.p.num_heads, self.p.head_dim, self.groups["max_prefix"])
+        if self.ws is None or self.ws.numel() < need:
+            self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        return self.ws
+
+    def step(self, out, q, key, value, slots_d, tables_d, lens_d, stream=None):
+        """The fused step: table update, cache write and decode, in the
+        decode's launch(es); ``tables_d`` is updated in place."""
+        if self.kernel == "cascade":
+            g = self.groups
+            self.pa.pa_decode_shared_prefix_step(
+                out, q, key, value, self.k_cache, self.v_cache, slots_d, tables_d, lens_d,
+                self.p.scale, g["starts"], g["prefix"], g["max_size"], g["max_prefix"],
+                self.prefix_workspace(), stream=stream)
+        else:
+            self.pa.pa_decode_step(out, q, key, value, self.k_cache, self.v_cache, slots_d,
+                                   tables_d, lens_d, self.p.scale, stream=stream)
 
     def decode(self, q, tables_d, lens_d, max_len):
         if self.kernel == "cascade":
             g = self.groups
-            need = self.pa.pa_decode_shared_prefix_workspace_bytes(
-                self.p.num_seqs, self.p.num_heads, self.p.head_dim, g["max_prefix"])
-            if self.ws is None or self.ws.numel() < need:
-                self.ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self.prefix_workspace()
             self.pa.pa_decode_shared_prefix(self.out, q, self.k_cache, self.v_cache, tables_d,
                                             lens_d, self.p.scale, g["starts"], g["prefix"],
                                             g["max_size"], g["max_prefix"], self.ws)
@@ -431,8 +448,7 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
 
     def decode_only(i):
         if loop.fused:
-            pa.pa_decode_step(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
-                              slots_d[i], tab_live, lens_d[i], p.scale)
+            loop.step(loop.out, qs[i], keys[i], vals[i], slots_d[i], tab_live, lens_d[i])
         else:
             loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
 
@@ -444,8 +460,7 @@ def run_device_timed(loop: DecodeLoop, steps: int, warmup: int, world: int, dev_
         if timed_index is not None:
             dec_ev[timed_index][0].record()            # the current (or capturing) stream
         if loop.fused:
-            pa.pa_decode_step(loop.out, qs[i], keys[i], vals[i], loop.k_cache, loop.v_cache,
-                              slots_d[i], tab_live, lens_d[i], p.scale)
+            loop.step(loop.out, qs[i], keys[i], vals[i], slots_d[i], tab_live, lens_d[i])
         else:
             loop.decode(qs[i], tabs_d[i], lens_d[i], max_lens[i])
         if timed_index is not None:
@@ -592,8 +607,9 @@ def run_other_configs(dev, local, peak, steps=10, warmup=3):
     MHA batch 64 (pa_decode_step: mapping update, append and decode in one
     launch), the long-context split at the config's 512-token partitions, and
     the prefix-sharing batch (block 16, head_dim 128) with plain decode
-    (pa_decode_step) and with the cascade.  Each builds its own pool, runs ``warmup`` eager steps and
-    ``steps`` device-timed steps replayed as one CUDA graph, and is freed."""
+    (pa_decode_step) and with the cascade (pa_decode_shared_prefix_step).
+    Each builds its own pool, runs ``warmup`` eager steps and ``steps``
+    device-timed steps replayed as one CUDA graph, and is freed."""
     out = []
     extra = 2 * (steps + warmup) + 4
 
@@ -614,7 +630,8 @@ def run_other_configs(dev, local, peak, steps=10, warmup=3):
     plain = run(lambda: build_prefix_loop(dev, extra, "decode", 512, 16, 128),
                 "prefix_sharing_b64_bs16_d128", "pa_decode_step", fused=True, unique=True)
     casc = run(lambda: build_prefix_loop(dev, extra, "cascade", 512, 16, 128),
-               "prefix_sharing_b64_bs16_d128", "pa_decode_shared_prefix", unique=True)
+               "prefix_sharing_b64_bs16_d128", "pa_decode_shared_prefix_step", fused=True,
+               unique=True)
     casc["speedup_vs_pa_decode"] = round(plain["ms_per_step"] / casc["ms_per_step"], 3)
     return out
 
@@ -749,9 +766,9 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
         if n:
             pa.pa_copy_blocks(loop.k_cache, loop.v_cache, b.cows[:n], stream=comp)
         if loop.fused:
-            # the mapping update, the cache write and the decode: one launch
-            pa.pa_decode_step(b.out, b.q, b.k, b.v, loop.k_cache, loop.v_cache, b.slots,
-                              tables_d, b.lens, p.scale, stream=comp)
+            # the mapping update, the cache write and the decode, in the
+            # decode's launch(es)
+            loop.step(b.out, b.q, b.k, b.v, b.slots, tables_d, b.lens, stream=comp)
         else:
             pa.pa_update_block_tables(tables_d, b.lens, b.slots, bs, p.num_blocks, stream=comp)
             pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
@@ -934,7 +951,7 @@ def workload_config(p, args):
             # internal fragmentation: unused rows of each sequence's last block
             "block_waste_frac": round(1.0 - float(lens.astype(np.int64).sum()) / float(sum(
                 -(-int(x) // p.block_size) * p.block_size for x in lens)), 5),
-            "kernel": args.kernel + (" step: table update + append + decode, one launch"
+            "kernel": args.kernel + (" step: table update + append fused into the decode"
                                      if args.fused else ""),
             "partition": args.partition,
             "pdl": not getattr(args, "no_pdl", False),
@@ -958,8 +975,9 @@ def main():
                     help="split kernel partition in tokens (the long-context config's 512; "
                          "4096 measures faster on B200)")
     ap.add_argument("--unfused", action="store_true",
-                    help="decode kernel: pa_reshape_and_cache then pa_decode (two launches) "
-                         "instead of pa_decode_step (the table update and the cache write "
+                    help="decode and cascade kernels: pa_reshape_and_cache then pa_decode "
+                         "or pa_decode_shared_prefix, instead of pa_decode_step or "
+                         "pa_decode_shared_prefix_step (the table update and the cache write "
                          "fused into the decode)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -985,10 +1003,11 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.kernel is None:
         args.kernel = "split" if args.workload == "long" else "decode"
-    if args.unfused and args.kernel != "decode":
-        ap.error("--unfused applies to the decode kernel (split and cascade write separately)")
-    # the decode kernel's step is the fused append + decode unless asked otherwise
-    args.fused = args.kernel == "decode" and not args.unfused
+    if args.unfused and args.kernel == "split":
+        ap.error("--unfused applies to the decode and cascade kernels (split writes separately)")
+    # the decode and cascade kernels' step has the table update and the cache
+    # write fused in unless asked otherwise
+    args.fused = args.kernel in ("decode", "cascade") and not args.unfused
     if args.compact and args.workload not in ("gqa", "mha"):
         ap.error("--compact runs on the gqa and mha workloads")
     if (args.block_size or args.head_dim) and args.workload not in ("gqa", "prefix"):
@@ -1058,8 +1077,10 @@ def main():
             "roofline": {"bound": "hbm",
                          "kernel": {"decode": "pa_decode_step" if args.fused else "pa_decode",
                                     "split": "pa_decode_split (partition + reduce)",
-                                    "cascade": "pa_decode_shared_prefix (shared pass, then own "
-                                               "tokens merged)"}[args.kernel],
+                                    "cascade": ("pa_decode_shared_prefix_step" if args.fused else
+                                                "pa_decode_shared_prefix") +
+                                               " (shared pass, then own tokens merged)"
+                                    }[args.kernel],
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "peak_source": peak_src,
                          "frac_of_nominal_8tbps": round(achieved / NOMINAL_HBM_GBS, 4),

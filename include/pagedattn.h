@@ -328,6 +328,33 @@ pa_status pa_decode_shared_prefix(void* out_d, const void* q_d, const void* k_ca
                                   void* workspace_d, size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_decode_shared_prefix_step -- pa_decode_shared_prefix as a whole decode
+ * step, the shared-prefix counterpart of pa_decode_step: the own-token pass
+ * also stores each sequence's new token (key_d/value_d rows at
+ * slot_mapping_d, as pa_decode_append) and the mapping update
+ * (block_tables[s, (context_lens[s] - 1) / block_size] = slot / block_size,
+ * as pa_decode_step), so a step is the two launches of the cascade and no
+ * cache-write or table-update launch.  Arguments as pa_decode_shared_prefix
+ * plus those of pa_decode_step; context_lens count the new token, which must
+ * lie past its group's prefix (in a block of its own, as the allocator's
+ * copy-on-write guarantees).  block_tables_d is written (the last entry of
+ * each sequence with a new token).  Validate mode checks the preconditions
+ * of both.  Results equal pa_update_block_tables, pa_reshape_and_cache and
+ * pa_decode_shared_prefix on the same stream, bit for bit.
+ */
+pa_status pa_decode_shared_prefix_step(void* out_d, const void* q_d, const void* key_d,
+                                       const void* value_d, void* k_cache_d, void* v_cache_d,
+                                       const int64_t* slot_mapping_d, int32_t* block_tables_d,
+                                       int max_blocks_per_seq, const int32_t* context_lens_d,
+                                       int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_dim, int block_size, int num_blocks, float scale,
+                                       pa_dtype dtype, const int32_t* group_starts_d,
+                                       const int32_t* prefix_lens_d, int num_groups,
+                                       int max_group_size, int max_prefix_len,
+                                       void* workspace_d, size_t workspace_bytes,
+                                       pa_stream_t stream);
+
+/*
  * pa_copy_blocks -- copy-on-write of shared blocks: for each pair
  * (src, dst) the whole key block and value block dst <- src ([course] 2.4.3:
  * a write to a block whose reference count exceeds one first copies it).

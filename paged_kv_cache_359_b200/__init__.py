@@ -15,6 +15,7 @@ Functions carry the C names:
 * ``pa_decode_split(out, q, ..., max_context_len, partition_size, workspace)``
 * ``pa_decode_split_workspace_bytes(num_seqs, num_heads, head_dim, max_context_len, partition_size)``
 * ``pa_decode_shared_prefix(out, q, ..., group_starts, prefix_lens, ...)``
+* ``pa_decode_shared_prefix_step(out, q, key, value, ..., slot_mapping, block_tables, ...)``
 * ``pa_copy_blocks(k_cache, v_cache, block_mapping)``
 * ``pa_swap_blocks(dst_k, dst_v, src_k, src_v, block_mapping)``
 * ``pa_device_error(clear=True)``, ``pa_set_option(name, value)``
@@ -36,7 +37,8 @@ from ._native import (DEVERR_BITS, PA_DTYPE_BF16, PA_DTYPE_F32, PA_OPT_DECODE_SP
 __all__ = [
     "pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_step", "pa_decode_split",
     "pa_decode_split_workspace_bytes",
-    "pa_decode_split_noalloc", "pa_decode_shared_prefix", "pa_update_block_tables",
+    "pa_decode_split_noalloc", "pa_decode_shared_prefix", "pa_decode_shared_prefix_step",
+    "pa_update_block_tables",
     "pa_decode_shared_prefix_workspace_bytes", "pa_copy_blocks", "pa_swap_blocks",
     "pa_device_error", "pa_set_option", "pa_get_option", "BlockAllocator",
     "PagedAttnError", "OutOfBlocks", "DEVERR_BITS",
@@ -229,6 +231,33 @@ def pa_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, context_lens
         _ptr(group_starts), _ptr(prefix_lens), prefix_lens.shape[0], int(max_group_size),
         int(max_prefix_len), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
+    return out
+
+
+def pa_decode_shared_prefix_step(out, q, key, value, k_cache, v_cache, slot_mapping,
+                                 block_tables, context_lens, scale, group_starts, prefix_lens,
+                                 max_group_size, max_prefix_len, workspace=None, stream=None):
+    """pa_decode_shared_prefix as a whole step: the own-token pass also stores
+    each sequence's new row (key/value [S, Hk, D] at slot_mapping int64 [S],
+    -1 = none) and sets its last table entry from the slot (``block_tables``
+    is updated in place)."""
+    s, hq, d, nb, bs, hk = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens)
+    _dev(group_starts, prefix_lens, key, value, slot_mapping)
+    _need(group_starts.dtype == torch.int32 and prefix_lens.dtype == torch.int32 and
+          group_starts.dim() == 1 and prefix_lens.dim() == 1 and
+          group_starts.shape[0] == prefix_lens.shape[0] + 1,
+          "group_starts must be int32 [groups + 1] and prefix_lens int32 [groups]")
+    _new_rows(key, value, s, hk, d, k_cache.dtype, slot_mapping)
+    need = pa_decode_shared_prefix_workspace_bytes(s, hq, d, max_prefix_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _dev(workspace)
+    check(lib().pa_decode_shared_prefix_step(
+        _ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+        _ptr(slot_mapping), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), s, hq,
+        hk, d, bs, nb, float(scale), _dtype(q), _ptr(group_starts), _ptr(prefix_lens),
+        prefix_lens.shape[0], int(max_group_size), int(max_prefix_len), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
 
 

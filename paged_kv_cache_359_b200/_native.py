@@ -58,6 +58,10 @@ SIGNATURES = {
     "pa_decode_shared_prefix": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _vp, _c_int, _c_int,
                                          _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp,
                                          _vp, _c_int, _c_int, _c_int, _vp, _c_size, _vp]),
+    "pa_decode_shared_prefix_step": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int,
+                                              _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                              _c_int, _c_float, _c_int, _vp, _vp, _c_int, _c_int,
+                                              _c_int, _vp, _c_size, _vp]),
     "pa_update_block_tables": (_c_int, [_vp, _c_int, _vp, _vp, _c_int, _c_int, _c_int, _vp]),
     "pa_copy_blocks": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _vp]),

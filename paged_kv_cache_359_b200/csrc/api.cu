@@ -643,14 +643,23 @@ size_t pa_decode_shared_prefix_workspace_bytes(int num_seqs, int num_heads, int 
     return 2 * align256(rows * sizeof(float)) + rows * head_dim * sizeof(float);
 }
 
-pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
-                                  const void* v_cache, const int32_t* block_tables,
-                                  int max_blocks_per_seq, const int32_t* context_lens,
-                                  int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                                  int block_size, int num_blocks, float scale, pa_dtype dtype,
-                                  const int32_t* group_starts, const int32_t* prefix_lens,
-                                  int num_groups, int max_group_size, int max_prefix_len,
-                                  void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// pa_decode_shared_prefix, optionally as a whole step (new_slots and
+// table_out both set): the own-token pass then also appends one new token
+// per sequence (new_k/new_v at new_slots), taking each sequence's last block
+// from its new slot and storing it in the table.
+pa_status shared_prefix_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* context_lens, int num_seqs, int num_heads,
+                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                             float scale, pa_dtype dtype, const int32_t* group_starts,
+                             const int32_t* prefix_lens, int num_groups, int max_group_size,
+                             int max_prefix_len, void* workspace, size_t workspace_bytes,
+                             const void* new_k, const void* new_v, const int64_t* new_slots,
+                             int32_t* table_out, pa_stream_t stream) {
     if (pa_status s = check_decode_args(out, q, k_cache, v_cache, block_tables,
                                         max_blocks_per_seq, context_lens, num_seqs, num_heads,
                                         num_kv_heads, head_dim, block_size, num_blocks, dtype,
@@ -666,21 +675,41 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
         return fail(PA_ERR_UNSUPPORTED, "too many groups x row blocks for one launch");
     if (num_seqs == 0) return PA_OK;
     if (!group_starts || !prefix_lens) return fail(PA_ERR_INVALID_ARG, "null group arrays");
+    const bool append = new_slots != nullptr;
+    if (append && (!new_k || !new_v || !aligned16(new_k) || !aligned16(new_v)))
+        return fail(PA_ERR_INVALID_ARG, "key and value rows must be 16-byte aligned device pointers");
     const size_t need = pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, head_dim,
                                                                 max_prefix_len);
     if (!workspace || workspace_bytes < need || !aligned16(workspace))
         return fail(PA_ERR_INVALID_ARG, "workspace needs %zu bytes, 16-byte aligned", need);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (validate_enabled()) {
-        if (pa_status s = validate_decode(block_tables, max_blocks_per_seq, context_lens,
-                                          num_seqs, block_size, num_blocks, st))
-            return s;
         std::vector<int32_t> gs, pl, t, l;
+        std::vector<int64_t> sl;
         if (!copy_to_host(gs, group_starts, (size_t)num_groups + 1, st) ||
             !copy_to_host(pl, prefix_lens, (size_t)num_groups, st) ||
             !copy_to_host(l, context_lens, (size_t)num_seqs, st) ||
-            !copy_to_host(t, block_tables, (size_t)num_seqs * max_blocks_per_seq, st))
+            !copy_to_host(t, block_tables, (size_t)num_seqs * max_blocks_per_seq, st) ||
+            (append && !copy_to_host(sl, new_slots, (size_t)num_seqs, st)))
             return fail(PA_ERR_CUDA, "validation copy failed");
+        const int64_t num_slots = (int64_t)num_blocks * block_size;
+        for (int s = 0; append && s < num_seqs; ++s) {
+            // the new token: the sequence's last position, past its prefix
+            // (checked below, per group), in the slot's row
+            if (sl[s] < 0) continue;
+            const int pos = l[s] - 1;
+            if (sl[s] >= num_slots || pos < 0 ||
+                (int64_t)pos >= (int64_t)max_blocks_per_seq * block_size)
+                return fail(PA_ERR_BAD_BLOCK_ID, "new slot of sequence %d is %lld", s,
+                            (long long)sl[s]);
+            if (sl[s] % block_size != pos % block_size)
+                return fail(PA_ERR_BAD_BLOCK_ID,
+                            "new slot of sequence %d is %lld, not row %d of a pool block", s,
+                            (long long)sl[s], pos % block_size);
+            t[(size_t)s * max_blocks_per_seq + pos / block_size] = (int32_t)(sl[s] / block_size);
+        }
+        if (pa_status s = check_tables(t, l, max_blocks_per_seq, num_seqs, block_size, num_blocks))
+            return s;
         if (gs[0] != 0 || gs[num_groups] != num_seqs)
             return fail(PA_ERR_BAD_BLOCK_ID, "groups must cover sequences 0..num_seqs-1");
         for (int g = 0; g < num_groups; ++g) {
@@ -693,6 +722,9 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
             for (int s = gs[g]; s < gs[g + 1]; ++s) {
                 if (l[s] < pl[g])
                     return fail(PA_ERR_BAD_BLOCK_ID, "sequence %d is shorter than its prefix", s);
+                if (append && sl[s] >= 0 && l[s] - 1 < pl[g])
+                    return fail(PA_ERR_BAD_BLOCK_ID,
+                                "the new token of sequence %d falls in its group's prefix", s);
                 for (int j = 0; j < nb; ++j)
                     if (t[(size_t)s * max_blocks_per_seq + j] !=
                         t[(size_t)gs[g] * max_blocks_per_seq + j])
@@ -730,6 +762,12 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
     l.args.prefix_slot0 = 0;
     l.args.slot_stride = chunks ? chunks : 1;
     l.args.sched = SCHED_LPT;
+    l.args.new_k = new_k;
+    l.args.new_v = new_v;
+    l.args.new_slots = new_slots;
+    l.args.table_out = table_out;
+    l.args.k_cache = const_cast<void*>(k_cache);
+    l.args.v_cache = const_cast<void*>(v_cache);
     l.k_cache = k_cache;
     l.v_cache = v_cache;
     l.num_seqs = num_seqs;
@@ -744,6 +782,43 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
     l.row_blocks = (max_rows + PREFIX_ROWS_PER_CTA - 1) / PREFIX_ROWS_PER_CTA;
     l.stream = st;
     return dispatch_decode(l, dtype, head_dim);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  int max_blocks_per_seq, const int32_t* context_lens,
+                                  int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int num_blocks, float scale, pa_dtype dtype,
+                                  const int32_t* group_starts, const int32_t* prefix_lens,
+                                  int num_groups, int max_group_size, int max_prefix_len,
+                                  void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+    return shared_prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                              context_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                              block_size, num_blocks, scale, dtype, group_starts, prefix_lens,
+                              num_groups, max_group_size, max_prefix_len, workspace,
+                              workspace_bytes, nullptr, nullptr, nullptr, nullptr, stream);
+}
+
+pa_status pa_decode_shared_prefix_step(void* out, const void* q, const void* key,
+                                       const void* value, void* k_cache, void* v_cache,
+                                       const int64_t* slot_mapping, int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens,
+                                       int num_seqs, int num_heads, int num_kv_heads,
+                                       int head_dim, int block_size, int num_blocks, float scale,
+                                       pa_dtype dtype, const int32_t* group_starts,
+                                       const int32_t* prefix_lens, int num_groups,
+                                       int max_group_size, int max_prefix_len, void* workspace,
+                                       size_t workspace_bytes, pa_stream_t stream) {
+    if (num_seqs > 0 && !slot_mapping) return fail(PA_ERR_INVALID_ARG, "null slot_mapping");
+    return shared_prefix_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                              context_lens, num_seqs, num_heads, num_kv_heads, head_dim,
+                              block_size, num_blocks, scale, dtype, group_starts, prefix_lens,
+                              num_groups, max_group_size, max_prefix_len, workspace,
+                              workspace_bytes, key, value, slot_mapping, block_tables, stream);
 }
 
 pa_status pa_update_block_tables(int32_t* block_tables, int max_blocks_per_seq,

@@ -111,6 +111,11 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
             cfg.blockDim = dim3(Lo::NW * 32);
             cfg.dynamicSmemBytes = Lo::SMEM_BYTES;
             cfg.gridDim = dim3((unsigned)((long long)l.num_seqs * l.num_kv_heads));
+            // The own-token pass reads the cache before its dependency wait,
+            // which is safe only behind the shared pass (whose CTAs wait for
+            // the stream's previous kernel before they release it).  Without
+            // a shared pass it launches in plain stream order.
+            if (l.max_chunks <= 0) cfg.numAttrs = 0;
             e = cudaLaunchKernelEx(&cfg, ok, mk, mv, l.args);
             if (e != cudaSuccess)
                 return fail(PA_ERR_CUDA, "own-token launch: %s", cudaGetErrorString(e));
