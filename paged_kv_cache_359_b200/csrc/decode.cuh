@@ -951,10 +951,15 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
             return;
         } else {
             // Which sequence sits at rank r = blockIdx.x / Hk of the list sorted
-            // by (tokens this pass reads descending, index ascending)?  Warp 0
-            // selects it (rank_select); up to 256 sequences it holds the
-            // lengths in registers and the other warps go straight to the
-            // barrier, above that the CTA stages them in shared memory.
+            // by (tokens this pass reads descending, index ascending)?  Up to
+            // 64 sequences every thread stages some of the lengths in shared
+            // memory and counts, for one sequence, the entries that sort
+            // before it (a direct rank: 64 compares, measured faster than the
+            // search below on the shared-prefix decode's own-token pass and
+            // slower for 256 sequences); otherwise warp 0 selects it
+            // (rank_select), holding the lengths in registers up to 256
+            // sequences while the other warps go straight to the barrier, and
+            // above that the CTA stages them in shared memory.
             const int S = a.num_seqs, Hk = a.num_kv_heads;
             const int r = blockIdx.x / Hk;
             // sequence, tokens this pass reads, context length, shared prefix
@@ -971,12 +976,40 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                 return len - cmin(shared_prefix_of(a, i), len);
             };
             constexpr int REG_PER_LANE = 8;
+            constexpr int DIRECT_MAX = 64;
+            static_assert(3 * DIRECT_MAX <= MAX_SORT, "the direct rank's arrays fit the sort area");
             const bool in_regs = S <= 32 * REG_PER_LANE;
             if (!in_regs && S <= MAX_SORT) {
                 for (int i = threadIdx.x; i < S; i += NT) lens[i] = own_tokens(i);
                 __syncthreads();
             }
-            if (warp == 0) {
+            if (S <= DIRECT_MAX) {
+                int* own = lens;                     // tokens this pass, length, prefix
+                int* cl = lens + DIRECT_MAX;
+                int* pr = lens + 2 * DIRECT_MAX;
+                for (int i = threadIdx.x; i < S; i += NT) {
+                    const int ln = clamped_len(i);
+                    const int p = cmin(shared_prefix_of(a, i), ln);
+                    own[i] = ln - p;
+                    cl[i] = ln;
+                    pr[i] = p;
+                }
+                __syncthreads();
+                for (int i = threadIdx.x; i < S; i += NT) {
+                    const int vi = own[i];
+                    int before = 0;
+                    for (int k = 0; k < S; ++k) {
+                        const int vk = own[k];
+                        before += (vk > vi) | ((vk == vi) & (k < i));
+                    }
+                    if (before == r) {               // ranks are a permutation: one writer
+                        pick[0] = i;
+                        pick[1] = vi;
+                        pick[2] = cl[i];
+                        pick[3] = pr[i];
+                    }
+                }
+            } else if (warp == 0) {
                 int found = r, tokens = -1;                  // natural order beyond MAX_SORT
                 int len_of = 0, pre_of = 0;
                 if (in_regs) {
