@@ -170,11 +170,54 @@ __device__ __forceinline__ int rank_select(Get&& get, int r, int lane, int& valu
     return (int)__reduce_max_sync(FULL_MASK, (unsigned)(found + 1)) - 1;
 }
 
-// Fused append: the CTA of (seq, kvh) writes kv head kvh's part of the new
-// token's key and value rows into the cache, then makes the writes visible
-// to its own TMA loads.  Only this sequence reads the new token's block (a
-// shared block is copied before it is written), so no other CTA can race
-// with the write.  The caller follows with a CTA (or cluster) barrier.
+// Fused append in two phases, so that the loads of both go out before
+// anything waits on them: append_load reads the new token's slot and this
+// thread's share (at most two 16-byte vectors: vectors j and j + NT of the
+// key | value row pair of kv head kvh) of the new rows; append_store writes
+// them at the slot and makes the writes visible to the CTA's own TMA loads.
+// The caller follows with a CTA barrier.  Only this sequence reads the new
+// token's block (a shared block is copied before it is written), so no
+// other CTA can race with the write.
+struct AppendLoad {
+    int64_t slot;
+    uint4 x[2];
+};
+
+template <typename T, int D, int NT>
+__device__ __forceinline__ AppendLoad append_load(const DecodeArgs& a, int seq, int kvh) {
+    constexpr int NV = D * (int)sizeof(T) / 16;        // 16-byte vectors per head row
+    static_assert(2 * NV <= 2 * NT, "two vectors per thread cover the key and value rows");
+    AppendLoad al;
+    al.slot = a.new_slots[seq];
+    const size_t row = ((size_t)seq * a.num_kv_heads + kvh) * NV;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int j = (int)threadIdx.x + h * NT;
+        al.x[h] = make_uint4(0, 0, 0, 0);
+        if (j < 2 * NV)
+            al.x[h] = reinterpret_cast<const uint4*>(j >= NV ? a.new_v : a.new_k)[row + j % NV];
+    }
+    return al;
+}
+
+template <typename T, int D, int BS, int NT>
+__device__ __forceinline__ void append_store(const AppendLoad& al, const DecodeArgs& a, int kvh) {
+    constexpr int NV = D * (int)sizeof(T) / 16;
+    if (al.slot < 0) return;
+    if (al.slot >= (int64_t)a.num_blocks * BS) {
+        if (threadIdx.x == 0) raise_error(a.err, PA_DEVERR_SLOT);
+        return;
+    }
+    const size_t row = ((size_t)al.slot * a.num_kv_heads + kvh) * NV;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int j = (int)threadIdx.x + h * NT;
+        if (j < 2 * NV) reinterpret_cast<uint4*>(j >= NV ? a.v_cache : a.k_cache)[row + j % NV] = al.x[h];
+    }
+    fence_proxy_async_global();
+}
+
+// The same in one call (the cluster path), for any number of threads.
 template <typename T, int D, int BS>
 __device__ __forceinline__ void append_row(const DecodeArgs& a, int seq, int kvh, void* k_cache,
                                            void* v_cache) {
@@ -642,11 +685,10 @@ struct Ctx {
 // sequences, slots outside the pool and empty sequences keep their entry.
 template <class U>
 __device__ __forceinline__ void map_new_block(Ctx<U>& cx, const DecodeArgs& a, int seq, int L,
-                                              bool writer) {
+                                              bool writer, int64_t slot) {
     cx.sub_blk = -1;
     cx.sub_id = 0;
     if (!a.table_out || L <= 0) return;
-    const int64_t slot = a.new_slots[seq];
     if (slot < 0 || slot >= (int64_t)a.num_blocks * U::BS) return;
     cx.sub_blk = (L - 1) / U::BS;
     cx.sub_id = (int)(slot / U::BS);
@@ -659,11 +701,18 @@ __device__ __forceinline__ void map_new_block(Ctx<U>& cx, const DecodeArgs& a, i
 // over the NW warps, then merge the warps into shared memory.  Returns with
 // the CTA-merged (max, sum, unnormalised output) per (g, d) computed by
 // `epilogue`.  Every thread of the CTA must call it (it holds barriers).
-template <class U, class Ly, class Epi>
+struct NoHook {
+    __device__ void operator()() const {}
+};
+
+// `before_first` runs (on every thread) after the first window of block ids
+// has been requested and before it is used: work whose loads should be in
+// flight together with the window's (the fused append) goes there.
+template <class U, class Ly, class Epi, class Hook = NoHook>
 __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
                                          const CUtensorMap* tm_v, const DecodeArgs& a, int seq,
                                          int kvh, int L, int u_begin, int u_end, int ctas,
-                                         int crank, Epi&& epilogue) {
+                                         int crank, Epi&& epilogue, Hook&& before_first = Hook()) {
     using T = typename U::T;
     constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
     const int warp = cx.warp, lane = cx.lane;
@@ -682,21 +731,40 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
         }
         return id;
     };
-    int win = 0, win1 = -1;
-    auto load_window = [&](int k0) {
+    // a window: the block ids of this warp's next 32 units, one per lane;
+    // requested first, then resolved (the new token's block comes from its
+    // slot under pa_decode_step, and only then is an id checked)
+    int win = 0, win1 = -1, wb0 = -1;
+    bool two = false;                    // the unit's second 8-token block holds tokens
+    auto request_window = [&](int k0) {
         const int k = k0 + lane;
-        int id = 0, id1 = -1;
+        win = 0;
+        win1 = -1;
+        wb0 = -1;
+        two = false;
         if (k < nk) {
             const int t0 = (first + ustride * k) * R;
-            const int b0 = t0 / U::BS;
-            id = checked(b0 == cx.sub_blk ? cx.sub_id : __ldg(table + b0));
+            wb0 = t0 / U::BS;
+            win = __ldg(table + wb0);
             if constexpr (HALVES == 2) {
-                if (t0 + U::BOX_ROWS < L)
-                    id1 = checked(b0 + 1 == cx.sub_blk ? cx.sub_id : __ldg(table + b0 + 1));
+                two = t0 + U::BOX_ROWS < L;
+                if (two) win1 = __ldg(table + wb0 + 1);
             }
         }
-        win = id;
-        win1 = id1;
+    };
+    auto resolve_window = [&]() {
+        if (wb0 < 0) {
+            win = 0;
+            return;
+        }
+        win = checked(wb0 == cx.sub_blk ? cx.sub_id : win);
+        if constexpr (HALVES == 2) {
+            if (two) win1 = checked(wb0 + 1 == cx.sub_blk ? cx.sub_id : win1);
+        }
+    };
+    auto load_window = [&](int k0) {
+        request_window(k0);
+        resolve_window();
     };
     auto slot = [&](int k) { return (cx.ring + k) % DEPTH; };
     auto issue = [&](int k, int id, int id1) {     // lane 0 only
@@ -722,7 +790,9 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
         }
     };
 
-    load_window(0);
+    request_window(0);
+    before_first();
+    resolve_window();
     const int pro = cmin(DEPTH, nk);
     for (int k = 0; k < pro; ++k) {
         const int id = __shfl_sync(FULL_MASK, win, k);
@@ -905,7 +975,7 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
             const int ctas = gridDim.x;
             if (a.new_slots) {
                 if (blockIdx.x == 0) append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
-                map_new_block(cx, a, seq, L, kvh == 0 && blockIdx.x == 0);
+                map_new_block(cx, a, seq, L, kvh == 0 && blockIdx.x == 0, a.new_slots[seq]);
                 if (ctas > 1)
                     cg::this_cluster().sync();         // every rank loads after the write
                 else
@@ -1059,11 +1129,11 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                 L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
                 tok0 = cmin(shared_prefix_of(a, seq), L);
             }
-            if (a.new_slots) {
-                append_row<T, D, U::BS>(a, seq, kvh, a.k_cache, a.v_cache);
-                map_new_block(cx, a, seq, L, kvh == 0);
-                __syncthreads();                       // the loads below see the new row
-            }
+            // the new row's loads go out here and are waited on (written,
+            // fenced, barrier) only after the first window of block ids has
+            // been requested, so both round trips overlap
+            AppendLoad al = {};
+            if (a.new_slots) al = append_load<T, D, NT>(a, seq, kvh);
             const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
             const int nchunks = a.group_starts ? (tok0 + a.chunk_tokens - 1) / a.chunk_tokens : 0;
             // x: this CTA's own part, [G] max, [G] sum, [G][D] unnormalised output,
@@ -1080,6 +1150,13 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                                 return;
                             }
                             store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                        },
+                        [&] {
+                            if (a.new_slots) {
+                                append_store<T, D, U::BS, NT>(al, a, kvh);
+                                map_new_block(cx, a, seq, L, kvh == 0, al.slot);
+                                __syncthreads();       // the loads below see the new row
+                            }
                         });
             pdl_wait();                                // the shared pass is complete
             if (nchunks) {
