@@ -114,6 +114,36 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// ------------------------------------------------ cluster launch control --
+// Work stealing on sm_100: a running CTA asks the hardware to cancel the
+// launch of a CTA of the same grid that has not started yet; the 16-byte
+// answer lands in shared memory and completes 16 bytes of `bar`'s phase.  If
+// the cancellation succeeded, the answer names the cancelled CTA, whose work
+// the asking CTA then does.  One thread issues it.
+__device__ __forceinline__ void clc_try_cancel(void* response16, uint64_t* bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 "
+        "[%0], [%1];" ::"r"(smem_addr(response16)),
+        "r"(smem_addr(bar))
+        : "memory");
+}
+
+// The cancelled CTA's blockIdx.x, or -1 when the cancellation failed (no CTA
+// of the grid was left to start).
+__device__ __forceinline__ int clc_cancelled_x(const void* response16) {
+    uint32_t ok, x;
+    asm volatile(
+        "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+        : "=r"(ok), "=r"(x)
+        : "r"(smem_addr(response16))
+        : "memory");
+    return ok ? (int)x : -1;
+}
+
 // 4-D tiled TMA load (no multicast) into this CTA's shared memory; the
 // mbarrier counts the bytes as they land.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,

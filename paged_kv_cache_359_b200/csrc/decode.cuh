@@ -661,7 +661,10 @@ struct Layout {
     static constexpr int PBUF_OFFSET = MAIN_REGION;
     static constexpr int ORDER_OFFSET = PBUF_OFFSET + NW * U::PBUF_FLOATS * 4;
     static constexpr int BAR_OFFSET = ORDER_OFFSET + (MAX_SORT + 4) * 4;
-    static constexpr int SMEM_BYTES = BAR_OFFSET + NW * DEPTH * 8 + 1024;   // + alignment slack
+    // work stealing (Mode::Decode): the 16-byte cancellation response, its
+    // mbarrier and the next item's index
+    static constexpr int STEAL_OFFSET = (BAR_OFFSET + NW * DEPTH * 8 + 15) / 16 * 16;
+    static constexpr int SMEM_BYTES = STEAL_OFFSET + 32 + 1024;   // + alignment slack
     static_assert(MAIN_REGION % 1024 == 0 && STAGE_BYTES % 1024 == 0, "1 KiB aligned stages");
     static_assert(BAR_OFFSET % 8 == 0, "mbarrier alignment");
 };
@@ -708,11 +711,15 @@ struct NoHook {
 // `before_first` runs (on every thread) after the first window of block ids
 // has been requested and before it is used: work whose loads should be in
 // flight together with the window's (the fused append) goes there.
-template <class U, class Ly, class Epi, class Hook = NoHook>
+// `streamed` runs on every thread once its warp has consumed its units,
+// before the warps merge (the work-stealing request goes out there, so
+// that its answer arrives during the merge).
+template <class U, class Ly, class Epi, class Hook = NoHook, class Hook2 = NoHook>
 __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
                                          const CUtensorMap* tm_v, const DecodeArgs& a, int seq,
                                          int kvh, int L, int u_begin, int u_end, int ctas,
-                                         int crank, Epi&& epilogue, Hook&& before_first = Hook()) {
+                                         int crank, Epi&& epilogue, Hook&& before_first = Hook(),
+                                         Hook2&& streamed = Hook2()) {
     using T = typename U::T;
     constexpr int NW = Ly::NW, DEPTH = Ly::DEPTH, R = U::R, D = U::D, G = U::G;
     const int warp = cx.warp, lane = cx.lane;
@@ -842,6 +849,7 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
     } else {
         cx.ring += nk;
     }
+    streamed();                          // this thread's warp has consumed its units
 
     // ---- merge the warps (the merge area overlays the stage ring) ----
     __syncthreads();
@@ -1020,18 +1028,16 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
             }
             return;
         } else {
-            // Which sequence sits at rank r = blockIdx.x / Hk of the list sorted
-            // by (tokens this pass reads descending, index ascending)?  Up to
-            // 64 sequences every thread stages some of the lengths in shared
-            // memory and counts, for one sequence, the entries that sort
-            // before it (a direct rank: 64 compares, measured faster than the
-            // search below on the shared-prefix decode's own-token pass and
-            // slower for 256 sequences); otherwise warp 0 selects it
-            // (rank_select), holding the lengths in registers up to 256
-            // sequences while the other warps go straight to the barrier, and
-            // above that the CTA stages them in shared memory.
+            // Which sequence sits at rank r = item / Hk of the list sorted by
+            // (tokens this pass reads descending, index ascending)?  The CTA
+            // stages the lengths in shared memory once.  Up to 64 sequences
+            // every thread then counts, for one sequence, the entries that
+            // sort before it (a direct rank: 64 compares, measured faster
+            // than the search on the shared-prefix decode's own-token pass
+            // and slower for 256 sequences); otherwise warp 0 selects it
+            // (rank_select) from the staged values while the other warps go
+            // straight to the barrier.
             const int S = a.num_seqs, Hk = a.num_kv_heads;
-            const int r = blockIdx.x / Hk;
             // sequence, tokens this pass reads, context length, shared prefix
             int* pick = reinterpret_cast<int*>(smem + Ly::ORDER_OFFSET);
             int* lens = pick + 4;                                           // S <= MAX_SORT
@@ -1048,185 +1054,219 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
             constexpr int REG_PER_LANE = 8;
             constexpr int DIRECT_MAX = 64;
             static_assert(3 * DIRECT_MAX <= MAX_SORT, "the direct rank's arrays fit the sort area");
-            const bool in_regs = S <= 32 * REG_PER_LANE;
-            if (!in_regs && S <= MAX_SORT) {
-                for (int i = threadIdx.x; i < S; i += NT) lens[i] = own_tokens(i);
-                __syncthreads();
+            constexpr int STAGED = 32 * REG_PER_LANE;
+            static_assert(3 * STAGED <= MAX_SORT, "the staged lengths fit the sort area");
+            const bool in_regs = S <= STAGED;
+            int* own = lens;                          // up to 256: tokens this pass, length, prefix
+            int* cl = lens + STAGED;
+            int* pr = lens + 2 * STAGED;
+            // Work stealing (pa_decode's grid): when a CTA has streamed its
+            // item it asks the hardware to cancel the launch of the next CTA
+            // of the grid that has not started (the next item in longest-
+            // first order) and runs that item itself, until none is left.
+            // The lengths are read once per CTA, and the CTA's launch, set-up
+            // and length loads are not repeated per item.
+            constexpr bool STEAL = MODE == Mode::Decode;
+            unsigned char* steal_answer = smem + Ly::STEAL_OFFSET;          // 16 bytes
+            uint64_t* steal_bar = reinterpret_cast<uint64_t*>(steal_answer + 16);
+            int* steal_next = reinterpret_cast<int*>(steal_answer + 24);
+            uint32_t steal_phase = 0;
+            if (STEAL && threadIdx.x == 0) {
+                mbar_init(steal_bar, 1);
+                fence_mbar_init();
             }
-            if (S <= DIRECT_MAX) {
-                int* own = lens;                     // tokens this pass, length, prefix
-                int* cl = lens + DIRECT_MAX;
-                int* pr = lens + 2 * DIRECT_MAX;
+            // the lengths, once per CTA, staged in shared memory by every thread
+            if (in_regs) {
                 for (int i = threadIdx.x; i < S; i += NT) {
-                    const int ln = clamped_len(i);
-                    const int p = cmin(shared_prefix_of(a, i), ln);
-                    own[i] = ln - p;
-                    cl[i] = ln;
+                    const int len = clamped_len(i);
+                    const int p = cmin(shared_prefix_of(a, i), len);
+                    own[i] = len - p;
+                    cl[i] = len;
                     pr[i] = p;
                 }
-                __syncthreads();
-                for (int i = threadIdx.x; i < S; i += NT) {
-                    const int vi = own[i];
-                    int before = 0;
-                    for (int k = 0; k < S; ++k) {
-                        const int vk = own[k];
-                        before += (vk > vi) | ((vk == vi) & (k < i));
-                    }
-                    if (before == r) {               // ranks are a permutation: one writer
-                        pick[0] = i;
-                        pick[1] = vi;
-                        pick[2] = cl[i];
-                        pick[3] = pr[i];
-                    }
-                }
-            } else if (warp == 0) {
-                int found = r, tokens = -1;                  // natural order beyond MAX_SORT
-                int len_of = 0, pre_of = 0;
-                if (in_regs) {
-                    int v[REG_PER_LANE], ln[REG_PER_LANE], pr[REG_PER_LANE];
-#pragma unroll
-                    for (int j = 0; j < REG_PER_LANE; ++j) {
-                        const int i = lane + 32 * j;
-                        ln[j] = i < S ? clamped_len(i) : 0;
-                        pr[j] = i < S ? cmin(shared_prefix_of(a, i), ln[j]) : 0;
-                        v[j] = i < S ? ln[j] - pr[j] : -1;
-                    }
-                    found = rank_select<REG_PER_LANE>([&](int j) { return v[j]; }, r, lane,
-                                                      tokens);
-                    // the lane holding the picked entry hands over its length and
-                    // prefix, which saves two dependent loads after the pick
-#pragma unroll
-                    for (int j = 0; j < REG_PER_LANE; ++j)
-                        if (j == (found >> 5)) {
-                            len_of = ln[j];
-                            pre_of = pr[j];
-                        }
-                    len_of = __shfl_sync(FULL_MASK, len_of, found & 31);
-                    pre_of = __shfl_sync(FULL_MASK, pre_of, found & 31);
-                } else if (S <= MAX_SORT) {
-                    found = rank_select<MAX_SORT / 32>(
-                        [&](int j) {
-                            const int i = lane + 32 * j;
-                            return i < S ? lens[i] : -1;
-                        },
-                        r, lane, tokens);
-                }
-                if (lane == 0) {
-                    pick[0] = found;
-                    pick[1] = tokens;
-                    pick[2] = len_of;
-                    pick[3] = pre_of;
-                }
+            } else if (S <= MAX_SORT) {
+                for (int i = threadIdx.x; i < S; i += NT) lens[i] = own_tokens(i);
             }
             __syncthreads();
-            seq = pick[0];
-            kvh = blockIdx.x % Hk;
-            int tok0;                                   // whole 16-token units
-            if (in_regs) {
-                L = pick[2];
-                tok0 = pick[3];
-            } else {
-                L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
-                tok0 = cmin(shared_prefix_of(a, seq), L);
-            }
-            // the new row's loads go out here and are waited on (written,
-            // fenced, barrier) only after the first window of block ids has
-            // been requested, so both round trips overlap
-            AppendLoad al = {};
-            if (a.new_slots) al = append_load<T, D, NT>(a, seq, kvh);
-            const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
-            const int nchunks = a.group_starts ? (tok0 + a.chunk_tokens - 1) / a.chunk_tokens : 0;
-            // x: this CTA's own part, [G] max, [G] sum, [G][D] unnormalised output,
-            // kept after the exchange area when it is merged with prefix chunks
-            float* x = reinterpret_cast<float*>(smem) + NW * G * (D + 2);
-            run_item<U, Ly>(cx, &tm_k, &tm_v, a, seq, kvh, L, tok0 / R, (L + R - 1) / R, 1, 0,
-                        [&](int g, int d, float big, float num, float den, float*) {
-                            if (nchunks) {
-                                if (d == 0) {
-                                    x[g] = big;
-                                    x[G + g] = den;
-                                }
-                                x[2 * G + g * D + d] = num;
-                                return;
-                            }
-                            store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
-                        },
-                        [&] {
-                            if (a.new_slots) {
-                                append_store<T, D, U::BS, NT>(al, a, kvh);
-                                map_new_block(cx, a, seq, L, kvh == 0, al.slot);
-                                __syncthreads();       // the loads below see the new row
-                            }
-                        });
-            pdl_wait();                                // the shared pass is complete
-            if (nchunks) {
-                // merge with the shared pass's chunks of each head.  A thread
-                // writes OPT groups of 4 outputs (g, d .. d+3); it first loads
-                // the chunk maxima of its heads, then the chunks' float4
-                // outputs and sums, CB chunks of every output at a time, all
-                // loads of a batch in flight at once (about 8 float4 per
-                // thread, which keeps them in registers at every head_dim)
-                __syncthreads();                       // x is complete
-                constexpr int Q4 = D / 4;                        // float4 per head row
-                constexpr int OPT = (G * Q4 + NT - 1) / NT;
-                constexpr int CB = OPT >= 8 ? 1 : 8 / OPT;     // chunks per batch
-                float mm[OPT], den[OPT];
-                float4 num[OPT];
-                int gg[OPT], qq[OPT];
-#pragma unroll
-                for (int k = 0; k < OPT; ++k) {
-                    const int idx = threadIdx.x + k * NT;
-                    gg[k] = idx < G * Q4 ? idx / Q4 : 0;
-                    qq[k] = idx % Q4;
-                    mm[k] = x[gg[k]];
-                }
-                auto slot_of = [&](int k, int c) {
-                    return (head0 + gg[k]) * a.slot_stride + a.prefix_slot0 + c;
-                };
-                for (int c0 = 0; c0 < nchunks; c0 += 8) {
-#pragma unroll
-                    for (int k = 0; k < OPT; ++k)
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            if (c0 + c < nchunks) mm[k] = fmaxf(mm[k], a.ws_m[slot_of(k, c0 + c)]);
-                }
-#pragma unroll
-                for (int k = 0; k < OPT; ++k) {
-                    const float own = x[gg[k]];
-                    const float e0 = own == -INFINITY ? 0.f : exp2_approx(own - mm[k]);
-                    const float* xo = x + 2 * G + gg[k] * D + 4 * qq[k];
-                    num[k] = make_float4(e0 * xo[0], e0 * xo[1], e0 * xo[2], e0 * xo[3]);
-                    den[k] = e0 * x[G + gg[k]];
-                }
-                for (int c0 = 0; c0 < nchunks; c0 += CB) {
-#pragma unroll
-                    for (int k = 0; k < OPT; ++k)
-#pragma unroll
-                        for (int c = 0; c < CB; ++c)
-                            if (c0 + c < nchunks) {
-                                const size_t sl = slot_of(k, c0 + c);
-                                const float ec = exp2_approx(a.ws_m[sl] - mm[k]);
-                                const float4 o4 =
-                                    reinterpret_cast<const float4*>(a.ws_o + sl * D)[qq[k]];
-                                num[k].x = fmaf(ec, o4.x, num[k].x);
-                                num[k].y = fmaf(ec, o4.y, num[k].y);
-                                num[k].z = fmaf(ec, o4.z, num[k].z);
-                                num[k].w = fmaf(ec, o4.w, num[k].w);
-                                den[k] = fmaf(ec, a.ws_l[sl], den[k]);
-                            }
-                }
-#pragma unroll
-                for (int k = 0; k < OPT; ++k)
-                    if (threadIdx.x + k * NT < G * Q4) {
-                        T* o = out + (head0 + gg[k]) * D + 4 * qq[k];
-                        const float inv = den[k] > 0.f ? 1.f / den[k] : 0.f;
-                        store_out(o + 0, den[k] > 0.f ? num[k].x * inv : 0.f);
-                        store_out(o + 1, den[k] > 0.f ? num[k].y * inv : 0.f);
-                        store_out(o + 2, den[k] > 0.f ? num[k].z * inv : 0.f);
-                        store_out(o + 3, den[k] > 0.f ? num[k].w * inv : 0.f);
+            for (int item = blockIdx.x;;) {
+                const int r = item / Hk;
+                if (S <= DIRECT_MAX) {
+                    for (int i = threadIdx.x; i < S; i += NT) {
+                        const int vi = own[i];
+                        int before = 0;
+                        for (int k = 0; k < S; ++k) {
+                            const int vk = own[k];
+                            before += (vk > vi) | ((vk == vi) & (k < i));
+                        }
+                        if (before == r) {               // ranks are a permutation: one writer
+                            pick[0] = i;
+                            pick[1] = vi;
+                            pick[2] = cl[i];
+                            pick[3] = pr[i];
+                        }
                     }
+                } else if (warp == 0) {
+                    int found = r, tokens = -1;                  // natural order beyond MAX_SORT
+                    int len_of = 0, pre_of = 0;
+                    if (in_regs) {
+                        int v[REG_PER_LANE];
+    #pragma unroll
+                        for (int j = 0; j < REG_PER_LANE; ++j) {
+                            const int i = lane + 32 * j;
+                            v[j] = i < S ? own[i] : -1;
+                        }
+                        found = rank_select<REG_PER_LANE>([&](int j) { return v[j]; }, r, lane,
+                                                          tokens);
+                        len_of = cl[found];
+                        pre_of = pr[found];
+                    } else if (S <= MAX_SORT) {
+                        found = rank_select<MAX_SORT / 32>(
+                            [&](int j) {
+                                const int i = lane + 32 * j;
+                                return i < S ? lens[i] : -1;
+                            },
+                            r, lane, tokens);
+                    }
+                    if (lane == 0) {
+                        pick[0] = found;
+                        pick[1] = tokens;
+                        pick[2] = len_of;
+                        pick[3] = pre_of;
+                    }
+                }
+                __syncthreads();
+                seq = pick[0];
+                kvh = item % Hk;
+                int tok0;                                   // whole 16-token units
+                if (in_regs) {
+                    L = pick[2];
+                    tok0 = pick[3];
+                } else {
+                    L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
+                    tok0 = cmin(shared_prefix_of(a, seq), L);
+                }
+                // the new row's loads go out here and are waited on (written,
+                // fenced, barrier) only after the first window of block ids has
+                // been requested, so both round trips overlap
+                AppendLoad al = {};
+                if (a.new_slots) al = append_load<T, D, NT>(a, seq, kvh);
+                const size_t head0 = (size_t)seq * a.num_heads + (size_t)kvh * G;
+                const int nchunks = a.group_starts ? (tok0 + a.chunk_tokens - 1) / a.chunk_tokens : 0;
+                // x: this CTA's own part, [G] max, [G] sum, [G][D] unnormalised output,
+                // kept after the exchange area when it is merged with prefix chunks
+                float* x = reinterpret_cast<float*>(smem) + NW * G * (D + 2);
+                run_item<U, Ly>(cx, &tm_k, &tm_v, a, seq, kvh, L, tok0 / R, (L + R - 1) / R, 1, 0,
+                            [&](int g, int d, float big, float num, float den, float*) {
+                                if (nchunks) {
+                                    if (d == 0) {
+                                        x[g] = big;
+                                        x[G + g] = den;
+                                    }
+                                    x[2 * G + g * D + d] = num;
+                                    return;
+                                }
+                                store_out(out + (head0 + g) * D + d, den > 0.f ? num / den : 0.f);
+                            },
+                            [&] {
+                                if (a.new_slots) {
+                                    append_store<T, D, U::BS, NT>(al, a, kvh);
+                                    map_new_block(cx, a, seq, L, kvh == 0, al.slot);
+                                    __syncthreads();       // the loads below see the new row
+                                }
+                            },
+                            [&] {
+                                if (STEAL && threadIdx.x == 0) {
+                                    mbar_arrive_expect_tx(steal_bar, 16);
+                                    clc_try_cancel(steal_answer, steal_bar);
+                                }
+                            });
+                if constexpr (STEAL) {
+                    if (threadIdx.x == 0) {
+                        int next = -1;
+                        if (mbar_wait_bounded(steal_bar, steal_phase, a.wait_ns))
+                            next = clc_cancelled_x(steal_answer);
+                        else
+                            raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
+                        *steal_next = next;
+                    }
+                    steal_phase ^= 1;
+                    // every thread is done with the merge area (the next item's
+                    // tiles land there) and reads the answer
+                    __syncthreads();
+                    item = *steal_next;
+                    if (item < 0 || item >= (int)gridDim.x) return;
+                    continue;
+                }
+                pdl_wait();                                // the shared pass is complete
+                if (nchunks) {
+                    // merge with the shared pass's chunks of each head.  A thread
+                    // writes OPT groups of 4 outputs (g, d .. d+3); it first loads
+                    // the chunk maxima of its heads, then the chunks' float4
+                    // outputs and sums, CB chunks of every output at a time, all
+                    // loads of a batch in flight at once (about 8 float4 per
+                    // thread, which keeps them in registers at every head_dim)
+                    __syncthreads();                       // x is complete
+                    constexpr int Q4 = D / 4;                        // float4 per head row
+                    constexpr int OPT = (G * Q4 + NT - 1) / NT;
+                    constexpr int CB = OPT >= 8 ? 1 : 8 / OPT;     // chunks per batch
+                    float mm[OPT], den[OPT];
+                    float4 num[OPT];
+                    int gg[OPT], qq[OPT];
+    #pragma unroll
+                    for (int k = 0; k < OPT; ++k) {
+                        const int idx = threadIdx.x + k * NT;
+                        gg[k] = idx < G * Q4 ? idx / Q4 : 0;
+                        qq[k] = idx % Q4;
+                        mm[k] = x[gg[k]];
+                    }
+                    auto slot_of = [&](int k, int c) {
+                        return (head0 + gg[k]) * a.slot_stride + a.prefix_slot0 + c;
+                    };
+                    for (int c0 = 0; c0 < nchunks; c0 += 8) {
+    #pragma unroll
+                        for (int k = 0; k < OPT; ++k)
+    #pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                if (c0 + c < nchunks) mm[k] = fmaxf(mm[k], a.ws_m[slot_of(k, c0 + c)]);
+                    }
+    #pragma unroll
+                    for (int k = 0; k < OPT; ++k) {
+                        const float own = x[gg[k]];
+                        const float e0 = own == -INFINITY ? 0.f : exp2_approx(own - mm[k]);
+                        const float* xo = x + 2 * G + gg[k] * D + 4 * qq[k];
+                        num[k] = make_float4(e0 * xo[0], e0 * xo[1], e0 * xo[2], e0 * xo[3]);
+                        den[k] = e0 * x[G + gg[k]];
+                    }
+                    for (int c0 = 0; c0 < nchunks; c0 += CB) {
+    #pragma unroll
+                        for (int k = 0; k < OPT; ++k)
+    #pragma unroll
+                            for (int c = 0; c < CB; ++c)
+                                if (c0 + c < nchunks) {
+                                    const size_t sl = slot_of(k, c0 + c);
+                                    const float ec = exp2_approx(a.ws_m[sl] - mm[k]);
+                                    const float4 o4 =
+                                        reinterpret_cast<const float4*>(a.ws_o + sl * D)[qq[k]];
+                                    num[k].x = fmaf(ec, o4.x, num[k].x);
+                                    num[k].y = fmaf(ec, o4.y, num[k].y);
+                                    num[k].z = fmaf(ec, o4.z, num[k].z);
+                                    num[k].w = fmaf(ec, o4.w, num[k].w);
+                                    den[k] = fmaf(ec, a.ws_l[sl], den[k]);
+                                }
+                    }
+    #pragma unroll
+                    for (int k = 0; k < OPT; ++k)
+                        if (threadIdx.x + k * NT < G * Q4) {
+                            T* o = out + (head0 + gg[k]) * D + 4 * qq[k];
+                            const float inv = den[k] > 0.f ? 1.f / den[k] : 0.f;
+                            store_out(o + 0, den[k] > 0.f ? num[k].x * inv : 0.f);
+                            store_out(o + 1, den[k] > 0.f ? num[k].y * inv : 0.f);
+                            store_out(o + 2, den[k] > 0.f ? num[k].z * inv : 0.f);
+                            store_out(o + 3, den[k] > 0.f ? num[k].w * inv : 0.f);
+                        }
+                }
+                return;
             }
-            return;
         }
     }
 }
