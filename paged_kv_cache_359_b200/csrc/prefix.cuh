@@ -15,24 +15,29 @@
 // 256 (head_dim <= 128) or 128 (head_dim 256).  Roles:
 //  * producer warp: TMA loads of the CTA's 128 query rows (a 3-D box over
 //    q [S][Hq][D]: members x G heads, row = member * G + head) and of the
-//    chunk's K tiles in groups of 64 tokens, all 128-byte swizzled; once the
-//    first MMA has read Q, the chunk's V tiles into Q's space (so the CTA
-//    needs ~128 KB of shared memory and a decode CTA fits beside it); a
-//    unit past the prefix is loaded from outside the pool map, which TMA
-//    fills with zeros;
+//    chunk's K, then V, tiles in 64-token groups through a ring of two
+//    group slots (a slot is refilled once the MMAs that read its previous
+//    group are done), all 128-byte swizzled; a unit past the prefix is
+//    loaded from outside the pool map, which TMA fills with zeros;
 //  * MMA warp (one elected thread): S = Q K^T into TMEM (M = 128 rows,
-//    N = 64 tokens per group as its K tiles land, K = head_dim), commit;
-//    then, once P is in shared memory, O = P V into TMEM (M = 128,
-//    N = head_dim, K = CH tokens, V read MN-major), commit;
+//    N = 64 tokens per group as its K tiles land, K = head_dim), a commit
+//    per group; then, group by group as its P and V tiles land, O += P V
+//    into TMEM (M = 128, N = head_dim, K = 64 tokens, V read MN-major), a
+//    commit per group that frees the group's P and V slots;
 //  * four softmax warps, one TMEM lane (query row) per thread: the exact
 //    maximum of the row's scores over the chunk (masked past the prefix),
-//    then p = 2^(s * scale * log2 e - max), rounded to bf16, into the
-//    swizzled P tile (which reuses the K tile's space) and the fp32 sum of p;
-//    after the second MMA each thread stages its row's output in the (now
-//    free) tiles, up to 128 columns at a time, and sends it with one TMA
-//    bulk copy to the workspace slot prefix_slot0 + chunk, with the row's
-//    maximum and sum; pa_decode's CTAs for each sequence's own tokens merge
-//    these into the output.
+//    then per group p = 2^(s * scale * log2 e - max), rounded to bf16, into
+//    a ring of two swizzled P slots in Q's space, and the fp32 sum of p;
+//    after the last MMA each thread stages its row's output in the freed
+//    tiles and sends it with TMA bulk copies to the workspace slot
+//    prefix_slot0 + chunk, with the row's maximum and sum; pa_decode's CTAs
+//    for each sequence's own tokens merge these into the output.
+// The rings keep the CTA at ~66 KB of shared memory at head_dim 128 (half of
+// what holding the chunk's whole K and V takes).  Beside it on an SM the
+// own-token pass then fits one four-warp CTA: shared memory would hold two,
+// but an SM's registers sit in four per-quarter files and this CTA's six
+// warps take two of them twice.  Bounding the registers here so that two fit
+// made the step no faster (the two passes then contend for the same SMs).
 // Every wait is bounded; a wait that runs out sets PA_DEVERR_WAIT_TIMEOUT,
 // the CTA skips what depends on it, waits (bounded) for its own loads and
 // MMAs, frees its TMEM and leaves without writing.
@@ -49,24 +54,28 @@ struct PrefixCfg {
     static constexpr int BOX_ROWS = BS < R ? BS : R;   // 8-token blocks: two boxes per unit
     static constexpr int CH = D <= 128 ? 256 : 128;    // chunk tokens
     static constexpr int U = CH / R;                   // units per chunk
-    static constexpr int NG = CH / 64;                 // 64-token groups (S MMAs, K barriers)
+    static constexpr int NG = CH / 64;                 // 64-token groups
     static constexpr int KSL = D / 64;                 // 64-dim slabs of a 128-byte-swizzled tile
     static constexpr int M = 128;                      // query rows per CTA
     static constexpr int Q_BYTES = KSL * M * 128;
-    static constexpr int KV_BYTES = KSL * CH * 128;
-    static constexpr int P_BYTES = NG * M * 128;
-    static constexpr int KP_BYTES = KV_BYTES > P_BYTES ? KV_BYTES : P_BYTES;
-    static constexpr int QV_BYTES = KV_BYTES > Q_BYTES ? KV_BYTES : Q_BYTES;
-    // Q, then V over the same bytes; K, then P over the same bytes
-    static constexpr int QV_OFF = 0, K_OFF = QV_BYTES;
-    static constexpr int BAR_OFF = QV_BYTES + KP_BYTES;
-    // q_full, k_full[NG], v_full, s_full[NG], p_full, o_full; then the TMEM address
-    static constexpr int NBARS = 2 * NG + 4;
+    static constexpr int GROUP_BYTES = KSL * 64 * 128; // one 64-token group of K or V
+    static constexpr int P_BYTES = M * 128;            // one 64-token group of P
+    // region A: Q, then a ring of two P groups; region B: a ring of two K
+    // groups, then of two V groups
+    static constexpr int A_BYTES = Q_BYTES > 2 * P_BYTES ? Q_BYTES : 2 * P_BYTES;
+    static constexpr int B_BYTES = 2 * GROUP_BYTES;
+    static constexpr int A_OFF = 0, B_OFF = A_BYTES;
+    static constexpr int BAR_OFF = A_BYTES + B_BYTES;
+    // q_full; k_full[2], v_full[2], p_full[2], pv_done[2] (per ring slot);
+    // s_full[NG] (S of group g done); o_full; then the TMEM address
+    static constexpr int NBARS = 9 + NG + 1;
     static constexpr int SOFT_WARPS = 4;
     static constexpr int PRODUCER = SOFT_WARPS, MMA_WARP = SOFT_WARPS + 1;
     static constexpr int THREADS = (SOFT_WARPS + 2) * 32;
-    // the output is staged OCOLS columns at a time, rows padded by 4 floats
-    static constexpr int OCOLS = D < 128 ? D : 128;
+    // the output is staged OCOLS columns at a time, rows padded by 4 floats,
+    // over the freed tiles
+    static constexpr int OCOLS_MAX = D < 128 ? D : 128;
+    static constexpr int OCOLS = M * (OCOLS_MAX + 4) * 4 <= BAR_OFF ? OCOLS_MAX : 64;
     static constexpr int OSTRIDE = OCOLS + 4;
     // barriers, the TMEM address, agreement flags, then alignment slack
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 2 * 4 * 4 + 1024;
@@ -74,6 +83,7 @@ struct PrefixCfg {
     static_assert(M * OSTRIDE * 4 <= BAR_OFF, "staged output fits the freed tiles");
     static_assert((BS % R == 0 || BS == 8) && D % 64 == 0, "shared-prefix shape");
     static_assert(CH + D <= TMEM_COLS, "S and O must fit TMEM");
+    static_assert(NG >= 2, "two-slot rings");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -114,16 +124,16 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* qs = smem + C::QV_OFF;                 // Q, then V
-    unsigned char* ks = smem + C::K_OFF;                  // K tiles, then P
-    unsigned char* vs = qs;
+    unsigned char* ra = smem + C::A_OFF;                  // Q, then the P ring
+    unsigned char* rb = smem + C::B_OFF;                  // the K ring, then the V ring
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;                          // [NG]
-    uint64_t* v_full = bars + 1 + NG;
-    uint64_t* s_full = v_full + 1;                        // [NG]: S of 64-token group g done
-    uint64_t* p_full = s_full + NG;
-    uint64_t* o_full = p_full + 1;
+    uint64_t* k_full = bars + 1;                          // [2] per ring slot
+    uint64_t* v_full = bars + 3;                          // [2]
+    uint64_t* p_full = bars + 5;                          // [2]: the softmax warps wrote P
+    uint64_t* pv_done = bars + 7;                         // [2]: O += P V of the slot's group done
+    uint64_t* s_full = bars + 9;                          // [NG]: S of 64-token group g done
+    uint64_t* o_full = s_full + NG;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
     int* okw = reinterpret_cast<int*>(tmem_slot + 4);             // [2][SOFT_WARPS]
     // set by a role that gave up, read by the others after the final barrier
@@ -132,7 +142,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     if (threadIdx.x == 0) {
         failed = 0;
         for (int i = 0; i < C::NBARS; ++i)
-            mbar_init(&bars[i], i == 2 * NG + 2 ? 32 * C::SOFT_WARPS : 1);
+            mbar_init(&bars[i], (i == 5 || i == 6) ? 32 * C::SOFT_WARPS : 1);
         fence_mbar_init();
     }
     if (warp == C::MMA_WARP) {                            // the MMA warp owns TMEM
@@ -144,7 +154,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     const uint32_t s_tmem = tmem, o_tmem = tmem + CH;
-    bool v_issued = false;                                // producer lane 0 only
+    int k_issued = 0, v_issued = 0;                       // producer lane 0: groups loaded
 
     if (warp == C::PRODUCER) {
         // ------------------------------------------------ producer (lane 0) --
@@ -164,36 +174,49 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             mbar_arrive_expect_tx(q_full, C::Q_BYTES + a.tx_extra);
 #pragma unroll
             for (int b = 0; b < KSL; ++b)
-                tma_load_3d(qs + b * M * 128, &tm_q, q_full, 64 * b, kvh * G, gs + row0 / G);
-            // unit j of the chunk lands at row 16 j of every 64-dim slab
-            auto load_unit = [&](const CUtensorMap* map, unsigned char* base, uint64_t* bar,
-                                 int j) {
-                const int u = u_begin + j;
-                int id = a.num_blocks, id1 = a.num_blocks, rr = 0;
-                if (u < u_end) {                    // the prefix is whole 16-token units
-                    id = checked(__ldg(table + (u * R) / BS));
-                    if (C::BOX_ROWS < R) id1 = checked(__ldg(table + (u * R) / BS + 1));
-                    else rr = (u * R) % BS;
-                }
+                tma_load_3d(ra + b * M * 128, &tm_q, q_full, 64 * b, kvh * G, gs + row0 / G);
+            // group g (units 4g .. 4g+3 of the chunk) into ring slot g % 2:
+            // unit jj lands at row 16 jj of every 64-dim slab of the slot
+            auto load_group = [&](const CUtensorMap* map, uint64_t* bar, int g) {
+                unsigned char* base = rb + (g % 2) * C::GROUP_BYTES;
+                mbar_arrive_expect_tx(bar, C::GROUP_BYTES + a.tx_extra);
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int u = u_begin + 4 * g + jj;
+                    int id = a.num_blocks, id1 = a.num_blocks, rr = 0;
+                    if (u < u_end) {                // the prefix is whole 16-token units
+                        id = checked(__ldg(table + (u * R) / BS));
+                        if (C::BOX_ROWS < R) id1 = checked(__ldg(table + (u * R) / BS + 1));
+                        else rr = (u * R) % BS;
+                    }
 #pragma unroll
-                for (int b = 0; b < KSL; ++b) {
-                    unsigned char* dst = base + b * CH * 128 + j * R * 128;
-                    tma_load_4d(dst, map, bar, 64 * b, kvh, rr, id);
-                    if (C::BOX_ROWS < R)
-                        tma_load_4d(dst + C::BOX_ROWS * 128, map, bar, 64 * b, kvh, 0, id1);
+                    for (int b = 0; b < KSL; ++b) {
+                        unsigned char* dst = base + b * (64 * 128) + jj * R * 128;
+                        tma_load_4d(dst, map, bar, 64 * b, kvh, rr, id);
+                        if (C::BOX_ROWS < R)
+                            tma_load_4d(dst + C::BOX_ROWS * 128, map, bar, 64 * b, kvh, 0, id1);
+                    }
                 }
             };
-            for (int g = 0; g < NG; ++g) {
-                mbar_arrive_expect_tx(&k_full[g], 4 * KSL * R * 128 + a.tx_extra);
-                for (int j = 4 * g; j < 4 * g + 4; ++j) load_unit(&tm_k, ks, &k_full[g], j);
+            bool ok = true;
+            // K: a slot is refilled once the S MMAs of its previous group are done
+            for (int g = 0; g < NG && ok; ++g) {
+                if (g >= 2) ok = mbar_wait_bounded(&s_full[g - 2], 0, a.wait_ns);
+                if (ok) {
+                    load_group(&tm_k, &k_full[g % 2], g);
+                    k_issued = g + 1;
+                }
             }
-            // V goes over Q once the first MMA has read it (the last group's
-            // commit covers every S MMA)
-            if (mbar_wait_bounded(&s_full[NG - 1], 0, a.wait_ns)) {
-                mbar_arrive_expect_tx(v_full, C::KV_BYTES + a.tx_extra);
-                for (int j = 0; j < C::U; ++j) load_unit(&tm_v, vs, v_full, j);
-                v_issued = true;
-            } else {
+            // V: into the K ring once its last K groups are consumed, then once
+            // the slot's previous V group has been multiplied
+            for (int g = 0; g < NG && ok; ++g) {
+                ok = g < 2 ? mbar_wait_bounded(&s_full[NG - 2 + g], 0, a.wait_ns)
+                           : mbar_wait_bounded(&pv_done[g % 2], ((g - 2) / 2) & 1, a.wait_ns);
+                if (ok) {
+                    load_group(&tm_v, &v_full[g % 2], g);
+                    v_issued = g + 1;
+                }
+            }
+            if (!ok) {
                 raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
                 failed = 1;
             }
@@ -201,56 +224,61 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     } else if (warp == C::MMA_WARP) {
         // --------------------------------------------- MMA issuer (lane 0) --
         if (lane == 0) {
-            const uint32_t q0 = smem_addr(qs), k0 = smem_addr(ks), v0 = smem_addr(vs);
+            const uint32_t a0 = smem_addr(ra), b0 = smem_addr(rb);
             // base descriptors; a step's operand is the base plus a byte
             // offset (>> 4) added to the start-address field, which stays
             // inside its 14 bits for any shared-memory address
-            const uint64_t qd = sw128_desc(q0, 16, 1024), kd = sw128_desc(k0, 16, 1024);
-            const uint64_t pd = kd, vd = sw128_desc(v0, CH * 128, 1024);
+            const uint64_t qd = sw128_desc(a0, 16, 1024);
+            uint64_t* last = nullptr;                     // the last commit issued
+            uint32_t last_parity = 0;
             bool ok = mbar_wait_bounded(q_full, 0, a.wait_ns);
-            bool s_issued = false;
-            if (ok) {
-                for (int g = 0; g < NG && ok; ++g) {
-                    ok = mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-#pragma unroll
-                    for (int kk = 0; kk < 4 * KSL; ++kk) {
-                        const uint64_t ad = qd + (uint64_t)(((kk / 4) * M * 128 + (kk % 4) * 32) >> 4);
-                        const uint64_t bd =
-                            kd + (uint64_t)(((kk / 4) * CH * 128 + g * 64 * 128 + (kk % 4) * 32) >> 4);
-                        umma_bf16(s_tmem + 64 * g, ad, bd, umma_idesc_bf16(M, 64, false),
-                                  kk > 0);
-                    }
-                    umma_commit(&s_full[g]);          // the softmax starts on this group
-                    s_issued = true;
-                }
-            }
-            bool o_issued = false;
-            if (ok) ok = mbar_wait_bounded(p_full, 0, a.wait_ns) &&
-                         mbar_wait_bounded(v_full, 0, a.wait_ns);
-            if (ok) {
+            // S = Q K^T, one 64-token group at a time as its K tiles land
+            for (int g = 0; g < NG && ok; ++g) {
+                ok = mbar_wait_bounded(&k_full[g % 2], (g / 2) & 1, a.wait_ns);
+                if (!ok) break;
                 tc_fence_after_sync();
+                const uint64_t kd = sw128_desc(b0 + (g % 2) * C::GROUP_BYTES, 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < CH / 16; ++kk) {
-                    const uint64_t ad = pd + (uint64_t)(((kk / 4) * M * 128 + (kk % 4) * 32) >> 4);
-                    // V as B, MN-major: 64-dim slabs CH * 128 bytes apart (leading
-                    // offset), 8-token atoms 1 KiB apart (stride offset)
-                    const uint64_t bd = vd + (uint64_t)((kk * 16 * 128) >> 4);
-                    umma_bf16(o_tmem, ad, bd, umma_idesc_bf16(M, D, true), kk > 0);
+                for (int kk = 0; kk < 4 * KSL; ++kk) {
+                    const uint64_t ad = qd + (uint64_t)(((kk / 4) * M * 128 + (kk % 4) * 32) >> 4);
+                    const uint64_t bd = kd + (uint64_t)(((kk / 4) * 64 * 128 + (kk % 4) * 32) >> 4);
+                    umma_bf16(s_tmem + 64 * g, ad, bd, umma_idesc_bf16(M, 64, false), kk > 0);
                 }
-                umma_commit(o_full);
-                o_issued = true;
+                umma_commit(&s_full[g]);              // the softmax starts on this group
+                last = &s_full[g];
+                last_parity = 0;
             }
-            if (!ok) {
+            // O = P V, group by group as P and V land (P K-major; V MN-major:
+            // 64-dim slabs 64 * 128 bytes apart as the leading offset,
+            // 8-token atoms 1 KiB apart as the stride offset)
+            for (int g = 0; g < NG && ok; ++g) {
+                ok = mbar_wait_bounded(&p_full[g % 2], (g / 2) & 1, a.wait_ns) &&
+                     mbar_wait_bounded(&v_full[g % 2], (g / 2) & 1, a.wait_ns);
+                if (!ok) break;
+                tc_fence_after_sync();
+                const uint64_t pd = sw128_desc(a0 + (g % 2) * C::P_BYTES, 16, 1024);
+                const uint64_t vd = sw128_desc(b0 + (g % 2) * C::GROUP_BYTES, 64 * 128, 1024);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = pd + (uint64_t)((kk * 32) >> 4);
+                    const uint64_t bd = vd + (uint64_t)((kk * 16 * 128) >> 4);
+                    umma_bf16(o_tmem, ad, bd, umma_idesc_bf16(M, D, true), g > 0 || kk > 0);
+                }
+                umma_commit(&pv_done[g % 2]);         // the slot's P and V are free again
+                last = &pv_done[g % 2];
+                last_parity = (g / 2) & 1;
+            }
+            if (ok) {
+                umma_commit(o_full);
+                last = o_full;
+                last_parity = 0;
+            } else {
                 raise_error(a.err, PA_DEVERR_WAIT_TIMEOUT);
                 failed = 1;
             }
-            // nothing this thread issued may still run when TMEM is freed
-            if (o_issued) (void)mbar_wait_bounded(o_full, 0, a.wait_ns);
-            else if (s_issued)   // the last group committed covers every earlier MMA
-                for (int g = NG - 1; g >= 0; --g)
-                    if (mbar_wait_bounded(&s_full[g], 0, a.wait_ns)) break;
+            // nothing this thread issued may still run when TMEM is freed (the
+            // last commit covers every earlier MMA)
+            if (last) (void)mbar_wait_bounded(last, last_parity, a.wait_ns);
         }
     } else {
         // -------------------------------- softmax and epilogue: warps 0-3 --
@@ -290,11 +318,17 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             }
         }
         if (ok) {
-            // pass 2: p = 2^(x - m) into the P tile (bf16, 128-byte swizzle), sum of p;
-            // 64 tokens = one slab row of 128 bytes per round trip
-            const uint32_t prow = smem_addr(ks) + (uint32_t)r * 128;
+            // pass 2: p = 2^(x - m) into the P ring (bf16, 128-byte swizzle), sum
+            // of p; a group of 64 tokens is one slab row of 128 bytes, written
+            // once the slot's previous group has been multiplied
+            const uint32_t prow = smem_addr(ra) + (uint32_t)r * 128;
 #pragma unroll 1
-            for (int c = 0; c < CH / 64; ++c) {
+            for (int c = 0; c < CH / 64 && ok; ++c) {
+                if (c >= 2) {
+                    ok = __all_sync(FULL_MASK, mbar_wait_bounded(&pv_done[c % 2],
+                                                                 ((c - 2) / 2) & 1, a.wait_ns));
+                    if (!ok) break;
+                }
                 float v[64];
                 tmem_ld32(s_tmem + lane_off + 64 * c, *reinterpret_cast<float(*)[32]>(v));
                 tmem_ld32(s_tmem + lane_off + 64 * c + 32,
@@ -310,7 +344,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                     l += p0 + p1;
                     w[j] = pack_bf16x2(p0, p1);
                 }
-                const uint32_t base = prow + (uint32_t)c * (M * 128);
+                const uint32_t base = prow + (uint32_t)(c % 2) * C::P_BYTES;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const uint32_t addr = base + (uint32_t)((q ^ (r & 7)) << 4);
@@ -319,11 +353,11 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                                  "r"(w[4 * q + 3])
                                  : "memory");
                 }
+                fence_proxy_async_smem();               // P is read by the tensor cores
+                tc_fence_before_sync();
+                mbar_arrive(&p_full[c % 2]);
             }
-            fence_proxy_async_smem();                   // P is read by the tensor cores
-            tc_fence_before_sync();
-            mbar_arrive(p_full);
-            ok = __all_sync(FULL_MASK, mbar_wait_bounded(o_full, 0, a.wait_ns));
+            if (ok) ok = __all_sync(FULL_MASK, mbar_wait_bounded(o_full, 0, a.wait_ns));
         }
         ok = all_ok(0, ok);
         if (!ok) {
@@ -373,10 +407,16 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     tc_fence_before_sync();
     __syncthreads();
     if (failed && warp == C::PRODUCER && lane == 0) {
-        // loads may still be in flight after a role gave up: wait (bounded) for them
+        // loads may still be in flight after a role gave up: wait (bounded) for
+        // them.  A slot is refilled only after its previous group landed and
+        // was consumed, so only each slot's last group can be outstanding.
         (void)mbar_wait_bounded(q_full, 0, a.wait_ns);
-        for (int g = 0; g < NG; ++g) (void)mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
-        if (v_issued) (void)mbar_wait_bounded(v_full, 0, a.wait_ns);
+        for (int sl = 0; sl < 2; ++sl) {
+            const int gk = k_issued - 1 - ((k_issued - 1 - sl) & 1);   // last K group in slot sl
+            if (gk >= 0 && gk % 2 == sl) (void)mbar_wait_bounded(&k_full[sl], (gk / 2) & 1, a.wait_ns);
+            const int gv = v_issued - 1 - ((v_issued - 1 - sl) & 1);
+            if (gv >= 0 && gv % 2 == sl) (void)mbar_wait_bounded(&v_full[sl], (gv / 2) & 1, a.wait_ns);
+        }
     }
     if (warp == C::MMA_WARP) {
         tc_fence_after_sync();
