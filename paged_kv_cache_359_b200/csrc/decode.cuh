@@ -1202,11 +1202,13 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                 pdl_wait();                                // the shared pass is complete
                 if (nchunks) {
                     // merge with the shared pass's chunks of each head.  A thread
-                    // writes OPT groups of 4 outputs (g, d .. d+3); it first loads
-                    // the chunk maxima of its heads, then the chunks' float4
-                    // outputs and sums, CB chunks of every output at a time, all
-                    // loads of a batch in flight at once (about 8 float4 per
-                    // thread, which keeps them in registers at every head_dim)
+                    // writes OPT groups of 4 outputs (g, d .. d+3).  It loads the
+                    // maxima, sums and float4 outputs of CB chunks of every output
+                    // at a time, all in flight at once (about 8 float4 per thread,
+                    // which keeps them in registers at every head_dim), then
+                    // rescales what it holds to the batch's new maximum and adds
+                    // the batch in chunk order: one round trip per batch, and with
+                    // every chunk in one batch the sums of the common maximum
                     __syncthreads();                       // x is complete
                     constexpr int Q4 = D / 4;                        // float4 per head row
                     constexpr int OPT = (G * Q4 + NT - 1) / NT;
@@ -1220,41 +1222,54 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                         gg[k] = idx < G * Q4 ? idx / Q4 : 0;
                         qq[k] = idx % Q4;
                         mm[k] = x[gg[k]];
+                        const float* xo = x + 2 * G + gg[k] * D + 4 * qq[k];
+                        num[k] = make_float4(xo[0], xo[1], xo[2], xo[3]);
+                        den[k] = x[G + gg[k]];
                     }
                     auto slot_of = [&](int k, int c) {
                         return (head0 + gg[k]) * a.slot_stride + a.prefix_slot0 + c;
                     };
-                    for (int c0 = 0; c0 < nchunks; c0 += 8) {
-    #pragma unroll
-                        for (int k = 0; k < OPT; ++k)
-    #pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                if (c0 + c < nchunks) mm[k] = fmaxf(mm[k], a.ws_m[slot_of(k, c0 + c)]);
-                    }
-    #pragma unroll
-                    for (int k = 0; k < OPT; ++k) {
-                        const float own = x[gg[k]];
-                        const float e0 = own == -INFINITY ? 0.f : exp2_approx(own - mm[k]);
-                        const float* xo = x + 2 * G + gg[k] * D + 4 * qq[k];
-                        num[k] = make_float4(e0 * xo[0], e0 * xo[1], e0 * xo[2], e0 * xo[3]);
-                        den[k] = e0 * x[G + gg[k]];
-                    }
+                    bool first = true;                     // num / den still unscaled
                     for (int c0 = 0; c0 < nchunks; c0 += CB) {
+                        float bm[OPT][CB], bl[OPT][CB];
+                        float4 bo[OPT][CB];
     #pragma unroll
                         for (int k = 0; k < OPT; ++k)
+    #pragma unroll
+                            for (int c = 0; c < CB; ++c) {
+                                bm[k][c] = -INFINITY;
+                                if (c0 + c < nchunks) {
+                                    const size_t sl = slot_of(k, c0 + c);
+                                    bm[k][c] = a.ws_m[sl];
+                                    bl[k][c] = a.ws_l[sl];
+                                    bo[k][c] = reinterpret_cast<const float4*>(a.ws_o + sl * D)[qq[k]];
+                                }
+                            }
+    #pragma unroll
+                        for (int k = 0; k < OPT; ++k) {
+                            float nm = mm[k];
+    #pragma unroll
+                            for (int c = 0; c < CB; ++c) nm = fmaxf(nm, bm[k][c]);
+                            // the own tokens (first batch) or the earlier batches, at nm
+                            const float e0 = mm[k] == -INFINITY ? 0.f : exp2_approx(mm[k] - nm);
+                            if (first || nm != mm[k]) {
+                                num[k] = make_float4(e0 * num[k].x, e0 * num[k].y,
+                                                     e0 * num[k].z, e0 * num[k].w);
+                                den[k] = e0 * den[k];
+                            }
+                            mm[k] = nm;
     #pragma unroll
                             for (int c = 0; c < CB; ++c)
                                 if (c0 + c < nchunks) {
-                                    const size_t sl = slot_of(k, c0 + c);
-                                    const float ec = exp2_approx(a.ws_m[sl] - mm[k]);
-                                    const float4 o4 =
-                                        reinterpret_cast<const float4*>(a.ws_o + sl * D)[qq[k]];
-                                    num[k].x = fmaf(ec, o4.x, num[k].x);
-                                    num[k].y = fmaf(ec, o4.y, num[k].y);
-                                    num[k].z = fmaf(ec, o4.z, num[k].z);
-                                    num[k].w = fmaf(ec, o4.w, num[k].w);
-                                    den[k] = fmaf(ec, a.ws_l[sl], den[k]);
+                                    const float ec = exp2_approx(bm[k][c] - nm);
+                                    num[k].x = fmaf(ec, bo[k][c].x, num[k].x);
+                                    num[k].y = fmaf(ec, bo[k][c].y, num[k].y);
+                                    num[k].z = fmaf(ec, bo[k][c].z, num[k].z);
+                                    num[k].w = fmaf(ec, bo[k][c].w, num[k].w);
+                                    den[k] = fmaf(ec, bl[k][c], den[k]);
                                 }
+                        }
+                        first = false;
                     }
     #pragma unroll
                     for (int k = 0; k < OPT; ++k)
