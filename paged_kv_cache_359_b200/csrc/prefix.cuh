@@ -15,15 +15,15 @@
 // 256 (head_dim <= 128) or 128 (head_dim 256).  Roles:
 //  * producer warp: TMA loads of the CTA's 128 query rows (a 3-D box over
 //    q [S][Hq][D]: members x G heads, row = member * G + head) and of the
-//    chunk's K, then V, tiles in 64-token groups through a ring of two
-//    group slots (a slot is refilled once the MMAs that read its previous
-//    group are done), all 128-byte swizzled; a unit past the prefix is
-//    loaded from outside the pool map, which TMA fills with zeros;
+//    chunk's K tiles in 64-token groups, all at once, one slot per group;
+//    each group's V tiles go into its slot once the MMAs that read its K
+//    are done; all 128-byte swizzled; a unit past the prefix is loaded from
+//    outside the pool map, which TMA fills with zeros;
 //  * MMA warp (one elected thread): S = Q K^T into TMEM (M = 128 rows,
 //    N = 64 tokens per group as its K tiles land, K = head_dim), a commit
 //    per group; then, group by group as its P and V tiles land, O += P V
 //    into TMEM (M = 128, N = head_dim, K = 64 tokens, V read MN-major), a
-//    commit per group that frees the group's P and V slots;
+//    commit per group that frees the group's P slot;
 //  * four softmax warps, one TMEM lane (query row) per thread: the exact
 //    maximum of the row's scores over the chunk (masked past the prefix),
 //    then per group p = 2^(s * scale * log2 e - max), rounded to bf16, into
@@ -32,12 +32,12 @@
 //    tiles and sends it with TMA bulk copies to the workspace slot
 //    prefix_slot0 + chunk, with the row's maximum and sum; pa_decode's CTAs
 //    for each sequence's own tokens merge these into the output.
-// The rings keep the CTA at ~66 KB of shared memory at head_dim 128 (half of
-// what holding the chunk's whole K and V takes).  Beside it on an SM the
-// own-token pass then fits one four-warp CTA: shared memory would hold two,
-// but an SM's registers sit in four per-quarter files and this CTA's six
-// warps take two of them twice.  Bounding the registers here so that two fit
-// made the step no faster (the two passes then contend for the same SMs).
+// The CTA holds Q (or the P ring) and one chunk of K/V: 97 KB of shared
+// memory at head_dim 128.  Beside it on an SM the own-token pass fits one
+// four-warp CTA: an SM's registers sit in four per-quarter files, and this
+// CTA's six warps take two of them twice.  Bounding the registers here so
+// that two fit made the step no faster (the two passes then contend for the
+// same SMs); a two-slot K/V ring (67 KB) waited on four rounds of loads.
 // Every wait is bounded; a wait that runs out sets PA_DEVERR_WAIT_TIMEOUT,
 // the CTA skips what depends on it, waits (bounded) for its own loads and
 // MMAs, frees its TMEM and leaves without writing.
@@ -60,15 +60,16 @@ struct PrefixCfg {
     static constexpr int Q_BYTES = KSL * M * 128;
     static constexpr int GROUP_BYTES = KSL * 64 * 128; // one 64-token group of K or V
     static constexpr int P_BYTES = M * 128;            // one 64-token group of P
-    // region A: Q, then a ring of two P groups; region B: a ring of two K
-    // groups, then of two V groups
+    // region A: Q, then a ring of two P groups; region B: a slot per 64-token
+    // group, which holds the group's K and then its V
     static constexpr int A_BYTES = Q_BYTES > 2 * P_BYTES ? Q_BYTES : 2 * P_BYTES;
-    static constexpr int B_BYTES = 2 * GROUP_BYTES;
+    static constexpr int B_BYTES = NG * GROUP_BYTES;
     static constexpr int A_OFF = 0, B_OFF = A_BYTES;
     static constexpr int BAR_OFF = A_BYTES + B_BYTES;
-    // q_full; k_full[2], v_full[2], p_full[2], pv_done[2] (per ring slot);
-    // s_full[NG] (S of group g done); o_full; then the TMEM address
-    static constexpr int NBARS = 9 + NG + 1;
+    // q_full; k_full[NG], v_full[NG] (per group); p_full[2], pv_done[2] (per
+    // P slot); s_full[NG] (S of group g done); o_full; then the TMEM address
+    static constexpr int NBARS = 6 + 3 * NG;
+    static constexpr int P_FULL = 1 + 2 * NG;         // index of p_full[0]
     static constexpr int SOFT_WARPS = 4;
     static constexpr int PRODUCER = SOFT_WARPS, MMA_WARP = SOFT_WARPS + 1;
     static constexpr int THREADS = (SOFT_WARPS + 2) * 32;
@@ -83,7 +84,7 @@ struct PrefixCfg {
     static_assert(M * OSTRIDE * 4 <= BAR_OFF, "staged output fits the freed tiles");
     static_assert((BS % R == 0 || BS == 8) && D % 64 == 0, "shared-prefix shape");
     static_assert(CH + D <= TMEM_COLS, "S and O must fit TMEM");
-    static_assert(NG >= 2, "two-slot rings");
+    static_assert(NG >= 2, "a two-slot P ring");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -125,14 +126,14 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* ra = smem + C::A_OFF;                  // Q, then the P ring
-    unsigned char* rb = smem + C::B_OFF;                  // the K ring, then the V ring
+    unsigned char* rb = smem + C::B_OFF;                  // per group: K, then V
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     uint64_t* q_full = bars;
-    uint64_t* k_full = bars + 1;                          // [2] per ring slot
-    uint64_t* v_full = bars + 3;                          // [2]
-    uint64_t* p_full = bars + 5;                          // [2]: the softmax warps wrote P
-    uint64_t* pv_done = bars + 7;                         // [2]: O += P V of the slot's group done
-    uint64_t* s_full = bars + 9;                          // [NG]: S of 64-token group g done
+    uint64_t* k_full = bars + 1;                          // [NG] per group slot
+    uint64_t* v_full = k_full + NG;                       // [NG]
+    uint64_t* p_full = v_full + NG;                       // [2]: the softmax warps wrote P
+    uint64_t* pv_done = p_full + 2;                       // [2]: O += P V of the P slot's group done
+    uint64_t* s_full = pv_done + 2;                       // [NG]: S of 64-token group g done
     uint64_t* o_full = s_full + NG;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
     int* okw = reinterpret_cast<int*>(tmem_slot + 4);             // [2][SOFT_WARPS]
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     if (threadIdx.x == 0) {
         failed = 0;
         for (int i = 0; i < C::NBARS; ++i)
-            mbar_init(&bars[i], (i == 5 || i == 6) ? 32 * C::SOFT_WARPS : 1);
+            mbar_init(&bars[i], (i == C::P_FULL || i == C::P_FULL + 1) ? 32 * C::SOFT_WARPS : 1);
         fence_mbar_init();
     }
     if (warp == C::MMA_WARP) {                            // the MMA warp owns TMEM
@@ -175,10 +176,10 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
 #pragma unroll
             for (int b = 0; b < KSL; ++b)
                 tma_load_3d(ra + b * M * 128, &tm_q, q_full, 64 * b, kvh * G, gs + row0 / G);
-            // group g (units 4g .. 4g+3 of the chunk) into ring slot g % 2:
-            // unit jj lands at row 16 jj of every 64-dim slab of the slot
+            // group g (units 4g .. 4g+3 of the chunk) into slot g: unit jj
+            // lands at row 16 jj of every 64-dim slab of the slot
             auto load_group = [&](const CUtensorMap* map, uint64_t* bar, int g) {
-                unsigned char* base = rb + (g % 2) * C::GROUP_BYTES;
+                unsigned char* base = rb + g * C::GROUP_BYTES;
                 mbar_arrive_expect_tx(bar, C::GROUP_BYTES + a.tx_extra);
                 for (int jj = 0; jj < 4; ++jj) {
                     const int u = u_begin + 4 * g + jj;
@@ -198,21 +199,16 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
                 }
             };
             bool ok = true;
-            // K: a slot is refilled once the S MMAs of its previous group are done
-            for (int g = 0; g < NG && ok; ++g) {
-                if (g >= 2) ok = mbar_wait_bounded(&s_full[g - 2], 0, a.wait_ns);
-                if (ok) {
-                    load_group(&tm_k, &k_full[g % 2], g);
-                    k_issued = g + 1;
-                }
+            // every K group at once; then each V group into its K group's slot
+            // once the S MMAs of that group are done
+            for (int g = 0; g < NG; ++g) {
+                load_group(&tm_k, &k_full[g], g);
+                k_issued = g + 1;
             }
-            // V: into the K ring once its last K groups are consumed, then once
-            // the slot's previous V group has been multiplied
             for (int g = 0; g < NG && ok; ++g) {
-                ok = g < 2 ? mbar_wait_bounded(&s_full[NG - 2 + g], 0, a.wait_ns)
-                           : mbar_wait_bounded(&pv_done[g % 2], ((g - 2) / 2) & 1, a.wait_ns);
+                ok = mbar_wait_bounded(&s_full[g], 0, a.wait_ns);
                 if (ok) {
-                    load_group(&tm_v, &v_full[g % 2], g);
+                    load_group(&tm_v, &v_full[g], g);
                     v_issued = g + 1;
                 }
             }
@@ -234,10 +230,10 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             bool ok = mbar_wait_bounded(q_full, 0, a.wait_ns);
             // S = Q K^T, one 64-token group at a time as its K tiles land
             for (int g = 0; g < NG && ok; ++g) {
-                ok = mbar_wait_bounded(&k_full[g % 2], (g / 2) & 1, a.wait_ns);
+                ok = mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
                 if (!ok) break;
                 tc_fence_after_sync();
-                const uint64_t kd = sw128_desc(b0 + (g % 2) * C::GROUP_BYTES, 16, 1024);
+                const uint64_t kd = sw128_desc(b0 + g * C::GROUP_BYTES, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4 * KSL; ++kk) {
                     const uint64_t ad = qd + (uint64_t)(((kk / 4) * M * 128 + (kk % 4) * 32) >> 4);
@@ -253,18 +249,18 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
             // 8-token atoms 1 KiB apart as the stride offset)
             for (int g = 0; g < NG && ok; ++g) {
                 ok = mbar_wait_bounded(&p_full[g % 2], (g / 2) & 1, a.wait_ns) &&
-                     mbar_wait_bounded(&v_full[g % 2], (g / 2) & 1, a.wait_ns);
+                     mbar_wait_bounded(&v_full[g], 0, a.wait_ns);
                 if (!ok) break;
                 tc_fence_after_sync();
                 const uint64_t pd = sw128_desc(a0 + (g % 2) * C::P_BYTES, 16, 1024);
-                const uint64_t vd = sw128_desc(b0 + (g % 2) * C::GROUP_BYTES, 64 * 128, 1024);
+                const uint64_t vd = sw128_desc(b0 + g * C::GROUP_BYTES, 64 * 128, 1024);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t ad = pd + (uint64_t)((kk * 32) >> 4);
                     const uint64_t bd = vd + (uint64_t)((kk * 16 * 128) >> 4);
                     umma_bf16(o_tmem, ad, bd, umma_idesc_bf16(M, D, true), g > 0 || kk > 0);
                 }
-                umma_commit(&pv_done[g % 2]);         // the slot's P and V are free again
+                umma_commit(&pv_done[g % 2]);         // the P slot is free again
                 last = &pv_done[g % 2];
                 last_parity = (g / 2) & 1;
             }
@@ -408,15 +404,10 @@ __global__ void __launch_bounds__(PrefixCfg<D, BS, G>::THREADS, 1)
     __syncthreads();
     if (failed && warp == C::PRODUCER && lane == 0) {
         // loads may still be in flight after a role gave up: wait (bounded) for
-        // them.  A slot is refilled only after its previous group landed and
-        // was consumed, so only each slot's last group can be outstanding.
+        // them (a V group is loaded only after its slot's K group landed)
         (void)mbar_wait_bounded(q_full, 0, a.wait_ns);
-        for (int sl = 0; sl < 2; ++sl) {
-            const int gk = k_issued - 1 - ((k_issued - 1 - sl) & 1);   // last K group in slot sl
-            if (gk >= 0 && gk % 2 == sl) (void)mbar_wait_bounded(&k_full[sl], (gk / 2) & 1, a.wait_ns);
-            const int gv = v_issued - 1 - ((v_issued - 1 - sl) & 1);
-            if (gv >= 0 && gv % 2 == sl) (void)mbar_wait_bounded(&v_full[sl], (gv / 2) & 1, a.wait_ns);
-        }
+        for (int g = 0; g < k_issued; ++g) (void)mbar_wait_bounded(&k_full[g], 0, a.wait_ns);
+        for (int g = 0; g < v_issued; ++g) (void)mbar_wait_bounded(&v_full[g], 0, a.wait_ns);
     }
     if (warp == C::MMA_WARP) {
         tc_fence_after_sync();
