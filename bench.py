@@ -651,7 +651,7 @@ def _view(buf, seg, dtype, shape):
 
 
 # untimed steps the end-to-end loop runs after its timed window (see run_e2e)
-E2E_TRAIL = 4
+E2E_TRAIL = 8
 
 
 def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3):
