@@ -647,7 +647,8 @@ struct Layout {
     // warps per CTA: four, or two when a stage is 16 KiB (head_dim 256 on
     // the tensor-core unit), so that three CTAs still fit an SM with a
     // two-stage ring per warp (about 192 KiB of loads in flight per SM);
-    // half of that for the shared-prefix decode's own-token pass
+    // half of that for the shared-prefix decode's own-token pass at
+    // head_dim 64
     static constexpr int NW = (STAGE_BYTES >= 16384 ? 2 : 4) / (HALF_WARPS ? 2 : 1);
     // stages per warp: about 12 KiB of ring per warp, at least two; with
     // 4 KiB stages (head_dim 64) the smaller CTA lets four CTAs share an SM,
@@ -877,9 +878,12 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
     fence_proxy_async_smem();
 }
 
-// Whether the own-token pass of the shared-prefix decode runs half-width CTAs.
+// Whether the own-token pass of the shared-prefix decode runs half-width CTAs:
+// at head_dim 64, so that more of its short items start beside the shared
+// pass.  At 128 and 256 an item's tokens streamed by more warps finish sooner
+// (at 256 the one-warp CTA took 63 of a step's 83 us).
 template <class U>
-__host__ __device__ constexpr bool own_half_width() { return U::D != 128; }
+__host__ __device__ constexpr bool own_half_width() { return U::D == 64; }
 
 template <class U, Mode MODE>
 __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<U>()>::NW * 32)
@@ -1208,11 +1212,15 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                     // which keeps them in registers at every head_dim), then
                     // rescales what it holds to the batch's new maximum and adds
                     // the batch in chunk order: one round trip per batch, and with
-                    // every chunk in one batch the sums of the common maximum
+                    // every chunk in one batch the sums of the common maximum.
+                    // The own-token pass keeps up to 16 float4 per thread in
+                    // flight (4 chunks of 4 outputs at head_dim 256)
                     __syncthreads();                       // x is complete
                     constexpr int Q4 = D / 4;                        // float4 per head row
                     constexpr int OPT = (G * Q4 + NT - 1) / NT;
-                    constexpr int CB = OPT >= 8 ? 1 : 8 / OPT;     // chunks per batch
+                    constexpr int CB = MODE == Mode::Own
+                                           ? (OPT >= 16 ? 1 : OPT >= 8 ? 2 : OPT >= 4 ? 4 : 8 / OPT)
+                                           : (OPT >= 8 ? 1 : 8 / OPT);    // chunks per batch
                     float mm[OPT], den[OPT];
                     float4 num[OPT];
                     int gg[OPT], qq[OPT];

@@ -11,8 +11,9 @@
 // from HBM once per kv head (once per 128 query rows from L2) instead of
 // once per sequence.
 //
-// CTA = (prefix chunk of CH tokens, kv head, group x 128-row block); CH is
-// 256 (head_dim <= 128) or 128 (head_dim 256).  Roles:
+// CTA = (prefix chunk of CH = 256 tokens, kv head, group x 128-row block);
+// S (CH columns) and O (head_dim columns) share the SM's 512 TMEM columns, so
+// at head_dim 256 a CTA holds all of them.  Roles:
 //  * producer warp: TMA loads of the CTA's 128 query rows (a 3-D box over
 //    q [S][Hq][D]: members x G heads, row = member * G + head) and of the
 //    chunk's K tiles in 64-token groups, all at once, one slot per group;
@@ -33,7 +34,8 @@
 //    prefix_slot0 + chunk, with the row's maximum and sum; pa_decode's CTAs
 //    for each sequence's own tokens merge these into the output.
 // The CTA holds Q (or the P ring) and one chunk of K/V: 97 KB of shared
-// memory at head_dim 128.  Beside it on an SM the own-token pass fits one
+// memory at head_dim 128 (193 KB at 256, which leaves no room beside it).
+// At head_dim 128, beside it on an SM the own-token pass fits one
 // four-warp CTA: an SM's registers sit in four per-quarter files, and this
 // CTA's six warps take two of them twice.  Bounding the registers here so
 // that two fit made the step no faster (the two passes then contend for the
@@ -52,7 +54,7 @@ struct PrefixCfg {
     static constexpr int D = D_, BS = BS_, G = G_;
     static constexpr int R = 16;                       // tokens per unit (one or two TMA boxes)
     static constexpr int BOX_ROWS = BS < R ? BS : R;   // 8-token blocks: two boxes per unit
-    static constexpr int CH = D <= 128 ? 256 : 128;    // chunk tokens
+    static constexpr int CH = 256;                     // chunk tokens
     static constexpr int U = CH / R;                   // units per chunk
     static constexpr int NG = CH / 64;                 // 64-token groups
     static constexpr int KSL = D / 64;                 // 64-dim slabs of a 128-byte-swizzled tile
@@ -90,9 +92,13 @@ struct PrefixCfg {
 
 constexpr int PREFIX_ROWS_PER_CTA = 128;
 
-// Tokens per prefix chunk (one CTA's share of the shared prefix).
+// Tokens per prefix chunk (one CTA's share of the shared prefix).  At
+// head_dim 256, 128-token chunks (two CTAs' worth of the SM's TMEM columns in
+// one wave each) measured 0.0551 against 0.0657 ms per cascade step: twice
+// the CTAs in two waves, and twice the partials to merge.
 __host__ __device__ constexpr int prefix_chunk_tokens(int head_dim) {
-    return head_dim <= 128 ? 256 : 128;
+    (void)head_dim;
+    return 256;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
