@@ -648,7 +648,7 @@ struct Layout {
     // the tensor-core unit), so that three CTAs still fit an SM with a
     // two-stage ring per warp (about 192 KiB of loads in flight per SM);
     // half of that for the shared-prefix decode's own-token pass at
-    // head_dim 64
+    // head_dim 64 and 128
     static constexpr int NW = (STAGE_BYTES >= 16384 ? 2 : 4) / (HALF_WARPS ? 2 : 1);
     // stages per warp: about 12 KiB of ring per warp, at least two; with
     // 4 KiB stages (head_dim 64) the smaller CTA lets four CTAs share an SM,
@@ -879,11 +879,12 @@ __device__ __forceinline__ void run_item(Ctx<U>& cx, const CUtensorMap* tm_k,
 }
 
 // Whether the own-token pass of the shared-prefix decode runs half-width CTAs:
-// at head_dim 64, so that more of its short items start beside the shared
-// pass.  At 128 and 256 an item's tokens streamed by more warps finish sooner
-// (at 256 the one-warp CTA took 63 of a step's 83 us).
+// at head_dim 64 and 128, so that more of its short items start beside the
+// shared pass (three two-warp CTAs fit beside a 97 KB shared CTA at 128).  At
+// 256 the shared CTA leaves no room beside it, and a two-warp CTA streams an
+// item twice as fast as one warp (which took 63 of a step's 83 us).
 template <class U>
-__host__ __device__ constexpr bool own_half_width() { return U::D == 64; }
+__host__ __device__ constexpr bool own_half_width() { return U::D != 256; }
 
 template <class U, Mode MODE>
 __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<U>()>::NW * 32)

@@ -103,7 +103,7 @@ pa_status launch_decode_g(const DecodeLaunch& l) {
                 if (e != cudaSuccess)
                     return fail(PA_ERR_CUDA, "shared-prefix launch: %s", cudaGetErrorString(e));
             }
-            // the own-token pass: longest-first (half-width CTAs at head_dim 64)
+            // the own-token pass: longest-first (half-width CTAs but at head_dim 256)
             using Lo = Layout<U, own_half_width<U>()>;
             static std::atomic<unsigned long long> done_o{0};
             auto ok = paged_decode_kernel<U, Mode::Own>;

@@ -35,11 +35,12 @@
 //    for each sequence's own tokens merge these into the output.
 // The CTA holds Q (or the P ring) and one chunk of K/V: 97 KB of shared
 // memory at head_dim 128 (193 KB at 256, which leaves no room beside it).
-// At head_dim 128, beside it on an SM the own-token pass fits one
-// four-warp CTA: an SM's registers sit in four per-quarter files, and this
-// CTA's six warps take two of them twice.  Bounding the registers here so
-// that two fit made the step no faster (the two passes then contend for the
-// same SMs); a two-slot K/V ring (67 KB) waited on four rounds of loads.
+// At head_dim 128, beside it on an SM the own-token pass fits three two-warp
+// CTAs, or one four-warp CTA: an SM's registers sit in four per-quarter
+// files, and this CTA's six warps take two of them twice.  Bounding the
+// registers here so that two four-warp CTAs fit made the step no faster (the
+// two passes then contend for the same SMs); a two-slot K/V ring (67 KB)
+// waited on four rounds of loads.
 // Every wait is bounded; a wait that runs out sets PA_DEVERR_WAIT_TIMEOUT,
 // the CTA skips what depends on it, waits (bounded) for its own loads and
 // MMAs, frees its TMEM and leaves without writing.
