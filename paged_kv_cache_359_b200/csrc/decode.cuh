@@ -900,10 +900,16 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
     // past its own wait.  It therefore streams its tokens first and waits for
     // the shared pass only before the merge, so the two overlap where SMs
     // are free; every CTA still waits before it leaves, which keeps the
-    // stream's completion order.  Every other launch waits here.
-    const bool late_wait = MODE == Mode::Own;
+    // stream's completion order.  pa_decode's grid stages the context
+    // lengths and picks its first item before it waits: no kernel of this
+    // library writes the lengths, and a caller's kernel that does completes
+    // before this grid starts (it does not release its dependents early), so
+    // that set-up overlaps the previous grid's last wave.  It releases its
+    // own dependents only after its wait, so a grid never starts before the
+    // one two launches back has completed.  Every other launch waits here.
+    const bool late_wait = MODE == Mode::Own || MODE == Mode::Decode;
     if (!late_wait) pdl_wait();
-    pdl_launch_dependents();
+    if (MODE != Mode::Decode) pdl_launch_dependents();
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -1095,6 +1101,7 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                 for (int i = threadIdx.x; i < S; i += NT) lens[i] = own_tokens(i);
             }
             __syncthreads();
+            bool waited = false;                            // pa_decode: griddepcontrol.wait done
             for (int item = blockIdx.x;;) {
                 const int r = item / Hk;
                 if (S <= DIRECT_MAX) {
@@ -1142,6 +1149,13 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                     }
                 }
                 __syncthreads();
+                if constexpr (MODE == Mode::Decode) {
+                    if (!waited) {                          // first item: see the kernel's top
+                        pdl_wait();
+                        pdl_launch_dependents();
+                        waited = true;
+                    }
+                }
                 seq = pick[0];
                 kvh = item % Hk;
                 int tok0;                                   // whole 16-token units
