@@ -654,7 +654,7 @@ def _view(buf, seg, dtype, shape):
 E2E_TRAIL = 8
 
 
-def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3):
+def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 4):
     """Through the public API from host buffers, as a serving loop runs it.
 
     Every step: the host allocator appends a token to every sequence, writing
@@ -668,10 +668,12 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
     decodes, in one launch (unfused: pa_update_block_tables,
     pa_reshape_and_cache, then the decode); the step's output comes back
     device->host and the host reads it.  A ring of ``ring`` buffer sets lets
-    the host run up to ring - 1 steps ahead of the last completed download:
-    step i's uploads go out as soon as step i - ring has been read back, on
-    their own stream, and downloads have a third stream, so copies overlap
-    the neighbouring steps' kernels.  The timed region spans every copy of
+    the host run ahead of the last completed download: step i's uploads and
+    allocator work are staged, on their own stream, as soon as step i - ring
+    has been read back and before step i - 1 is launched, so that when step
+    i is launched its upload has usually landed and the compute stream needs
+    no dependency on the upload stream; downloads have a third stream, so
+    copies overlap the neighbouring steps' kernels.  The timed region spans every copy of
     every timed step.  Python's cyclic garbage collector is paused over it
     (after a collection), as a serving loop does once it has started, so
     that a collection pass does not stall the host in the middle.
@@ -733,6 +735,8 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
             self.h2d, self.done, self.d2h = (torch.cuda.Event(), torch.cuda.Event(),
                                              torch.cuda.Event())
             self.used = False
+            self.staged = -1                           # the step whose inputs it holds
+            self.n = self.meta_used = 0
 
     bufs = [Buf() for _ in range(ring)]
     counts = {"h2d": 0, "d2h": 0, "kv": 0}
@@ -743,7 +747,9 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
         float(b.out_h.view(-1)[0])                     # the host reads the result
         b.used = False
 
-    def step(i, count):
+    def stage(i):
+        """Step i's uploads and host allocator work, one step ahead of its
+        launch so that the upload has landed when the launch is issued."""
         b = bufs[i % ring]
         if b.used:
             read_back(b)                               # step i - ring is done with b
@@ -755,16 +761,23 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
         _, cw = loop.alloc.append_slots(tables_np, lens_np, slots_out=b.slots_h,
                                         pairs_out=pairs_h)
         b.lens_h[:] = lens_np
-        n = len(cw)
-        if n:
-            b.cows_h[:n] = cw
-        meta_used = cow_off + 16 * n                   # lengths, slots, this step's pairs
+        b.n = len(cw)
+        if b.n:
+            b.cows_h[:b.n] = cw
+        b.meta_used = cow_off + 16 * b.n               # lengths, slots, this step's pairs
         with torch.cuda.stream(up):
-            b.meta[:meta_used].copy_(b.meta_h[:meta_used], non_blocking=True)
+            b.meta[:b.meta_used].copy_(b.meta_h[:b.meta_used], non_blocking=True)
             b.h2d.record(up)
-        comp.wait_event(b.h2d)
-        if n:
-            pa.pa_copy_blocks(loop.k_cache, loop.v_cache, b.cows[:n], stream=comp)
+        b.staged = i
+
+    def launch(i, count):
+        b = bufs[i % ring]
+        assert b.staged == i
+        # an upload that has landed needs no stream dependency
+        if not b.h2d.query():
+            comp.wait_event(b.h2d)
+        if b.n:
+            pa.pa_copy_blocks(loop.k_cache, loop.v_cache, b.cows[:b.n], stream=comp)
         if loop.fused:
             # the mapping update, the cache write and the decode, in the
             # decode's launch(es)
@@ -774,7 +787,7 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
             pa.pa_reshape_and_cache(b.k, b.v, loop.k_cache, loop.v_cache, b.slots, stream=comp)
             saved_out, loop.out = loop.out, b.out
             with torch.cuda.stream(comp):
-                loop.decode(b.q, tables_d, b.lens, int(lens_np.max()))
+                loop.decode(b.q, tables_d, b.lens, int(b.lens_h.max()))
             loop.out = saved_out
         b.done.record(comp)
         with torch.cuda.stream(down):
@@ -782,10 +795,22 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
             b.out_h.copy_(b.out, non_blocking=True)
             b.d2h.record(down)
         b.used = True
+        b.staged = -1
         if count:
-            counts["h2d"] += in_bytes + meta_used
+            counts["h2d"] += in_bytes + b.meta_used
             counts["d2h"] += b.out_h.numel() * b.out_h.element_size()
-            counts["kv"] += decode_kv_bytes(lens_np, p)
+            counts["kv"] += decode_kv_bytes(b.lens_h, p)
+
+    def run(lo, hi, count, stage_below):
+        """Launch steps lo .. hi - 1, staging each next step (below
+        stage_below) before the current one is launched."""
+        for i in range(lo, hi):
+            if bufs[i % ring].staged != i:
+                stage(i)
+            if i + 1 < stage_below:
+                stage(i + 1)
+            launch(i, count)
+            next_step[0] = i + 1
 
     def drain():
         for k in range(ring):                          # oldest first
@@ -800,32 +825,25 @@ def run_e2e(loop: DecodeLoop, steps: int, warmup: int, world: int, ring: int = 3
     # follows their kernels on the compute stream and the timed uploads wait
     # for it
     pre = min(2, warmup)
-    for i in range(warmup - pre):
-        step(i, False)
-        next_step[0] = i + 1
+    run(0, warmup - pre, False, warmup - pre)
     drain()
     torch.cuda.synchronize()
     barrier(world)
     gc.collect()
     gc.disable()
     try:
-        for i in range(warmup - pre, warmup):
-            step(i, False)
-            next_step[0] = i + 1
+        # the first timed step is staged only after t0
+        run(warmup - pre, warmup, False, warmup)
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(comp)
         up.wait_event(t0)
         down.wait_event(t0)
-        for j in range(steps):
-            step(warmup + j, True)
-            next_step[0] = warmup + j + 1
+        run(warmup, warmup + steps, True, total)
         for b in bufs:
             if b.used:
                 comp.wait_event(b.d2h)
         t1.record(comp)
-        for i in range(warmup + steps, total):
-            step(i, False)
-            next_step[0] = i + 1
+        run(warmup + steps, total, False, total)
     finally:
         gc.enable()
     drain()
