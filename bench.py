@@ -602,36 +602,38 @@ def _config_entry(loop, res, steps, peak, label, kernel):
     return e
 
 
-def run_other_configs(dev, local, peak, steps=10, warmup=3):
+def run_other_configs(dev, local, peak, steps=10, warmup=3, prefix_steps=64, prefix_warmup=8):
     """The other decode workloads, measured briefly after the headline run:
     MHA batch 64 (pa_decode_step: mapping update, append and decode in one
     launch), the long-context split at the config's 512-token partitions, and
     the prefix-sharing batch (block 16, head_dim 128) with plain decode
     (pa_decode_step) and with the cascade (pa_decode_shared_prefix_step).
     Each builds its own pool, runs ``warmup`` eager steps and ``steps``
-    device-timed steps replayed as one CUDA graph, and is freed."""
+    device-timed steps replayed as one CUDA graph, and is freed.  The prefix
+    steps take ~0.03-0.07 ms, so they run ``prefix_steps`` of them: over ten,
+    the replay's fixed start and end (~12 us) would add ~4 % to each."""
     out = []
-    extra = 2 * (steps + warmup) + 4
 
-    def run(build, label, kernel, fused=False, unique=False):
-        loop = build()
+    def run(build, label, kernel, fused=False, unique=False, n=steps, w=warmup):
+        loop = build(2 * (n + w) + 4)
         loop.fused = fused
-        res = run_device_timed(loop, steps, warmup, 1, local, unique=unique, graph=True)
-        out.append(_config_entry(loop, res, steps, peak, label, kernel))
+        res = run_device_timed(loop, n, w, 1, local, unique=unique, graph=True)
+        out.append(_config_entry(loop, res, n, peak, label, kernel))
         del loop
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
         return out[-1]
 
-    run(lambda: DecodeLoop(make_problem("mha", extra, 0), dev, "decode", 512),
+    run(lambda extra: DecodeLoop(make_problem("mha", extra, 0), dev, "decode", 512),
         "mha_decode_b64", "pa_decode_step", fused=True)
-    run(lambda: DecodeLoop(make_problem("long", extra, 0), dev, "split", 512),
+    run(lambda extra: DecodeLoop(make_problem("long", extra, 0), dev, "split", 512),
         "long_context_split_p512", "pa_decode_split")
-    plain = run(lambda: build_prefix_loop(dev, extra, "decode", 512, 16, 128),
-                "prefix_sharing_b64_bs16_d128", "pa_decode_step", fused=True, unique=True)
-    casc = run(lambda: build_prefix_loop(dev, extra, "cascade", 512, 16, 128),
+    plain = run(lambda extra: build_prefix_loop(dev, extra, "decode", 512, 16, 128),
+                "prefix_sharing_b64_bs16_d128", "pa_decode_step", fused=True, unique=True,
+                n=prefix_steps, w=prefix_warmup)
+    casc = run(lambda extra: build_prefix_loop(dev, extra, "cascade", 512, 16, 128),
                "prefix_sharing_b64_bs16_d128", "pa_decode_shared_prefix_step", fused=True,
-               unique=True)
+               unique=True, n=prefix_steps, w=prefix_warmup)
     casc["speedup_vs_pa_decode"] = round(plain["ms_per_step"] / casc["ms_per_step"], 3)
     return out
 

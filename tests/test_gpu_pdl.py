@@ -84,3 +84,47 @@ def test_pdl_option_round_trip():
     pa.pa_set_option("pdl", 0)
     assert pa.pa_get_option("pdl") == 0
     pa.pa_set_option("pdl", 1)
+
+
+def _lengths_loop(pdl: bool, problem, data, lens_seq):
+    """pa_decode after a torch kernel that rewrites context_lens, back to back
+    on one stream with no host synchronisation: the decode grid stages the
+    lengths before its dependency wait, which is correct only because a
+    caller's kernel completes before a programmatic dependent starts."""
+    pa.pa_set_option("pdl", 1 if pdl else 0)
+    try:
+        lens_d = torch.zeros_like(data["context_lens"])
+        zero = torch.zeros_like(lens_d)
+        outs = [torch.empty_like(data["q"]) for _ in lens_seq]
+        torch.cuda.synchronize()
+        for src, out in zip(lens_seq, outs):
+            torch.add(src, zero, out=lens_d)              # a kernel right before the decode
+            pa.pa_decode(out, data["q"], data["k_cache"], data["v_cache"],
+                         data["block_tables"], lens_d, problem.scale)
+        torch.cuda.synchronize()
+        return outs
+    finally:
+        pa.pa_set_option("pdl", 1)
+
+
+def test_lengths_written_by_the_previous_kernel_are_seen():
+    # 100 sequences (the longest-first search path); lengths alternate
+    # between the full lengths and halves of them, so a decode that read
+    # the previous step's lengths would differ from its own
+    problem = pa_inputs.random_small(61, num_seqs=100, max_len=700, num_heads=HQ,
+                                     num_kv_heads=HK, head_dim=D, block_size=BS, dtype="bf16")
+    data = pa_inputs.materialize(problem, "cuda")
+    full = data["context_lens"]
+    half = torch.div(full, 2, rounding_mode="floor")
+    lens_seq = [full if st % 2 == 0 else half for st in range(10)]
+    on = _lengths_loop(True, problem, data, lens_seq)
+    off = _lengths_loop(False, problem, data, lens_seq)
+    assert all(same_bits(a, b) for a, b in zip(on, off))
+    assert not same_bits(on[0], on[1])
+    cpu = {k: data[k].cpu() for k in ("q", "k_cache", "v_cache")}
+    for st in (0, 1):
+        ref = oracle.paged_decode(cpu["q"], cpu["k_cache"], cpu["v_cache"], problem.block_tables,
+                                  lens_seq[st].cpu().numpy(), problem.scale)
+        assert_close(on[st], ref)
+        assert_close(on[st + 8], ref)
+    device_clean()
