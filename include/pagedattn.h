@@ -80,10 +80,17 @@ typedef enum pa_option {
     PA_OPT_VALIDATE = 0,         /* 0/1: host-side index validation before launch */
     PA_OPT_DECODE_SPLIT_CTAS = 1, /* pa_decode CTAs per (sequence, kv head): 0 = auto, 1, 2, 4, 8 */
     PA_OPT_PDL = 2,               /* 0/1 (default 1, or PA_PDL in the environment): launch with
-                                     programmatic dependent launch.  Every kernel still waits
-                                     for the grid before it on the stream to complete before
-                                     touching memory; only the launch and the CTA placement
-                                     overlap that grid's tail */
+                                     programmatic dependent launch.  A kernel may start during
+                                     the tail of the grid before it on the stream, and waits
+                                     for that grid to complete before it reads anything that
+                                     grid may write.  Before that wait, pa_decode's grid (and
+                                     pa_decode_append's, pa_decode_step's) reads only
+                                     context_lens, which no kernel of this library writes: a
+                                     caller's kernel that writes it must not release its
+                                     dependents early (griddepcontrol.launch_dependents), or
+                                     this option must be 0.  The shared-prefix decode's
+                                     own-token pass streams the cache behind the shared pass,
+                                     which has waited for the grid before it */
     PA_OPT_WAIT_LIMIT_US = 3,     /* upper bound, in microseconds, on every pipeline wait inside
                                      the decode kernels (default 2000000 = 2 s; 100 .. 10000000).
                                      A wait that runs out sets PA_DEVERR_WAIT_TIMEOUT; the warp
