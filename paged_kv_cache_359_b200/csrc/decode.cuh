@@ -1149,13 +1149,6 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                     }
                 }
                 __syncthreads();
-                if constexpr (MODE == Mode::Decode) {
-                    if (!waited) {                          // first item: see the kernel's top
-                        pdl_wait();
-                        pdl_launch_dependents();
-                        waited = true;
-                    }
-                }
                 seq = pick[0];
                 kvh = item % Hk;
                 int tok0;                                   // whole 16-token units
@@ -1165,6 +1158,34 @@ __global__ void __launch_bounds__(Layout<U, MODE == Mode::Own && own_half_width<
                 } else {
                     L = S <= MAX_SORT && !a.group_starts ? pick[1] : clamp_len(seq);
                     tok0 = cmin(shared_prefix_of(a, seq), L);
+                }
+                if constexpr (MODE == Mode::Decode) {
+                    if (!waited) {                          // first item: see the kernel's top
+                        // While the previous grid finishes, bring the tiles of
+                        // each warp's first DEPTH units into L2.  The block ids
+                        // are read around L1 (the grid before may still rewrite
+                        // the table; the loads after the wait read it again), and
+                        // a prefetch changes no data, so a stale id costs only
+                        // bandwidth; ids outside the pool are skipped.
+                        const int k = lane;                 // unit k of this warp
+                        const int uu = tok0 / R + warp + NW * k;
+                        if (k < DEPTH && uu * R < L) {
+                            const int32_t* table = a.block_tables + (size_t)seq * a.max_blocks;
+                            const int t0 = uu * R;
+                            const int id = __ldcg(table + t0 / U::BS);
+                            if (id >= 0 && id < a.num_blocks) {
+                                const int row0 = U::BOX_ROWS < R ? 0 : t0 % U::BS;
+#pragma unroll
+                                for (int b = 0; b < U::BOXES; ++b) {
+                                    tma_prefetch_l2_4d(&tm_k, b * U::BOX_INNER, kvh, row0, id);
+                                    tma_prefetch_l2_4d(&tm_v, b * U::BOX_INNER, kvh, row0, id);
+                                }
+                            }
+                        }
+                        pdl_wait();
+                        pdl_launch_dependents();
+                        waited = true;
+                    }
                 }
                 // the new row's loads go out here and are waited on (written,
                 // fenced, barrier) only after the first window of block ids has
