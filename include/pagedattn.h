@@ -84,11 +84,13 @@ typedef enum pa_option {
                                      the tail of the grid before it on the stream, and waits
                                      for that grid to complete before it reads anything that
                                      grid may write.  Before that wait, pa_decode's grid (and
-                                     pa_decode_append's, pa_decode_step's) reads only
-                                     context_lens, which no kernel of this library writes: a
-                                     caller's kernel that writes it must not release its
-                                     dependents early (griddepcontrol.launch_dependents), or
-                                     this option must be 0.  The shared-prefix decode's
+                                     pa_decode_append's, pa_decode_step's) reads context_lens,
+                                     which no kernel of this library writes: a caller's kernel
+                                     that writes it must not release its dependents early
+                                     (griddepcontrol.launch_dependents), or this option must
+                                     be 0.  It also reads a few block-table entries there, but
+                                     only to prefetch their tiles into L2; the entries it
+                                     decodes with are read after the wait.  The shared-prefix decode's
                                      own-token pass streams the cache behind the shared pass,
                                      which has waited for the grid before it */
     PA_OPT_WAIT_LIMIT_US = 3,     /* upper bound, in microseconds, on every pipeline wait inside
