@@ -33,7 +33,7 @@ Reported line (rank 0):
              of three buffer sets, overlapping the neighbouring steps'
              kernels as a serving loop would.
   other_configs  (default gqa run, 1 GPU) short device-timed runs of the
-             mha, long-context split and prefix-sharing workloads, each with
+             mha, gqa at head_dim 64, long-context split and prefix-sharing workloads, each with
              its kernel's roofline fraction.
   roofline   the decode kernel: algorithmic bytes per launch / mean launch
              time (CUDA events on the launching stream) vs measured HBM GB/s.
@@ -605,7 +605,8 @@ def _config_entry(loop, res, steps, peak, label, kernel):
 def run_other_configs(dev, local, peak, steps=10, warmup=3, prefix_steps=64, prefix_warmup=8):
     """The other decode workloads, measured briefly after the headline run:
     MHA batch 64 (pa_decode_step: mapping update, append and decode in one
-    launch), the long-context split at the config's 512-token partitions, and
+    launch), the headline's GQA batch at head_dim 64 (pa_decode_step), the
+    long-context split at the config's 512-token partitions, and
     the prefix-sharing batch (block 16, head_dim 128) with plain decode
     (pa_decode_step) and with the cascade (pa_decode_shared_prefix_step).
     Each builds its own pool, runs ``warmup`` eager steps and ``steps``
@@ -626,6 +627,8 @@ def run_other_configs(dev, local, peak, steps=10, warmup=3, prefix_steps=64, pre
 
     run(lambda extra: DecodeLoop(make_problem("mha", extra, 0), dev, "decode", 512),
         "mha_decode_b64", "pa_decode_step", fused=True)
+    run(lambda extra: DecodeLoop(make_problem("gqa", extra, 0, None, 64), dev, "decode", 512),
+        "gqa_decode_b256_d64", "pa_decode_step", fused=True)
     run(lambda extra: DecodeLoop(make_problem("long", extra, 0), dev, "split", 512),
         "long_context_split_p512", "pa_decode_split")
     plain = run(lambda extra: build_prefix_loop(dev, extra, "decode", 512, 16, 128),
